@@ -1,0 +1,134 @@
+"""Seeded synthetic inputs shaped like the MoE checkpoints the quantizer
+converts.  Random numbers only: nothing here quantizes, scales or rounds
+beyond the single cast of each drawn value to bf16.
+
+The real checkpoints (Qwen3.8-Flash-Next bf16 experts) are not available,
+so these stand in for them, with the shapes the model cards give:
+
+* routed experts stored stacked, fused gate_up ``[E, 2I, H]`` and down
+  ``[E, H, I]`` (dabsLabs/Qwen3.8-Flash-Next-NVFP4, "What makes this build
+  different": ``[512, out, in]``, fused gate_up; the census there is 48
+  layers x 512 experts x 3 projections);
+* the shared expert, gate/up ``[2560, 2048]`` and down ``[2048, 1280]``,
+  with an MTP-style copy whose widening 640 -> 1280 is zero rows in gate
+  and up and zero columns in down (azampatti/Qwen3.8-Flash-Next-FP4-Local-AZ,
+  "The shared expert");
+* activation token tiles ``[T, 2048]`` (MJPansa/Qwen3.8-Flash-Next-MXFP4-FP8-R12,
+  "Quantization format": activations dynamically quantized at run time).
+
+Every generator takes a seed and a torch device and returns bf16 tensors.
+A given (seed, device type) always yields the same bits.
+"""
+import math
+
+import torch
+
+# Four fixed outlier channels of the activation tiles (a fixed reading:
+# the workload asks for "4 fixed outlier channels" without naming them).
+ACT_OUTLIER_CHANNELS = (101, 717, 1333, 1949)
+
+
+def _gen(seed, device):
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    return g
+
+
+def _normal_bf16(shape, std, gen, device):
+    return (torch.randn(shape, generator=gen, device=device, dtype=torch.float32) * std)
+
+
+def tiny_moe_layer(seed=0, device="cpu", experts=8, hidden=256, inter=128):
+    """Tiny routed-expert layer: gate_up [E, 2I, H], down [E, H, I] with
+    2I = hidden here (8 x 256 x 256 and 8 x 256 x 128 by default).
+    Values N(0, 0.02); 0.1 % of entries (Bernoulli per element) x 10."""
+    g = _gen(seed, device)
+    out = []
+    for shape in ((experts, 2 * inter, hidden), (experts, hidden, inter)):
+        w = _normal_bf16(shape, 0.02, g, device)
+        mask = torch.rand(shape, generator=g, device=device) < 0.001
+        w = torch.where(mask, w * 10.0, w)
+        out.append(w.to(torch.bfloat16))
+    return out[0], out[1]
+
+
+def full_moe_layer(seed=0, device="cuda", experts=512, hidden=2048, inter=768,
+                   chunk=64):
+    """Full-size routed-expert layer: gate_up [E, 2I, H], down [E, H, I]
+    (512 x 1536 x 2048 and 512 x 2048 x 768 by default, 2,415,919,104
+    values).  Per expert sigma_e = exp(U(ln 0.005, ln 0.05)), shared by
+    that expert's gate_up and down; values N(0, sigma_e); 0.05 % of entries
+    replaced by sign(x) * 8 sigma_e."""
+    g = _gen(seed, device)
+    sig = torch.exp(torch.empty(experts, device=device).uniform_(
+        math.log(0.005), math.log(0.05), generator=g))
+    gate_up = torch.empty((experts, 2 * inter, hidden), dtype=torch.bfloat16, device=device)
+    down = torch.empty((experts, hidden, inter), dtype=torch.bfloat16, device=device)
+    for t in (gate_up, down):
+        for e0 in range(0, experts, chunk):
+            e1 = min(experts, e0 + chunk)
+            s = sig[e0:e1].view(-1, 1, 1)
+            w = torch.randn((e1 - e0,) + tuple(t.shape[1:]), generator=g, device=device) * s
+            mask = torch.rand(w.shape, generator=g, device=device) < 0.0005
+            w = torch.where(mask, torch.sign(w) * 8.0 * s, w)
+            t[e0:e1] = w.to(torch.bfloat16)
+            del w, mask
+    return gate_up, down, sig
+
+
+def shared_expert_layer(seed=0, device="cpu", inter=1280, hidden=2048,
+                        pad_from=640, padded=False, pad_up=True):
+    """One layer's shared expert: fused gate/up [2*inter, hidden] (gate rows
+    first) and down [hidden, inter], values N(0, 0.02).  ``padded`` gives the
+    MTP-style copy: gate rows [pad_from, inter) zero, up rows likewise when
+    ``pad_up`` (fused rows [inter + pad_from, 2*inter)), and down columns
+    [pad_from, inter) zero."""
+    g = _gen(seed, device)
+    gu = _normal_bf16((2 * inter, hidden), 0.02, g, device)
+    dn = _normal_bf16((hidden, inter), 0.02, g, device)
+    if padded:
+        gu[pad_from:inter] = 0
+        if pad_up:
+            gu[inter + pad_from:] = 0
+        dn[:, pad_from:] = 0
+    return gu.to(torch.bfloat16), dn.to(torch.bfloat16)
+
+
+def student_t_mix_layer(seed=0, device="cuda", experts=512, hidden=2048, inter=768,
+                        p_tail=0.01, chunk=64):
+    """Mixed-format layer input: gate_up [E, 2I, H], down [E, H, I]; values
+    N(0, 0.02), except a fraction ``p_tail`` (a reading: the workload names a
+    Student-t(4) tail mix without its weight) drawn from 0.02 * t_4 with
+    t_4 = N / sqrt(chi2_4 / 4)."""
+    g = _gen(seed, device)
+    out = []
+    for shape in ((experts, 2 * inter, hidden), (experts, hidden, inter)):
+        t = torch.empty(shape, dtype=torch.bfloat16, device=device)
+        for e0 in range(0, experts, chunk):
+            e1 = min(experts, e0 + chunk)
+            sub = (e1 - e0,) + shape[1:]
+            w = torch.randn(sub, generator=g, device=device) * 0.02
+            z = torch.randn(sub, generator=g, device=device)
+            chi2 = torch.randn(sub + (4,), generator=g, device=device).square().sum(-1)
+            tail = 0.02 * z / torch.sqrt(chi2 / 4.0)
+            mask = torch.rand(sub, generator=g, device=device) < p_tail
+            t[e0:e1] = torch.where(mask, tail, w).to(torch.bfloat16)
+            del w, z, chi2, tail, mask
+        out.append(t)
+    return out[0], out[1]
+
+
+def activation_tile(T, seed=0, device="cpu", hidden=2048):
+    """Token tile [T, hidden], values N(0, 1) with the four fixed outlier
+    channels scaled x 30."""
+    g = _gen(seed, device)
+    a = torch.randn((T, hidden), generator=g, device=device)
+    for c in ACT_OUTLIER_CHANNELS:
+        if c < hidden:
+            a[:, c] *= 30.0
+    return a.to(torch.bfloat16)
+
+
+def bf16_bits(t):
+    """bf16 tensor -> numpy uint16 array of its bit patterns (host copy)."""
+    return t.detach().contiguous().view(torch.int16).cpu().numpy().view("uint16")

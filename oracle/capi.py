@@ -1,0 +1,160 @@
+"""ctypes front end of the C oracle (test infrastructure only).
+
+Numpy arrays in, numpy arrays out.  Inputs are bf16 bit patterns held in
+``uint16`` arrays, the same bits the CUDA path reads.
+"""
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "mxq_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+# No FMA contraction, no fast-math, denormals kept: every float operation
+# in the oracle is one correctly rounded IEEE operation.
+CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
+          "-fPIC", "-shared", "-Wall", "-Wextra"]
+
+GLOBAL_DIVISOR = 2688.0  # 6 * 448: weight_scale_2 and input_scale
+
+
+def build(force=False):
+    """Compile the oracle into oracle/liboracle.so (gcc)."""
+    if (not force and os.path.exists(_LIB)
+            and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC)):
+        return _LIB
+    tmp = _LIB + ".tmp%d" % os.getpid()
+    subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"])
+    os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB)
+        d, u, i, i64, vp = (ctypes.c_double, ctypes.c_uint, ctypes.c_int,
+                            ctypes.c_int64, ctypes.c_void_p)
+        L.oracle_e2m1_value.restype = d
+        L.oracle_e2m1_value.argtypes = [u]
+        L.oracle_e4m3_value.restype = d
+        L.oracle_e4m3_value.argtypes = [u]
+        L.oracle_ue8m0_value.restype = d
+        L.oracle_ue8m0_value.argtypes = [u]
+        L.oracle_e2m1_encode.restype = u
+        L.oracle_e2m1_encode.argtypes = [d]
+        L.oracle_e4m3_encode.restype = u
+        L.oracle_e4m3_encode.argtypes = [d]
+        L.oracle_mx_exponent.restype = i
+        L.oracle_mx_exponent.argtypes = [d, d]
+        L.oracle_quantize_nvfp4.restype = i
+        L.oracle_quantize_nvfp4.argtypes = [vp, i64, i64, i64, i, d, vp, vp, vp, vp]
+        L.oracle_quantize_mx.restype = i
+        L.oracle_quantize_mx.argtypes = [vp, i64, i64, i, vp, vp]
+        L.oracle_dequant_relerr.restype = i
+        L.oracle_dequant_relerr.argtypes = [vp, vp, vp, vp, i, i64, i64, i64, i64, vp, vp]
+        _lib = L
+    return _lib
+
+
+def _ptr(a):
+    return a.ctypes.data_as(ctypes.c_void_p) if a is not None else None
+
+
+def e2m1_value(code):
+    return lib().oracle_e2m1_value(int(code))
+
+
+def e4m3_value(code):
+    return lib().oracle_e4m3_value(int(code))
+
+
+def ue8m0_value(code):
+    return lib().oracle_ue8m0_value(int(code))
+
+
+def e2m1_encode(v):
+    return lib().oracle_e2m1_encode(float(v))
+
+
+def e4m3_encode(v):
+    return lib().oracle_e4m3_encode(float(v))
+
+
+def mx_exponent(amax, qmax):
+    return lib().oracle_mx_exponent(float(amax), float(qmax))
+
+
+def _as_bits(x):
+    x = np.ascontiguousarray(x)
+    if x.dtype != np.uint16:
+        raise TypeError("oracle inputs are bf16 bit patterns (uint16)")
+    return x
+
+
+def quantize_nvfp4(x_bits, mode=1, global_div=GLOBAL_DIVISOR):
+    """x_bits: uint16 [G, R, C].  Returns codes [G,R,C/2], scales [G,R,C/16],
+    s2 [G] float32, m4 [G, R*C/16] uint8 (1 = the M=4 plan won)."""
+    x = _as_bits(x_bits)
+    G, R, C = x.shape
+    codes = np.zeros((G, R, C // 2), np.uint8)
+    scales = np.zeros((G, R, C // 16), np.uint8)
+    s2 = np.zeros(G, np.float32)
+    m4 = np.zeros((G, R * C // 16), np.uint8)
+    rc = lib().oracle_quantize_nvfp4(_ptr(x), G, R, C, int(mode), float(global_div),
+                                     _ptr(codes), _ptr(scales), _ptr(s2), _ptr(m4))
+    if rc != 0:
+        raise RuntimeError("oracle_quantize_nvfp4 failed: %d" % rc)
+    return codes, scales, s2, m4
+
+
+def quantize_mx(x_bits, fmt):
+    """fmt: 'mxfp4' or 'mxfp8'.  x_bits uint16 [R, C] (or any shape whose
+    last dim is C).  Returns codes, scales."""
+    x = _as_bits(x_bits)
+    C = x.shape[-1]
+    R = x.size // C if C else 0
+    f = {"mxfp4": 1, "mxfp8": 2}[fmt]
+    codes = np.zeros(x.shape[:-1] + ((C // 2) if f == 1 else C,), np.uint8)
+    scales = np.zeros(x.shape[:-1] + (C // 32,), np.uint8)
+    rc = lib().oracle_quantize_mx(_ptr(x), R, C, f, _ptr(codes), _ptr(scales))
+    if rc != 0:
+        raise RuntimeError("oracle_quantize_mx failed: %d" % rc)
+    return codes, scales
+
+
+def dequant_relerr(x_bits, codes, scales, s2, fmt, n_tensors, rows, cols,
+                   tensors_per_scale=1):
+    """Per-tensor (sum_sq_err, sum_sq_ref) as float64 arrays [n_tensors]."""
+    x = _as_bits(x_bits)
+    f = {"nvfp4": 0, "mxfp4": 1, "mxfp8": 2}[fmt]
+    codes = np.ascontiguousarray(codes, np.uint8)
+    scales = np.ascontiguousarray(scales, np.uint8)
+    s2a = np.ascontiguousarray(s2, np.float32) if s2 is not None else None
+    err = np.zeros(n_tensors, np.float64)
+    ref = np.zeros(n_tensors, np.float64)
+    rc = lib().oracle_dequant_relerr(_ptr(x), _ptr(codes), _ptr(scales), _ptr(s2a), f,
+                                     n_tensors, rows, cols, tensors_per_scale,
+                                     _ptr(err), _ptr(ref))
+    if rc != 0:
+        raise RuntimeError("oracle_dequant_relerr failed: %d" % rc)
+    return err, ref
+
+
+def relerr_from_sums(err, ref):
+    """rel = sqrt(sum_sq_err) / sqrt(sum_sq_ref); 0 for an all-zero tensor
+    reproduced exactly."""
+    err = np.asarray(err, np.float64)
+    ref = np.asarray(ref, np.float64)
+    out = np.zeros_like(err)
+    nz = ref > 0
+    out[nz] = np.sqrt(err[nz]) / np.sqrt(ref[nz])
+    out[(~nz) & (err > 0)] = np.inf
+    return out

@@ -1,0 +1,384 @@
+/*
+ * mxq_oracle.c -- plain, slow, scalar CPU oracle of the block-scaled
+ * microscaling quantizer (NVFP4 4/6-optimal, MXFP4, MXFP8) and its
+ * dequantize + relative-error verifier.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the checker, not the product:
+ * only the test suite, the package smoke check and the benchmark's CPU
+ * baseline leg load it.  It shares no code, header, table or helper with
+ * the CUDA library, and the CUDA library never calls it.
+ *
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -fPIC -shared
+ * (no FMA contraction, no flush-to-zero: every float operation below is
+ * one IEEE-754 binary32 or binary64 operation, rounded to nearest even).
+ *
+ * Sources (model-card pages; section in quotes):
+ *  [P1] josch15366/Qwen3.8-Flash-Next-NVFP4-LocalHessian-Experts,
+ *       introduction (input_scale = amax/2688; gate and up share one
+ *       weight_scale_2) and "What is different about it" (one
+ *       weight_scale_2 per expert).
+ *  [P2] azampatti/Qwen3.8-Flash-Next-FP4-Local-AZ, "The shared expert"
+ *       (MXFP8: e4m3 values, one power-of-two scale per 32 weights,
+ *       e = ceil(log2(amax / 448))) and the zero-padded 640 -> 1280
+ *       shared expert (silu(0) * 0 = 0).
+ *  [P3] dabsLabs/Qwen3.8-Flash-Next-NVFP4, "What makes this build
+ *       different" (per 16-element block, choose between the amax/6 plan
+ *       and the four-over-six plan by exact post-rounding squared error;
+ *       never worse than plain RTN) and the metric table (relative error
+ *       of quantized experts against the bf16 source).
+ *  [P4] MJPansa/Qwen3.8-Flash-Next-MXFP4-FP8-R12, "Quantization format"
+ *       (MXFP4 E2M1 weights with UE8M0 microscales; activations
+ *       dynamically quantized to MXFP8).
+ *
+ * Readings taken where the pages are silent are stated at each function.
+ * Every function here is pinned by tests that do not use this file's
+ * arithmetic (see tests/test_oracle_*.py).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------ */
+/* Number formats.  The pages name E2M1, E4M3 and UE8M0 without giving  */
+/* bit layouts; the reading is the OCP microscaling / OCP FP8 "fn"       */
+/* definitions: E2M1 = sign, 2 exponent bits (bias 1), 1 mantissa bit;   */
+/* E4M3 = sign, 4 exponent bits (bias 7), 3 mantissa bits, no infinity,  */
+/* S.1111.111 is NaN, largest finite 448; UE8M0 byte b = 2^(b-127),      */
+/* 0xFF is NaN.                                                          */
+/* ------------------------------------------------------------------ */
+
+double oracle_e2m1_value(unsigned code)
+{
+    unsigned s = (code >> 3) & 1u, e = (code >> 1) & 3u, m = code & 1u;
+    double mag;
+    if (e == 0)
+        mag = 0.5 * (double)m;                      /* subnormal: m * 2^-1 */
+    else
+        mag = ldexp(1.0 + 0.5 * (double)m, (int)e - 1);
+    return s ? -mag : mag;
+}
+
+double oracle_e4m3_value(unsigned code)
+{
+    unsigned s = (code >> 7) & 1u, e = (code >> 3) & 15u, m = code & 7u;
+    double mag;
+    if (e == 15 && m == 7)
+        return NAN;
+    if (e == 0)
+        mag = ldexp((double)m / 8.0, -6);           /* subnormal: m/8 * 2^-6 */
+    else
+        mag = ldexp(1.0 + (double)m / 8.0, (int)e - 7);
+    return s ? -mag : mag;
+}
+
+double oracle_ue8m0_value(unsigned code)
+{
+    if ((code & 0xFFu) == 0xFFu)
+        return NAN;
+    return ldexp(1.0, (int)(code & 0xFFu) - 127);
+}
+
+/* Round a finite real value to the nearest representable magnitude of a
+ * format, ties to the even code (the code whose last mantissa bit is 0),
+ * magnitudes beyond the largest finite one saturate to it ("satfinite"),
+ * and the sign bit is copied from the input, so a negative value that
+ * rounds to zero gives negative zero.  This is round-to-nearest-even
+ * stated as a search over the format's codes: it needs no bit tricks. */
+static unsigned nearest_code(double v, unsigned n_mag_codes,
+                             double (*value_of)(unsigned), unsigned sign_bit,
+                             double max_finite, unsigned max_code)
+{
+    double a = fabs(v);
+    unsigned best = 0;
+    if (a >= max_finite) {
+        best = max_code;
+    } else {
+        double best_dist = INFINITY;
+        for (unsigned c = 0; c < n_mag_codes; ++c) {
+            double dist = fabs(a - value_of(c));   /* exact: both are short dyadics */
+            if (dist < best_dist || (dist == best_dist && (c & 1u) == 0u)) {
+                best = c;
+                best_dist = dist;
+            }
+        }
+    }
+    return signbit(v) ? (best | sign_bit) : best;
+}
+
+/* E2M1 encode of a real value (round to nearest even code, satfinite).
+ * Non-finite input returns 0xFF, which is not a valid code. */
+unsigned oracle_e2m1_encode(double v)
+{
+    if (!isfinite(v))
+        return 0xFFu;
+    return nearest_code(v, 8u, oracle_e2m1_value, 0x8u, 6.0, 0x7u);
+}
+
+/* E4M3 encode of a real value (round to nearest even code, satfinite to
+ * +-448: the NaN code is never produced).  Non-finite input -> 0xFFFF. */
+unsigned oracle_e4m3_encode(double v)
+{
+    if (!isfinite(v))
+        return 0xFFFFu;
+    return nearest_code(v, 127u, oracle_e4m3_value, 0x80u, 448.0, 0x7Eu);
+}
+
+/* MX shared exponent [P2 "The shared expert"; P4 "Quantization format"]:
+ * e = ceil(log2(amax / qmax)), read as the smallest integer e with
+ * amax <= qmax * 2^e, so no element of the block needs saturation.
+ * Clamped to the UE8M0 range [-127, 127]; amax = 0 gives -127 (byte 0). */
+int oracle_mx_exponent(double amax, double qmax)
+{
+    int e = -127;
+    if (!(amax > 0.0))
+        return -127;
+    while (e < 127 && amax > ldexp(qmax, e))
+        ++e;
+    return e;
+}
+
+static float bf16_to_float(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* ------------------------------------------------------------------ */
+/* Exactness guards.  The 4/6 decision below is evaluated with binary64 */
+/* operations that are exact for every block the method can produce;    */
+/* each step is checked and a violated premise is reported, never       */
+/* silently rounded.                                                     */
+/* ------------------------------------------------------------------ */
+static double exact_mul(double a, double b, int *ok)
+{
+    double p = a * b;
+    if (fma(a, b, -p) != 0.0)
+        *ok = 0;
+    return p;
+}
+
+static double exact_add(double a, double b, int *ok)
+{
+    double s = a + b;
+    double bb = s - a;
+    double err = (a - (s - bb)) + (b - bb);        /* Knuth two-sum */
+    if (err != 0.0)
+        *ok = 0;
+    return s;
+}
+
+/* One NVFP4 plan for one 16-element block [P3 "What makes this build
+ * different"; P1 introduction].
+ *   t   = RN32(RN32(amax_b / M) / s2)             block scale in s2 units
+ *   S   = E4M3(t), D its value                    stored weight_scale byte
+ *   d   = RN32(D * s2)                            fp32 effective block scale
+ *   c_i = E2M1(RN32(x_i / d))                     stored value codes
+ * Reading: D = 0, s2 = 0 or d = 0 (underflow) give all-zero codes 0x0.
+ * Returns, through G, the exact value of (SSE_M - sum x_i^2) / s2 where
+ * SSE_M = sum_i (x_i - q_i * D * s2)^2 is the exact squared error of the
+ * stored reconstruction q_i * D * s2 (q_i = value of c_i).  Expanding the
+ * square, SSE_M - sum x^2 = s2 * D * (D * s2 * B - 2 * A) with
+ * A = sum x_i q_i and B = sum q_i^2, so G = D * (D*s2*B - 2A).
+ * Return 0 on success, -2 if an exactness premise failed. */
+static int nvfp4_plan(const float x[16], float amax_b, float s2, float M,
+                      unsigned *scale_code, uint8_t codes[16], double *G)
+{
+    int ok = 1;
+    unsigned sc = 0;
+    double D = 0.0;
+    float d = 0.0f;
+
+    if (s2 > 0.0f) {
+        float t = amax_b / M;
+        t = t / s2;
+        sc = oracle_e4m3_encode((double)t);
+        D = oracle_e4m3_value(sc);
+        d = (float)D * s2;
+    }
+    *scale_code = sc;
+    if (D == 0.0 || d == 0.0f) {
+        for (int i = 0; i < 16; ++i)
+            codes[i] = 0;
+        *G = 0.0;
+        return 0;
+    }
+    double A = 0.0, B = 0.0;
+    for (int i = 0; i < 16; ++i) {
+        float y = x[i] / d;
+        unsigned c = oracle_e2m1_encode((double)y);
+        codes[i] = (uint8_t)c;
+        double q = oracle_e2m1_value(c);
+        A = exact_add(A, exact_mul((double)x[i], q, &ok), &ok);
+        B = exact_add(B, exact_mul(q, q, &ok), &ok);
+    }
+    double dS = exact_mul(D, (double)s2, &ok);
+    double P = exact_add(exact_mul(dS, B, &ok), -2.0 * A, &ok);
+    *G = exact_mul(D, P, &ok);
+    return ok ? 0 : -2;
+}
+
+/* NVFP4 quantization of a stack of groups [P1 introduction; P3 "What
+ * makes this build different"].
+ *   x            bf16 bits, [n_groups, rows, cols] row-major
+ *   global_div   2688 = 6 * 448 (weight_scale_2 and input_scale); tests
+ *                pass other values only to plant the historical bug
+ *   mode         0 = plain amax/6 (RTN), 1 = 4/6-optimal
+ *   codes        [n_groups, rows, cols/2]: element 2j in the low nibble,
+ *                element 2j+1 in the high nibble
+ *   scales       [n_groups, rows, cols/16] E4M3 bytes
+ *   s2_out       [n_groups] fp32 global scale RN32(amax_g / global_div)
+ *   m4           nullable, one byte per block: 1 if the M=4 plan won
+ * Group = one expert's fused gate_up slab (gate and up share one
+ * weight_scale_2), or one down slab, or one activation tile.
+ * The M=4 plan wins only when its exact squared error is strictly lower;
+ * ties keep the amax/6 plan, so the result equals plain RTN unless it is
+ * strictly better.  Returns 0, -1 on bad shape, -2 on a failed
+ * exactness premise, -3 on non-finite input. */
+int oracle_quantize_nvfp4(const uint16_t *x, int64_t n_groups, int64_t rows,
+                          int64_t cols, int mode, double global_div,
+                          uint8_t *codes, uint8_t *scales, float *s2_out,
+                          uint8_t *m4)
+{
+    if (n_groups < 0 || rows < 0 || cols < 0 || cols % 16 != 0)
+        return -1;
+    const int64_t gsize = rows * cols;
+    const int64_t nblk = gsize / 16;
+    int rc = 0;
+    for (int64_t g = 0; g < n_groups; ++g) {
+        const uint16_t *xg = x + g * gsize;
+        float amax_g = 0.0f;
+        for (int64_t i = 0; i < gsize; ++i) {
+            float v = fabsf(bf16_to_float(xg[i]));
+            if (!isfinite(v))
+                return -3;
+            if (v > amax_g)
+                amax_g = v;
+        }
+        float s2 = amax_g / (float)global_div;
+        s2_out[g] = s2;
+        for (int64_t b = 0; b < nblk; ++b) {
+            float xb[16];
+            float amax_b = 0.0f;
+            for (int i = 0; i < 16; ++i) {
+                xb[i] = bf16_to_float(xg[b * 16 + i]);
+                if (fabsf(xb[i]) > amax_b)
+                    amax_b = fabsf(xb[i]);
+            }
+            unsigned sc6, sc4 = 0;
+            uint8_t c6[16], c4[16];
+            double G6, G4 = 0.0;
+            int r = nvfp4_plan(xb, amax_b, s2, 6.0f, &sc6, c6, &G6);
+            if (r)
+                rc = r;
+            int use4 = 0;
+            if (mode == 1) {
+                r = nvfp4_plan(xb, amax_b, s2, 4.0f, &sc4, c4, &G4);
+                if (r)
+                    rc = r;
+                use4 = (G4 < G6);
+            }
+            const uint8_t *c = use4 ? c4 : c6;
+            int64_t gb = g * nblk + b;
+            for (int j = 0; j < 8; ++j)
+                codes[gb * 8 + j] = (uint8_t)((c[2 * j] & 0xF) | ((c[2 * j + 1] & 0xF) << 4));
+            scales[gb] = (uint8_t)(use4 ? sc4 : sc6);
+            if (m4)
+                m4[gb] = (uint8_t)use4;
+        }
+    }
+    return rc;
+}
+
+/* MX quantization, one UE8M0 scale per 32 consecutive elements of a row
+ * [P2 "The shared expert"; P4 "Quantization format"].
+ *   fmt 1 = MXFP4 (E2M1 values, qmax 6, codes [rows, cols/2] nibbles,
+ *           element 2j low), fmt 2 = MXFP8 (E4M3 values, qmax 448, codes
+ *           [rows, cols]).  scales [rows, cols/32] = e + 127.
+ * Value code = FMT(x * 2^-e), rounded to nearest even, satfinite (no
+ * element exceeds qmax by the choice of e).  Returns 0, -1 bad shape,
+ * -3 non-finite input. */
+int oracle_quantize_mx(const uint16_t *x, int64_t rows, int64_t cols, int fmt,
+                       uint8_t *codes, uint8_t *scales)
+{
+    if (rows < 0 || cols < 0 || cols % 32 != 0 || (fmt != 1 && fmt != 2))
+        return -1;
+    const double qmax = (fmt == 1) ? 6.0 : 448.0;
+    const int64_t nblk = rows * cols / 32;
+    for (int64_t b = 0; b < nblk; ++b) {
+        double v[32];
+        double amax = 0.0;
+        for (int i = 0; i < 32; ++i) {
+            v[i] = (double)bf16_to_float(x[b * 32 + i]);
+            if (!isfinite(v[i]))
+                return -3;
+            if (fabs(v[i]) > amax)
+                amax = fabs(v[i]);
+        }
+        int e = oracle_mx_exponent(amax, qmax);
+        scales[b] = (uint8_t)(e + 127);
+        for (int i = 0; i < 32; ++i) {
+            double y = ldexp(v[i], -e);                 /* exact */
+            if (fmt == 1) {
+                unsigned c = oracle_e2m1_encode(y) & 0xFu;
+                if (i & 1)
+                    codes[b * 16 + i / 2] |= (uint8_t)(c << 4);
+                else
+                    codes[b * 16 + i / 2] = (uint8_t)c;
+            } else {
+                codes[b * 32 + i] = (uint8_t)oracle_e4m3_encode(y);
+            }
+        }
+    }
+    return 0;
+}
+
+/* Dequantize and measure the relative error of every unstacked tensor
+ * [P3 metric table: relative error of quantized experts vs the bf16
+ * source; P2 "The shared expert": error against the bf16 master].
+ *   tensors t = 0..n_tensors-1, each [rows, cols], stored back to back;
+ *   NVFP4 (fmt 0): deq = q * D * s2[t / tensors_per_scale] (so the gate
+ *   and up halves of a fused slab read the same weight_scale_2);
+ *   MXFP4 / MXFP8: deq = q * 2^(b - 127).
+ * sum_sq_err[t] = sum (x - deq)^2, sum_sq_ref[t] = sum x^2, both as
+ * binary64 sums in element order.  Returns 0 or -1. */
+int oracle_dequant_relerr(const uint16_t *x, const uint8_t *codes,
+                          const uint8_t *scales, const float *s2, int fmt,
+                          int64_t n_tensors, int64_t rows, int64_t cols,
+                          int64_t tensors_per_scale, double *sum_sq_err,
+                          double *sum_sq_ref)
+{
+    const int blk = (fmt == 0) ? 16 : 32;
+    if (n_tensors < 0 || rows < 0 || cols < 0 || cols % blk != 0 ||
+        fmt < 0 || fmt > 2 || (fmt == 0 && tensors_per_scale < 1))
+        return -1;
+    const int64_t tsize = rows * cols;
+    for (int64_t t = 0; t < n_tensors; ++t) {
+        double err = 0.0, ref = 0.0;
+        for (int64_t i = 0; i < tsize; ++i) {
+            int64_t gi = t * tsize + i;
+            double xv = (double)bf16_to_float(x[gi]);
+            double deq;
+            if (fmt == 2) {
+                deq = oracle_e4m3_value(codes[gi]) *
+                      oracle_ue8m0_value(scales[gi / 32]);
+            } else {
+                uint8_t byte = codes[gi / 2];
+                unsigned c = (gi & 1) ? (byte >> 4) : (byte & 0xFu);
+                double q = oracle_e2m1_value(c);
+                if (fmt == 1)
+                    deq = q * oracle_ue8m0_value(scales[gi / 32]);
+                else
+                    deq = q * oracle_e4m3_value(scales[gi / 16]) *
+                          (double)s2[t / tensors_per_scale];
+            }
+            double e = xv - deq;
+            err += e * e;
+            ref += xv * xv;
+        }
+        sum_sq_err[t] = err;
+        sum_sq_ref[t] = ref;
+    }
+    return 0;
+}
