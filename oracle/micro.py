@@ -104,11 +104,11 @@ def plan_with_scale_code(x, s2, sc):
 
 
 def plan(x, s2, M):
-    """One plan: scale code from t = RN32(RN32(amax_b / M) / s2)."""
+    """One plan: scale code from t = RN32(amax_b / RN32(M * s2))."""
     if s2 == 0:
         return 0, [0] * len(x), sum(F(float(xi)) ** 2 for xi in x)
     amax_b = max(abs(xi) for xi in x)
-    t = f32(f32(amax_b / f32(M)) / s2)
+    t = f32(amax_b / f32(f32(M) * s2))
     sc = e4m3_encode(t)
     codes, sse = plan_with_scale_code(x, s2, sc)
     return sc, codes, sse

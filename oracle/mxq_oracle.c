@@ -171,11 +171,14 @@ static double exact_add(double a, double b, int *ok)
 
 /* One NVFP4 plan for one 16-element block [P3 "What makes this build
  * different"; P1 introduction].
- *   t   = RN32(RN32(amax_b / M) / s2)             block scale in s2 units
+ *   t   = RN32(amax_b / RN32(M * s2))             block scale in s2 units
  *   S   = E4M3(t), D its value                    stored weight_scale byte
  *   d   = RN32(D * s2)                            fp32 effective block scale
  *   c_i = E2M1(RN32(x_i / d))                     stored value codes
- * Reading: D = 0, s2 = 0 or d = 0 (underflow) give all-zero codes 0x0.
+ * Readings: the pages name the plan "amax/6" (in units of weight_scale_2)
+ * without an operation order; the divisor M * s2 is rounded once to fp32
+ * and the block amax divided by it once.  D = 0, s2 = 0 or d = 0
+ * (underflow) give all-zero codes 0x0.
  * Returns, through G, the exact value of (SSE_M - sum x_i^2) / s2 where
  * SSE_M = sum_i (x_i - q_i * D * s2)^2 is the exact squared error of the
  * stored reconstruction q_i * D * s2 (q_i = value of c_i).  Expanding the
@@ -191,8 +194,8 @@ static int nvfp4_plan(const float x[16], float amax_b, float s2, float M,
     float d = 0.0f;
 
     if (s2 > 0.0f) {
-        float t = amax_b / M;
-        t = t / s2;
+        float den = M * s2;                          /* RN32(M * s2) */
+        float t = amax_b / den;
         sc = oracle_e4m3_encode((double)t);
         D = oracle_e4m3_value(sc);
         d = (float)D * s2;

@@ -62,7 +62,7 @@ def test_worked_example_golden(orc):
 
 def test_global_scale_closed_form_and_amax_block_scale(orc):
     """s2 = RN32(amax / 2688); under plain RTN the block holding the group
-    amax gets scale t = RN32(RN32(amax/6)/s2), which rounds to E4M3 448."""
+    amax gets scale t = RN32(amax / RN32(6 * s2)), which rounds to E4M3 448."""
     rng = np.random.default_rng(3)
     x = to_bf16_bits(rng.normal(0, 0.02, (4, 32, 64)).astype(np.float32))
     codes, scales, s2, m4 = orc.quantize_nvfp4(x, mode=0)
