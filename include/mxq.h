@@ -1,0 +1,212 @@
+/*
+ * mxq.h -- C ABI of the B200 (sm_100a) block-scaled microscaling quantizer.
+ *
+ * One library, libmxq.so, converts bf16 tensors into three block-scaled
+ * formats and verifies the result:
+ *   NVFP4  E2M1 values, one E4M3 scale per 16 values, one fp32 global
+ *          scale per group (weight_scale_2 / input_scale = amax / 2688);
+ *          block scales chosen by plain amax/6 (RTN) or by the 4/6-optimal
+ *          rule;
+ *   MXFP4  E2M1 values, one UE8M0 power-of-two scale per 32 values;
+ *   MXFP8  E4M3 values, one UE8M0 power-of-two scale per 32 values;
+ * and measures ||W - deq(Q(W))|| / ||W|| per tensor.
+ *
+ * Sources (model-card pages, section in quotes):
+ *   dabsLabs/Qwen3.8-Flash-Next-NVFP4, "What makes this build different":
+ *     4/6-optimal block scales; stacked [512, out, in] experts with fused
+ *     gate_up, unstacked per expert; relative-error metrics.
+ *   josch15366/Qwen3.8-Flash-Next-NVFP4-LocalHessian-Experts, introduction:
+ *     input_scale = amax/2688 (not amax/6); gate and up share one
+ *     weight_scale_2; "What is different about it": one weight_scale_2 per
+ *     expert.
+ *   azampatti/Qwen3.8-Flash-Next-FP4-Local-AZ, "The shared expert":
+ *     MXFP8 = e4m3 values, one power-of-two scale per 32 weights,
+ *     e = ceil(log2(amax/448)).
+ *   MJPansa/Qwen3.8-Flash-Next-MXFP4-FP8-R12, "Quantization format":
+ *     MXFP4 E2M1 weights with UE8M0 microscales; activations dynamically
+ *     quantized to MXFP8 at run time.
+ *
+ * Conventions for every entry point
+ *   - All pointers are DEVICE pointers unless stated; the caller owns every
+ *     buffer.  The library allocates nothing and keeps no state between
+ *     calls, except a per-device cache of the SM count.
+ *   - All work is enqueued asynchronously on `stream` (0 = legacy default
+ *     stream).  The call returns after enqueueing; results are valid once
+ *     the stream has reached that point.
+ *   - Errors found on the host (bad arguments) are returned before anything
+ *     is enqueued, and no output is touched.  MXQ_ERR_CUDA means a CUDA
+ *     runtime call failed while enqueueing; outputs are then undefined.
+ *   - Conditions found on the device are OR-ed into *status (a uint32 the
+ *     caller zeroes and reads after synchronising): MXQ_DEV_NONFINITE_INPUT
+ *     when an input element is Inf or NaN (outputs are then undefined),
+ *     MXQ_DEV_WAIT_TIMEOUT when a bounded inter-CTA wait gave up (outputs
+ *     are then undefined).  `status` may be NULL on the MX entry point
+ *     only (the check is then skipped); elsewhere it is required.
+ *   - Input bf16 data must be 16-byte aligned; code and scale outputs
+ *     must be 16-byte aligned; fp32 / fp64 arrays naturally aligned.
+ *     Otherwise MXQ_ERR_ALIGN.
+ *   - Tensors are row-major and contiguous; blocks run along the last
+ *     dimension (`cols`), which must be a multiple of the block size
+ *     (16 for NVFP4, 32 for MX), otherwise MXQ_ERR_SHAPE.
+ *   - Value codes: two 4-bit codes per byte, element 2j in the low nibble
+ *     and element 2j+1 in the high nibble (NVFP4, MXFP4); one byte per
+ *     element for MXFP8.  Scales: one byte per block, row-major
+ *     [rows, cols / block] per group (the linear checkpoint layout).
+ */
+#ifndef MXQ_H
+#define MXQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define MXQ_API __attribute__((visibility("default")))
+#else
+#define MXQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum mxq_status {
+    MXQ_OK = 0,
+    MXQ_ERR_INVALID_ARG = 1,  /* null pointer, negative size, unknown enum */
+    MXQ_ERR_SHAPE = 2,        /* cols not a multiple of the block, overflow */
+    MXQ_ERR_ALIGN = 3,        /* a pointer is not aligned as required */
+    MXQ_ERR_WORKSPACE = 4,    /* workspace NULL or smaller than required */
+    MXQ_ERR_CUDA = 5,         /* a CUDA runtime call failed */
+    MXQ_ERR_UNSUPPORTED = 6   /* valid but unsupported request (MX block != 32) */
+} mxq_status;
+
+/* Bits of the device status word. */
+#define MXQ_DEV_NONFINITE_INPUT 0x1u
+#define MXQ_DEV_WAIT_TIMEOUT 0x2u
+
+typedef enum mxq_fmt {
+    MXQ_FMT_NVFP4 = 0,
+    MXQ_FMT_MXFP4 = 1,
+    MXQ_FMT_MXFP8 = 2
+} mxq_fmt;
+
+typedef enum mxq_scale_mode {
+    MXQ_SCALE_RTN = 0,       /* plain amax/6 block scales */
+    MXQ_SCALE_FOUR_SIX = 1   /* 4/6-optimal block scales */
+} mxq_scale_mode;
+
+typedef enum mxq_op {
+    MXQ_OP_QUANTIZE_NVFP4 = 0,
+    MXQ_OP_QUANTIZE_ACT = 1,
+    MXQ_OP_DEQUANT_RELERR = 2
+} mxq_op;
+
+/* Version of this ABI (major * 10000 + minor * 100 + patch). */
+MXQ_API int mxq_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+MXQ_API const char *mxq_status_string(mxq_status s);
+
+/* Bytes of device workspace an entry point needs (0 if none).
+ *   MXQ_OP_QUANTIZE_NVFP4: n = n_groups, rows, cols as passed to it;
+ *   MXQ_OP_QUANTIZE_ACT:   n = T, rows = hidden, cols ignored;
+ *   MXQ_OP_DEQUANT_RELERR: n = n_tensors, rows, cols as passed to it.
+ * Returns 0 for invalid arguments. */
+MXQ_API size_t mxq_workspace_bytes(mxq_op op, int64_t n, int64_t rows, int64_t cols);
+
+/* NVFP4 quantization of a stack of groups.
+ * Source: dabsLabs/Qwen3.8-Flash-Next-NVFP4, "What makes this build
+ * different"; josch15366/Qwen3.8-Flash-Next-NVFP4-LocalHessian-Experts,
+ * introduction.
+ *   x        bf16 [n_groups, rows, cols].  A group shares one global scale:
+ *            pass one expert's fused gate_up slab [2I, H] per group so that
+ *            gate and up share weight_scale_2; down slabs [H, I] form their
+ *            own groups.  cols % 16 == 0.
+ *   mode     MXQ_SCALE_RTN or MXQ_SCALE_FOUR_SIX.
+ *   codes    out, uint8 [n_groups, rows, cols/2] E2M1 nibbles.
+ *   scales   out, uint8 [n_groups, rows, cols/16] E4M3 block scales.
+ *   s2       out, fp32 [n_groups]: s2 = RN32(amax_g / 2688).
+ *   mbits    out, nullable, uint32 [ceil(n_groups*rows*cols/16 / 32)]:
+ *            bit (b % 32) of word (b / 32) is 1 when block b (row-major
+ *            block index over the whole stack) took the M=4 plan.  Unused
+ *            high bits of the last word are written 0.
+ *   m4_count out, nullable, uint32 [n_groups]: number of M=4 blocks per
+ *            group (4/6 mode; zeros in RTN mode).
+ *   status   required, see conventions.
+ *   workspace / workspace_bytes: at least
+ *            mxq_workspace_bytes(MXQ_OP_QUANTIZE_NVFP4, n_groups, rows, cols).
+ * Per block of 16 (M in {6, 4}): t = RN32(amax_b / RN32(M*s2)), scale byte
+ * S = E4M3(t) (round to nearest even, saturating at 448), D its value,
+ * d = RN32(D*s2), code_i = E2M1(RN32(x_i / d)) (round to nearest even,
+ * saturating at 6, sign kept; all codes 0 when D or d is 0).  In 4/6 mode
+ * the M=4 plan is kept only when its exact squared error
+ * sum (x_i - q_i*D*s2)^2 is strictly lower than the M=6 plan's. */
+MXQ_API mxq_status mxq_quantize_nvfp4(const uint16_t *x, int64_t n_groups, int64_t rows,
+                              int64_t cols, mxq_scale_mode mode, uint8_t *codes,
+                              uint8_t *scales, float *s2, uint32_t *mbits,
+                              uint32_t *m4_count, uint32_t *status, void *workspace,
+                              size_t workspace_bytes, cudaStream_t stream);
+
+/* MX quantization (MXFP4 or MXFP8), one UE8M0 scale per 32 values.
+ * Source: azampatti/Qwen3.8-Flash-Next-FP4-Local-AZ, "The shared expert";
+ * MJPansa/Qwen3.8-Flash-Next-MXFP4-FP8-R12, "Quantization format".
+ *   x       bf16 [rows, cols], cols % 32 == 0 (stacked tensors: pass
+ *           rows = product of the leading dimensions).
+ *   fmt     MXQ_FMT_MXFP4 (E2M1, qmax 6) or MXQ_FMT_MXFP8 (E4M3, qmax 448).
+ *   block   must be 32 (MXQ_ERR_UNSUPPORTED otherwise).
+ *   codes   out, uint8 [rows, cols/2] (MXFP4) or [rows, cols] (MXFP8).
+ *   scales  out, uint8 [rows, cols/32], byte = e + 127 with e the smallest
+ *           integer such that amax <= qmax * 2^e (= ceil(log2(amax/qmax))),
+ *           clamped to [-127, 127]; an all-zero block gives byte 0.
+ *   status  nullable.
+ * code_i = FMT(x_i * 2^-e), round to nearest even, sign kept. */
+MXQ_API mxq_status mxq_quantize_mx(const uint16_t *x, int64_t rows, int64_t cols, mxq_fmt fmt,
+                           int block, uint8_t *codes, uint8_t *scales, uint32_t *status,
+                           cudaStream_t stream);
+
+/* Dynamic activation quantization of a token tile [T, hidden].
+ * Source: josch15366/Qwen3.8-Flash-Next-NVFP4-LocalHessian-Experts,
+ * introduction (input_scale = amax/2688); MJPansa/Qwen3.8-Flash-Next-MXFP4-FP8-R12,
+ * "Quantization format" (activations dynamically quantized to MXFP8).
+ *   fmt = MXQ_FMT_NVFP4: the whole tile is one group, input_scale =
+ *         RN32(amax / 2688) written to *input_scale (device fp32), block
+ *         scales plain amax/6 (RTN); codes [T, hidden/2], scales
+ *         [T, hidden/16]; workspace required.
+ *   fmt = MXQ_FMT_MXFP8 or MXQ_FMT_MXFP4: as mxq_quantize_mx with block 32;
+ *         input_scale, workspace may be NULL.
+ *   status required. */
+MXQ_API mxq_status mxq_quantize_act(const uint16_t *tokens, int64_t T, int64_t hidden,
+                            mxq_fmt fmt, uint8_t *codes, uint8_t *scales,
+                            float *input_scale, uint32_t *status, void *workspace,
+                            size_t workspace_bytes, cudaStream_t stream);
+
+/* Dequantize and measure per-tensor squared errors (the verifier).
+ * Source: dabsLabs/Qwen3.8-Flash-Next-NVFP4 (relative error of the
+ * quantized experts against the bf16 source, per tensor, mean and max);
+ * azampatti/Qwen3.8-Flash-Next-FP4-Local-AZ, "The shared expert" (error
+ * against the bf16 master).
+ *   x, codes, scales  as written by the quantizers, viewed as n_tensors
+ *            tensors of [rows, cols] stored back to back (unstacking a
+ *            fused gate_up [E, 2I, H] gives 2E tensors of [I, H]).
+ *   s2       NVFP4 only: fp32 [n_tensors / tensors_per_scale]; tensor t
+ *            reads s2[t / tensors_per_scale] (2 for fused gate_up, so that
+ *            gate_e and up_e read the shared weight_scale_2).  NULL for MX.
+ *   sum_sq_err, sum_sq_ref   out, fp64 [n_tensors]: sum (x - deq)^2 and
+ *            sum x^2 with deq = RN32((q * D) * s2) (NVFP4) or q * 2^e (MX).
+ *   relerr   out, nullable, fp64 [n_tensors]: sqrt(err) / sqrt(ref)
+ *            (0 when both are 0).
+ *   workspace: mxq_workspace_bytes(MXQ_OP_DEQUANT_RELERR, n_tensors, rows, cols).
+ * The sums are formed in a fixed order that does not depend on scheduling,
+ * so repeated calls give bit-identical results. */
+MXQ_API mxq_status mxq_dequant_relerr(const uint16_t *x, const uint8_t *codes,
+                              const uint8_t *scales, const float *s2, mxq_fmt fmt,
+                              int64_t n_tensors, int64_t rows, int64_t cols,
+                              int64_t tensors_per_scale, double *sum_sq_err,
+                              double *sum_sq_ref, double *relerr, void *workspace,
+                              size_t workspace_bytes, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MXQ_H */

@@ -1,0 +1,212 @@
+// api.cu -- the C ABI declared in include/mxq.h: argument checks,
+// workspace carving and kernel launches.  No allocation, no host-device
+// synchronisation, no state beyond a per-device SM-count cache.
+#include "mxq.h"
+#include "mxq_internal.h"
+
+#include <limits.h>
+
+namespace mxq {
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+size_t nvfp4_workspace_bytes(int64_t n_groups)
+{
+    return 2 * align_up((size_t)n_groups * sizeof(uint32_t), 256);
+}
+
+static size_t verify_workspace_bytes(int64_t n_tensors, int64_t rows, int64_t cols)
+{
+    const int64_t tsize = rows * cols;
+    const int64_t cpt = tsize > 0 ? (tsize + kVerifyChunk - 1) / kVerifyChunk : 1;
+    return align_up((size_t)(n_tensors * cpt) * 2 * sizeof(double), 256);
+}
+
+static bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+// rows * cols * n without overflow, all non-negative.
+static bool mul_ok(int64_t a, int64_t b, int64_t *out)
+{
+    if (a < 0 || b < 0)
+        return false;
+    if (a != 0 && b > INT64_MAX / a)
+        return false;
+    *out = a * b;
+    return true;
+}
+
+} // namespace mxq
+
+using namespace mxq;
+
+extern "C" {
+
+int mxq_version(void) { return 10000; }
+
+const char *mxq_status_string(mxq_status s)
+{
+    switch (s) {
+    case MXQ_OK: return "ok";
+    case MXQ_ERR_INVALID_ARG: return "invalid argument";
+    case MXQ_ERR_SHAPE: return "unsupported shape (cols must be a multiple of the block size)";
+    case MXQ_ERR_ALIGN: return "misaligned pointer";
+    case MXQ_ERR_WORKSPACE: return "workspace missing or too small";
+    case MXQ_ERR_CUDA: return "CUDA runtime error";
+    case MXQ_ERR_UNSUPPORTED: return "unsupported request";
+    }
+    return "unknown status";
+}
+
+size_t mxq_workspace_bytes(mxq_op op, int64_t n, int64_t rows, int64_t cols)
+{
+    int64_t tmp;
+    if (n < 0 || rows < 0 || (op != MXQ_OP_QUANTIZE_ACT && cols < 0))
+        return 0;
+    switch (op) {
+    case MXQ_OP_QUANTIZE_NVFP4:
+        if (!mul_ok(rows, cols, &tmp) || !mul_ok(tmp, n, &tmp))
+            return 0;
+        return nvfp4_workspace_bytes(n);
+    case MXQ_OP_QUANTIZE_ACT:
+        if (!mul_ok(n, rows, &tmp))
+            return 0;
+        return nvfp4_workspace_bytes(1);
+    case MXQ_OP_DEQUANT_RELERR:
+        if (!mul_ok(rows, cols, &tmp) || !mul_ok(tmp, n, &tmp))
+            return 0;
+        return verify_workspace_bytes(n, rows, cols);
+    }
+    return 0;
+}
+
+mxq_status mxq_quantize_nvfp4(const uint16_t *x, int64_t n_groups, int64_t rows, int64_t cols,
+                              mxq_scale_mode mode, uint8_t *codes, uint8_t *scales, float *s2,
+                              uint32_t *mbits, uint32_t *m4_count, uint32_t *status,
+                              void *workspace, size_t workspace_bytes, cudaStream_t stream)
+{
+    if (n_groups < 0 || rows < 0 || cols < 0)
+        return MXQ_ERR_INVALID_ARG;
+    if (mode != MXQ_SCALE_RTN && mode != MXQ_SCALE_FOUR_SIX)
+        return MXQ_ERR_INVALID_ARG;
+    if (cols % 16 != 0)
+        return MXQ_ERR_SHAPE;
+    int64_t gsize, total;
+    if (!mul_ok(rows, cols, &gsize) || !mul_ok(gsize, n_groups, &total) || total > (INT64_MAX / 4))
+        return MXQ_ERR_SHAPE;
+    if (n_groups == 0)
+        return MXQ_OK;
+    if (!x || !codes || !scales || !s2 || !status)
+        return MXQ_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(scales, 16) || !aligned(s2, 4) ||
+        !aligned(status, 4) || (mbits && !aligned(mbits, 4)) || (m4_count && !aligned(m4_count, 4)))
+        return MXQ_ERR_ALIGN;
+    const size_t need = nvfp4_workspace_bytes(n_groups);
+    if (!workspace || workspace_bytes < need)
+        return MXQ_ERR_WORKSPACE;
+    if (!aligned(workspace, 256))
+        return MXQ_ERR_ALIGN;
+    const int64_t nb = gsize / 16;
+    const int64_t total_blocks = total / 16;
+    uint32_t *amax_bits = static_cast<uint32_t *>(workspace);
+    cudaError_t e = cudaMemsetAsync(amax_bits, 0, (size_t)n_groups * sizeof(uint32_t), stream);
+    if (e == cudaSuccess && m4_count)
+        e = cudaMemsetAsync(m4_count, 0, (size_t)n_groups * sizeof(uint32_t), stream);
+    const int mbits_atomic = (nb % 32) != 0;
+    if (e == cudaSuccess && mbits && (mbits_atomic || nb == 0 || total_blocks % 32 != 0))
+        e = cudaMemsetAsync(mbits, 0, (size_t)((total_blocks + 31) / 32) * sizeof(uint32_t), stream);
+    if (e == cudaSuccess)
+        e = launch_group_amax(x, n_groups, nb, amax_bits, status, stream);
+    if (e == cudaSuccess)
+        e = launch_nvfp4_quant(x, n_groups, nb, mode == MXQ_SCALE_FOUR_SIX, amax_bits, codes, scales,
+                               s2, mbits, mbits_atomic, mode == MXQ_SCALE_FOUR_SIX ? m4_count : nullptr,
+                               stream);
+    return e == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
+}
+
+mxq_status mxq_quantize_mx(const uint16_t *x, int64_t rows, int64_t cols, mxq_fmt fmt, int block,
+                           uint8_t *codes, uint8_t *scales, uint32_t *status, cudaStream_t stream)
+{
+    if (rows < 0 || cols < 0)
+        return MXQ_ERR_INVALID_ARG;
+    if (fmt != MXQ_FMT_MXFP4 && fmt != MXQ_FMT_MXFP8)
+        return MXQ_ERR_INVALID_ARG;
+    if (block != 32)
+        return MXQ_ERR_UNSUPPORTED;
+    if (cols % 32 != 0)
+        return MXQ_ERR_SHAPE;
+    int64_t total;
+    if (!mul_ok(rows, cols, &total) || total > (INT64_MAX / 4))
+        return MXQ_ERR_SHAPE;
+    if (total == 0)
+        return MXQ_OK;
+    if (!x || !codes || !scales)
+        return MXQ_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(scales, 16) || (status && !aligned(status, 4)))
+        return MXQ_ERR_ALIGN;
+    cudaError_t e = launch_mx_quant(x, total / 32, (int)fmt, codes, scales, status, stream);
+    return e == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
+}
+
+mxq_status mxq_quantize_act(const uint16_t *tokens, int64_t T, int64_t hidden, mxq_fmt fmt,
+                            uint8_t *codes, uint8_t *scales, float *input_scale, uint32_t *status,
+                            void *workspace, size_t workspace_bytes, cudaStream_t stream)
+{
+    if (T < 0 || hidden < 0)
+        return MXQ_ERR_INVALID_ARG;
+    if (!status)
+        return MXQ_ERR_INVALID_ARG;
+    if (fmt == MXQ_FMT_NVFP4) {
+        if (!input_scale)
+            return MXQ_ERR_INVALID_ARG;
+        if (T == 0 || hidden == 0) {
+            if (hidden % 16 != 0)
+                return MXQ_ERR_SHAPE;
+            return cudaMemsetAsync(input_scale, 0, sizeof(float), stream) == cudaSuccess ? MXQ_OK
+                                                                                          : MXQ_ERR_CUDA;
+        }
+        return mxq_quantize_nvfp4(tokens, 1, T, hidden, MXQ_SCALE_RTN, codes, scales, input_scale,
+                                  nullptr, nullptr, status, workspace, workspace_bytes, stream);
+    }
+    if (fmt == MXQ_FMT_MXFP4 || fmt == MXQ_FMT_MXFP8)
+        return mxq_quantize_mx(tokens, T, hidden, fmt, 32, codes, scales, status, stream);
+    return MXQ_ERR_INVALID_ARG;
+}
+
+mxq_status mxq_dequant_relerr(const uint16_t *x, const uint8_t *codes, const uint8_t *scales,
+                              const float *s2, mxq_fmt fmt, int64_t n_tensors, int64_t rows,
+                              int64_t cols, int64_t tensors_per_scale, double *sum_sq_err,
+                              double *sum_sq_ref, double *relerr, void *workspace,
+                              size_t workspace_bytes, cudaStream_t stream)
+{
+    if (n_tensors < 0 || rows < 0 || cols < 0)
+        return MXQ_ERR_INVALID_ARG;
+    if (fmt != MXQ_FMT_NVFP4 && fmt != MXQ_FMT_MXFP4 && fmt != MXQ_FMT_MXFP8)
+        return MXQ_ERR_INVALID_ARG;
+    if (fmt == MXQ_FMT_NVFP4 && tensors_per_scale < 1)
+        return MXQ_ERR_INVALID_ARG;
+    const int blk = (fmt == MXQ_FMT_NVFP4) ? 16 : 32;
+    if (cols % blk != 0)
+        return MXQ_ERR_SHAPE;
+    int64_t tsize, total;
+    if (!mul_ok(rows, cols, &tsize) || !mul_ok(tsize, n_tensors, &total) || total > (INT64_MAX / 4))
+        return MXQ_ERR_SHAPE;
+    if (n_tensors == 0)
+        return MXQ_OK;
+    if (!sum_sq_err || !sum_sq_ref)
+        return MXQ_ERR_INVALID_ARG;
+    if (total > 0 && (!x || !codes || !scales || (fmt == MXQ_FMT_NVFP4 && !s2)))
+        return MXQ_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(scales, 16) || (s2 && !aligned(s2, 4)) ||
+        !aligned(sum_sq_err, 8) || !aligned(sum_sq_ref, 8) || (relerr && !aligned(relerr, 8)))
+        return MXQ_ERR_ALIGN;
+    const size_t need = verify_workspace_bytes(n_tensors, rows, cols);
+    if (!workspace || workspace_bytes < need)
+        return MXQ_ERR_WORKSPACE;
+    if (!aligned(workspace, 256))
+        return MXQ_ERR_ALIGN;
+    cudaError_t e = launch_verify(x, codes, scales, s2, (int)fmt, n_tensors, tsize, tensors_per_scale,
+                                  static_cast<double *>(workspace), sum_sq_err, sum_sq_ref, relerr, stream);
+    return e == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
+}
+
+} // extern "C"

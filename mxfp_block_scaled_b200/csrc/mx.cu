@@ -1,0 +1,97 @@
+// mx.cu -- MXFP8 / MXFP4 quantization, one UE8M0 scale per 32 values
+// (sm_100a).
+//
+// Method (azampatti/Qwen3.8-Flash-Next-FP4-Local-AZ, "The shared expert":
+// e4m3 values, one power-of-two scale per 32 weights,
+// e = ceil(log2(amax / 448)); MJPansa/Qwen3.8-Flash-Next-MXFP4-FP8-R12,
+// "Quantization format": E2M1 weights with UE8M0 microscales, qmax 6):
+//   e = smallest integer with amax <= qmax * 2^e, clamped to [-127, 127];
+//   scale byte = e + 127; code_i = FMT(x_i * 2^-e), round to nearest even.
+//
+// The exponent is read off the bf16 bits of amax, exactly: with
+// amax = m * 2^E (1 <= m < 2) and qmax = c * 2^k (448 = 1.75 * 2^8,
+// 6 = 1.5 * 2^2), amax <= qmax * 2^e  <=>  e >= E - k + (m > c).  A
+// subnormal or zero amax always lands on the lower clamp.
+#include "mxq_device.cuh"
+#include "mxq_internal.h"
+#include "mxq.h"
+
+namespace mxq {
+
+template <int FMT>
+__device__ __forceinline__ int mx_exponent(uint32_t amax_bits)
+{
+    constexpr int k = (FMT == MXQ_FMT_MXFP8) ? 8 : 2;
+    constexpr uint32_t c_mant = (FMT == MXQ_FMT_MXFP8) ? 0x60u : 0x40u;  // .75 / .5 in 7 bits
+    const uint32_t E = amax_bits >> 7;
+    if (E == 0)
+        return -127;
+    int e = (int)E - 127 - k + ((amax_bits & 0x7Fu) > c_mant ? 1 : 0);
+    return e < -127 ? -127 : (e > 127 ? 127 : e);
+}
+
+// One thread per block of 32: 64 bytes in, 32 (MXFP8) or 16 (MXFP4) out.
+template <int FMT>
+__global__ void __launch_bounds__(256)
+mx_quant_kernel(const uint4 *__restrict__ x, int64_t nblk, uint8_t *__restrict__ codes,
+                uint8_t *__restrict__ scales, uint32_t *__restrict__ status)
+{
+    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk;
+         b += (int64_t)gridDim.x * blockDim.x) {
+        uint4 v[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            v[k] = __ldg(x + b * 4 + k);
+        const uint32_t w[16] = {v[0].x, v[0].y, v[0].z, v[0].w, v[1].x, v[1].y, v[1].z, v[1].w,
+                                v[2].x, v[2].y, v[2].z, v[2].w, v[3].x, v[3].y, v[3].z, v[3].w};
+        uint32_t m = 0;
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            m = abs_max_bits(m, w[j]);
+        const uint32_t a = fold_halves(m);
+        if (a >= 0x7F80u && status)
+            atomicOr(status, MXQ_DEV_NONFINITE_INPUT);
+        const int e = mx_exponent<FMT>(a);
+        const float sc = __uint_as_float((uint32_t)(127 - e) << 23);   // 2^-e, normal
+        const float2 sc2 = make_float2(sc, sc);
+        float2 y[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            y[j] = __fmul2_rn(make_float2(bf16_lo(w[j]), bf16_hi(w[j])), sc2);
+        scales[b] = (uint8_t)(e + 127);
+        if (FMT == MXQ_FMT_MXFP8) {
+            uint32_t o[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                o[j] = e4m3x2(y[2 * j].x, y[2 * j].y) | (e4m3x2(y[2 * j + 1].x, y[2 * j + 1].y) << 16);
+            uint4 *dst = reinterpret_cast<uint4 *>(codes) + b * 2;
+            dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+            dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+        } else {
+            uint4 o;
+            o.x = e2m1x8(y[0], y[1], y[2], y[3]);
+            o.y = e2m1x8(y[4], y[5], y[6], y[7]);
+            o.z = e2m1x8(y[8], y[9], y[10], y[11]);
+            o.w = e2m1x8(y[12], y[13], y[14], y[15]);
+            reinterpret_cast<uint4 *>(codes)[b] = o;
+        }
+    }
+}
+
+cudaError_t launch_mx_quant(const uint16_t *x, int64_t nblk32, int fmt, uint8_t *codes,
+                            uint8_t *scales, uint32_t *status, cudaStream_t s)
+{
+    if (nblk32 == 0)
+        return cudaSuccess;
+    int64_t ctas = (nblk32 + 255) / 256;
+    if (ctas > 0x7FFFFFFF)
+        ctas = 0x7FFFFFFF;
+    const uint4 *xv = reinterpret_cast<const uint4 *>(x);
+    if (fmt == MXQ_FMT_MXFP8)
+        mx_quant_kernel<MXQ_FMT_MXFP8><<<(unsigned)ctas, 256, 0, s>>>(xv, nblk32, codes, scales, status);
+    else
+        mx_quant_kernel<MXQ_FMT_MXFP4><<<(unsigned)ctas, 256, 0, s>>>(xv, nblk32, codes, scales, status);
+    return cudaGetLastError();
+}
+
+} // namespace mxq

@@ -1,0 +1,130 @@
+// mxq_device.cuh -- device helpers shared by the quantizer and verifier
+// kernels (sm_100a).  Number-format conversions use the PTX cvt
+// instructions of the public PTX ISA (e2m1x2 / e4m3x2 packing and
+// unpacking); everything else is plain IEEE fp32 / fp64 arithmetic with
+// explicit rounding intrinsics, so no FMA contraction changes a result.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace mxq {
+
+// ---- bf16 <-> fp32 ------------------------------------------------------
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Largest |x| of the 16-bit halves of `words` as bf16 magnitude bits.  Bit
+// patterns of non-negative bf16 values order like the values, and Inf / NaN
+// patterns (exponent all ones) sort above every finite value, so the result
+// is >= 0x7F80 exactly when some element is not finite.
+__device__ __forceinline__ uint32_t abs_max_bits(uint32_t acc, uint32_t w)
+{
+    return __vmaxu2(acc, w & 0x7FFF7FFFu);
+}
+__device__ __forceinline__ uint32_t fold_halves(uint32_t m) { return max(m & 0xFFFFu, m >> 16); }
+
+// ---- packed conversions (PTX ISA: cvt with .e2m1x2 / .e4m3x2) ------------
+// Eight fp32 values -> eight E2M1 codes in one word, element 2j in the low
+// nibble of byte j.  Round to nearest even, saturating at +-6, sign kept.
+__device__ __forceinline__ uint32_t e2m1x8(float2 p0, float2 p1, float2 p2, float2 p3)
+{
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(out)
+        : "f"(p0.x), "f"(p0.y), "f"(p1.x), "f"(p1.y), "f"(p2.x), "f"(p2.y), "f"(p3.x), "f"(p3.y));
+    return out;
+}
+
+// Byte j of `w` (two E2M1 codes) -> f16x2 values, low nibble in the low half.
+template <int J>
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t w)
+{
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b" "%2" ";\n\t}"
+        : "=r"(out) : "r"(w), "n"(J));
+    return out;
+}
+
+// Two fp32 -> two E4M3 bytes (lo from `lo`, hi from `hi`), round to nearest
+// even, saturating at +-448 (never the NaN code).
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi)
+{
+    uint16_t out;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(out) : "f"(lo), "f"(hi));
+    return out;
+}
+
+// Two E4M3 bytes (low 16 bits of `v`) -> f16x2 values, exact.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t v)
+{
+    uint32_t out;
+    uint16_t h = (uint16_t)v;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(out) : "h"(h));
+    return out;
+}
+
+__device__ __forceinline__ float2 f16x2_to_float2(uint32_t h)
+{
+    return __half22float2(*reinterpret_cast<const __half2 *>(&h));
+}
+
+__device__ __forceinline__ uint32_t hmul2_bits(uint32_t a, uint32_t b)
+{
+    __half2 r = __hmul2(*reinterpret_cast<const __half2 *>(&a), *reinterpret_cast<const __half2 *>(&b));
+    return *reinterpret_cast<uint32_t *>(&r);
+}
+
+__device__ __forceinline__ uint32_t hfma2_bits(uint32_t a, uint32_t b, uint32_t c)
+{
+    __half2 r = __hfma2(*reinterpret_cast<const __half2 *>(&a), *reinterpret_cast<const __half2 *>(&b),
+                        *reinterpret_cast<const __half2 *>(&c));
+    return *reinterpret_cast<uint32_t *>(&r);
+}
+
+// ---- correctly rounded quotient of a bf16 numerator ---------------------
+// y = RN32(x / d) from r = RN32(1 / d) with one FMA correction (Markstein,
+// IBM J. Res. Dev. 34(1), 1990).  Proven exact by exhaustion over every
+// pair of significands (8-bit x, 24-bit d) for normal operands and results
+// (tests/csrc/division_check.c); callers take __fdiv_rn outside that range.
+// The residual is formed as q0*d - x and subtracted, which keeps -0 / d = -0.
+__device__ __forceinline__ float div_bf16(float x, float d, float r)
+{
+    float q0 = __fmul_rn(x, r);
+    float e = __fmaf_rn(q0, d, -x);
+    return __fmaf_rn(-e, r, q0);
+}
+
+// Pairwise form on -x (nx), with nr = -r: returns x/d for both lanes.  The
+// operations are the same IEEE operations as div_bf16 with the negations
+// moved onto operands, so each lane's result is bit-identical to it.
+__device__ __forceinline__ float2 div2_bf16_neg(float2 nx, float2 d, float2 nr)
+{
+    float2 q0 = __fmul2_rn(nx, nr);          // x * r
+    float2 e = __ffma2_rn(q0, d, nx);        // q0 * d - x
+    return __ffma2_rn(e, nr, q0);            // q0 - e * r
+}
+
+// Bounded spin for inter-CTA flags: returns false after `limit` polls.
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p)
+{
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void red_release_add_u32(uint32_t *p, uint32_t v)
+{
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+} // namespace mxq

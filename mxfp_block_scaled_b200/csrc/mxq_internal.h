@@ -1,0 +1,40 @@
+// mxq_internal.h -- launch interface between the C-ABI layer (api.cu) and
+// the kernel translation units.  Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace mxq {
+
+constexpr float kGlobalDivisor = 2688.0f;  // 6 * 448: weight_scale_2 / input_scale
+
+// NVFP4 streaming kernels: CTA tile of 512 blocks of 16 (256 threads x 2).
+constexpr int kNvThreads = 256;
+constexpr int kNvTileBlocks = 512;
+
+// Verifier: one CTA reduces one chunk of a tensor.
+constexpr int kVerifyThreads = 256;
+constexpr int64_t kVerifyChunk = 16384;  // elements per chunk (multiple of 32)
+
+size_t align_up(size_t v, size_t a);
+
+// Workspace of the NVFP4 quantizer: per-group amax bits and per-group
+// arrival counters, each padded to 256 bytes.
+size_t nvfp4_workspace_bytes(int64_t n_groups);
+
+cudaError_t launch_group_amax(const uint16_t *x, int64_t n_groups, int64_t nb,
+                              uint32_t *amax_bits, uint32_t *status, cudaStream_t s);
+cudaError_t launch_nvfp4_quant(const uint16_t *x, int64_t n_groups, int64_t nb, int four_six,
+                               const uint32_t *amax_bits, uint8_t *codes, uint8_t *scales,
+                               float *s2, uint32_t *mbits, int mbits_atomic,
+                               uint32_t *m4_count, cudaStream_t s);
+cudaError_t launch_mx_quant(const uint16_t *x, int64_t nblk32, int fmt, uint8_t *codes,
+                            uint8_t *scales, uint32_t *status, cudaStream_t s);
+cudaError_t launch_verify(const uint16_t *x, const uint8_t *codes, const uint8_t *scales,
+                          const float *s2, int fmt, int64_t n_tensors, int64_t tsize,
+                          int64_t tensors_per_scale, double *partials, double *sum_sq_err,
+                          double *sum_sq_ref, double *relerr, cudaStream_t s);
+
+} // namespace mxq

@@ -1,0 +1,324 @@
+// nvfp4.cu -- NVFP4 quantization with 4/6-optimal block scales (sm_100a).
+//
+// Method (dabsLabs/Qwen3.8-Flash-Next-NVFP4, "What makes this build
+// different"; josch15366/Qwen3.8-Flash-Next-NVFP4-LocalHessian-Experts,
+// introduction):
+//   s2 = RN32(amax_g / 2688) per group (one expert's fused gate_up slab, so
+//   gate and up share weight_scale_2; or one down slab; or one token tile);
+//   per block of 16 and plan M in {6, 4}:
+//     t_M = RN32(amax_b / RN32(M * s2)),  S_M = E4M3(t_M),  D_M = value(S_M)
+//     d_M = RN32(D_M * s2),  code_i = E2M1(RN32(x_i / d_M))
+//   and the M=4 plan is kept only when its exact squared error
+//   sum (x_i - q_i D_M s2)^2 is strictly lower than the M=6 plan's.
+//
+// Exact decision.  sum x_i^2 is common to both plans, so
+//   SSE_M - sum x^2 = s2 * D_M * (D_M s2 B_M - 2 A_M),
+//   A_M = sum x_i q_i,  B_M = sum q_i^2,
+// and since s2 > 0 the comparison SSE_4 < SSE_6 is G_4 < G_6 with
+// G_M = D_M * (D_M s2 B_M - 2 A_M).  Every term is exact in the precision
+// it is formed in: x_i q_i has at most 8 + 2 significant bits and every
+// non-zero term lies within 2^21 of the smallest one (a non-zero code needs
+// |x| > d/4 and |x| <= 9 d), so A_M is exact in fp32 in any order; B_M is a
+// sum of quarter-integers <= 576, exact in f16 half-sums of 8 and in fp32;
+// D_M s2 (4 + 24 bits), D_M s2 B_M - 2 A_M (< 2^40 span) and D_M * P (4 + 40
+// bits) are exact in fp64.  So the decision has no rounding at all.
+//
+// Pipeline: group_amax_kernel (pass 1) -> nvfp4_quant_kernel (pass 2).
+#include "mxq_device.cuh"
+#include "mxq_internal.h"
+#include "mxq.h"
+
+namespace mxq {
+
+// ---------------------------------------------------------------------------
+// Pass 1: per-group amax as bf16 magnitude bits (atomicMax is order-free).
+// grid = (tiles of 512 blocks, groups); each thread reads 4 x 16 bytes.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kNvThreads)
+group_amax_kernel(const uint4 *__restrict__ x, int64_t n_groups, int64_t nb,
+                  uint32_t *__restrict__ amax_bits, uint32_t *__restrict__ status)
+{
+    __shared__ uint32_t warp_max[kNvThreads / 32];
+    const int64_t vec_per_group = nb * 2;  // 16-byte vectors per group
+    for (int64_t g = blockIdx.y; g < n_groups; g += gridDim.y) {
+        const uint4 *xg = x + g * vec_per_group;
+        uint32_t m = 0;
+        for (int64_t base = (int64_t)blockIdx.x * (kNvTileBlocks * 2); base < vec_per_group;
+             base += (int64_t)gridDim.x * (kNvTileBlocks * 2)) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                int64_t i = base + threadIdx.x + k * kNvThreads;
+                if (i < vec_per_group) {
+                    uint4 v = __ldg(xg + i);
+                    m = abs_max_bits(m, v.x);
+                    m = abs_max_bits(m, v.y);
+                    m = abs_max_bits(m, v.z);
+                    m = abs_max_bits(m, v.w);
+                }
+            }
+        }
+        uint32_t a = __reduce_max_sync(0xFFFFFFFFu, fold_halves(m));
+        if ((threadIdx.x & 31) == 0)
+            warp_max[threadIdx.x >> 5] = a;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            uint32_t r = 0;
+            for (int w = 0; w < kNvThreads / 32; ++w)
+                r = max(r, warp_max[w]);
+            if (r != 0)
+                atomicMax(amax_bits + g, r);
+            if (r >= 0x7F80u)
+                atomicOr(status, MXQ_DEV_NONFINITE_INPUT);
+        }
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Pass 2: the block quantizer.
+// ---------------------------------------------------------------------------
+struct GroupConst {
+    float s2;        // global scale
+    float den6, r6;  // RN32(6 s2), RN32(1 / den6)
+    float den4, r4;  // 4 s2 (exact), RN32(1 / den4)
+    int fast;        // den in the range where div_bf16 is exact
+};
+
+__device__ __forceinline__ GroupConst make_group_const(uint32_t amax_bits)
+{
+    GroupConst c;
+    const float amax = __uint_as_float(amax_bits << 16);
+    c.s2 = __fdiv_rn(amax, kGlobalDivisor);
+    c.den6 = __fmul_rn(6.0f, c.s2);
+    c.den4 = __fmul_rn(4.0f, c.s2);
+    c.fast = (c.s2 >= 0x1p-100f && c.s2 <= 0x1p100f) ? 1 : 0;
+    c.r6 = c.fast ? __frcp_rn(c.den6) : 0.0f;
+    c.r4 = c.fast ? __frcp_rn(c.den4) : 0.0f;
+    return c;
+}
+
+struct Plan {
+    uint2 codes;   // 16 E2M1 nibbles
+    float a_neg;   // -sum x_i q_i (exact)
+    float b;       // sum q_i^2 (exact)
+};
+
+// q pair (f16x2) of byte J of `w`: accumulate B in f16 (exact: <= 8 terms of
+// quarter-integers <= 36 per half) and -A in fp32 pairs.
+template <int J>
+__device__ __forceinline__ void accum_pair(uint32_t w, float2 nx, float2 &acc, uint32_t &bh)
+{
+    const uint32_t qh = e2m1x2_to_f16x2<J>(w);
+    bh = hfma2_bits(qh, qh, bh);
+    acc = __ffma2_rn(nx, f16x2_to_float2(qh), acc);
+}
+
+__device__ __forceinline__ Plan make_plan(const float2 (&nx)[8], float D, float s2)
+{
+    Plan p;
+    const float d = __fmul_rn(D, s2);
+    if (!(d > 0.0f)) {  // D == 0, or D * s2 underflowed: all codes 0
+        p.codes = make_uint2(0u, 0u);
+        p.a_neg = 0.0f;
+        p.b = 0.0f;
+        return p;
+    }
+    float2 y[8];
+    if (d >= 0x1p-60f && d <= 0x1p60f) {
+        const float r = __frcp_rn(d);
+        const float2 d2 = make_float2(d, d), nr2 = make_float2(-r, -r);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            y[j] = div2_bf16_neg(nx[j], d2, nr2);
+    } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            y[j] = make_float2(__fdiv_rn(-nx[j].x, d), __fdiv_rn(-nx[j].y, d));
+    }
+    p.codes.x = e2m1x8(y[0], y[1], y[2], y[3]);
+    p.codes.y = e2m1x8(y[4], y[5], y[6], y[7]);
+    float2 acc = make_float2(0.0f, 0.0f);
+    uint32_t bh = 0u;
+    accum_pair<0>(p.codes.x, nx[0], acc, bh);
+    accum_pair<1>(p.codes.x, nx[1], acc, bh);
+    accum_pair<2>(p.codes.x, nx[2], acc, bh);
+    accum_pair<3>(p.codes.x, nx[3], acc, bh);
+    accum_pair<0>(p.codes.y, nx[4], acc, bh);
+    accum_pair<1>(p.codes.y, nx[5], acc, bh);
+    accum_pair<2>(p.codes.y, nx[6], acc, bh);
+    accum_pair<3>(p.codes.y, nx[7], acc, bh);
+    p.a_neg = __fadd_rn(acc.x, acc.y);
+    const float2 bf = f16x2_to_float2(bh);
+    p.b = __fadd_rn(bf.x, bf.y);
+    return p;
+}
+
+// G_M = D (D s2 B - 2 A) in fp64, exact (see the file comment).
+__device__ __forceinline__ double plan_g(float D, float s2, const Plan &p)
+{
+    const double dS = (double)D * (double)s2;
+    const double P = fma(dS, (double)p.b, 2.0 * (double)p.a_neg);
+    return (double)D * P;
+}
+
+struct BlockOut {
+    uint2 codes;
+    uint32_t scale;
+    bool m4;
+};
+
+template <bool FOUR_SIX>
+__device__ __forceinline__ BlockOut quantize_block(uint4 v0, uint4 v1, const GroupConst &gc)
+{
+    BlockOut o;
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    uint32_t m = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        m = abs_max_bits(m, w[j]);
+    const float amax_b = __uint_as_float(fold_halves(m) << 16);
+    if (!(gc.s2 > 0.0f)) {  // all-zero group
+        o.codes = make_uint2(0u, 0u);
+        o.scale = 0u;
+        o.m4 = false;
+        return o;
+    }
+    float2 nx[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const uint32_t n = w[j] ^ 0x80008000u;
+        nx[j] = make_float2(bf16_lo(n), bf16_hi(n));
+    }
+    float t6, t4;
+    if (gc.fast) {
+        t6 = div_bf16(amax_b, gc.den6, gc.r6);
+        t4 = div_bf16(amax_b, gc.den4, gc.r4);
+    } else {
+        t6 = __fdiv_rn(amax_b, gc.den6);
+        t4 = __fdiv_rn(amax_b, gc.den4);
+    }
+    const uint32_t sb = e4m3x2(t6, FOUR_SIX ? t4 : 0.0f);   // S6 low byte, S4 high
+    const float2 D = f16x2_to_float2(e4m3x2_to_f16x2(sb));
+    const Plan p6 = make_plan(nx, D.x, gc.s2);
+    if (!FOUR_SIX) {
+        o.codes = p6.codes;
+        o.scale = sb & 0xFFu;
+        o.m4 = false;
+        return o;
+    }
+    const Plan p4 = make_plan(nx, D.y, gc.s2);
+    const bool use4 = plan_g(D.y, gc.s2, p4) < plan_g(D.x, gc.s2, p6);
+    o.codes = use4 ? p4.codes : p6.codes;
+    o.scale = use4 ? (sb >> 8) : (sb & 0xFFu);
+    o.m4 = use4;
+    return o;
+}
+
+// grid = (tiles of 512 blocks, groups).  Thread t of a tile handles blocks
+// t and t + 256, so each warp covers 32 consecutive blocks per step and its
+// M bits form one 32-bit word.
+template <bool FOUR_SIX>
+__global__ void __launch_bounds__(kNvThreads)
+nvfp4_quant_kernel(const uint4 *__restrict__ x, int64_t n_groups, int64_t nb,
+                   const uint32_t *__restrict__ amax_bits, uint2 *__restrict__ codes,
+                   uint8_t *__restrict__ scales, float *__restrict__ s2_out,
+                   uint32_t *__restrict__ mbits, int mbits_atomic, uint32_t *__restrict__ m4_count)
+{
+    __shared__ GroupConst s_gc;
+    __shared__ uint32_t s_m4;
+    const int lane = threadIdx.x & 31;
+    for (int64_t g = blockIdx.y; g < n_groups; g += gridDim.y) {
+        if (threadIdx.x == 0) {
+            s_gc = make_group_const(amax_bits[g]);
+            if (blockIdx.x == 0)
+                s2_out[g] = s_gc.s2;
+            s_m4 = 0;
+        }
+        __syncthreads();
+        const GroupConst gc = s_gc;
+        uint32_t my_m4 = 0;
+        for (int64_t tile = blockIdx.x; tile * kNvTileBlocks < nb; tile += gridDim.x) {
+            const int64_t b0 = tile * kNvTileBlocks + threadIdx.x;
+            uint4 v[2][2];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int64_t b = b0 + k * kNvThreads;
+                if (b < nb) {
+                    const uint4 *src = x + (g * nb + b) * 2;
+                    v[k][0] = __ldg(src);
+                    v[k][1] = __ldg(src + 1);
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int64_t b = b0 + k * kNvThreads;
+                const bool live = b < nb;
+                BlockOut o;
+                o.m4 = false;
+                if (live) {
+                    o = quantize_block<FOUR_SIX>(v[k][0], v[k][1], gc);
+                    const int64_t gb = g * nb + b;
+                    codes[gb] = o.codes;
+                    scales[gb] = (uint8_t)o.scale;
+                }
+                if (mbits) {
+                    const uint32_t word = __ballot_sync(0xFFFFFFFFu, o.m4);
+                    const int64_t warp_first = g * nb + (b - lane);
+                    if (!mbits_atomic) {
+                        if (lane == 0 && (b - lane) < nb)
+                            mbits[warp_first >> 5] = word;
+                    } else if (live && o.m4) {
+                        const int64_t gb = g * nb + b;
+                        atomicOr(mbits + (gb >> 5), 1u << (gb & 31));
+                    }
+                }
+                my_m4 += o.m4 ? 1u : 0u;
+            }
+        }
+        if (FOUR_SIX && m4_count) {
+            const uint32_t wsum = __reduce_add_sync(0xFFFFFFFFu, my_m4);
+            if (lane == 0 && wsum)
+                atomicAdd(&s_m4, wsum);
+            __syncthreads();
+            if (threadIdx.x == 0 && s_m4)
+                atomicAdd(m4_count + g, s_m4);
+        }
+        __syncthreads();
+    }
+}
+
+cudaError_t launch_group_amax(const uint16_t *x, int64_t n_groups, int64_t nb,
+                              uint32_t *amax_bits, uint32_t *status, cudaStream_t s)
+{
+    if (n_groups == 0 || nb == 0)
+        return cudaSuccess;
+    const int64_t tiles = (nb + kNvTileBlocks - 1) / kNvTileBlocks;
+    dim3 grid((unsigned)(tiles < 0x7FFFFFFF ? tiles : 0x7FFFFFFF),
+              (unsigned)(n_groups < 65535 ? n_groups : 65535));
+    group_amax_kernel<<<grid, kNvThreads, 0, s>>>(reinterpret_cast<const uint4 *>(x), n_groups, nb,
+                                                  amax_bits, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_nvfp4_quant(const uint16_t *x, int64_t n_groups, int64_t nb, int four_six,
+                               const uint32_t *amax_bits, uint8_t *codes, uint8_t *scales,
+                               float *s2, uint32_t *mbits, int mbits_atomic,
+                               uint32_t *m4_count, cudaStream_t s)
+{
+    if (n_groups == 0)
+        return cudaSuccess;
+    const int64_t tiles = nb > 0 ? (nb + kNvTileBlocks - 1) / kNvTileBlocks : 1;
+    dim3 grid((unsigned)(tiles < 0x7FFFFFFF ? tiles : 0x7FFFFFFF),
+              (unsigned)(n_groups < 65535 ? n_groups : 65535));
+    const uint4 *xv = reinterpret_cast<const uint4 *>(x);
+    uint2 *cv = reinterpret_cast<uint2 *>(codes);
+    if (four_six)
+        nvfp4_quant_kernel<true><<<grid, kNvThreads, 0, s>>>(xv, n_groups, nb, amax_bits, cv, scales,
+                                                             s2, mbits, mbits_atomic, m4_count);
+    else
+        nvfp4_quant_kernel<false><<<grid, kNvThreads, 0, s>>>(xv, n_groups, nb, amax_bits, cv, scales,
+                                                              s2, mbits, mbits_atomic, m4_count);
+    return cudaGetLastError();
+}
+
+} // namespace mxq

@@ -1,0 +1,211 @@
+// verify.cu -- fused dequantize + relative-error reduction (sm_100a).
+//
+// Method (dabsLabs/Qwen3.8-Flash-Next-NVFP4, metric table: relative error
+// of the quantized experts against the bf16 source, per tensor, mean and
+// max over the census; azampatti/Qwen3.8-Flash-Next-FP4-Local-AZ, "The
+// shared expert": error of the MXFP8 tensors against the bf16 master):
+//   deq_i = RN32((q_i * D) * s2)   NVFP4 (q_i * D is exact in f16)
+//   deq_i = q_i * 2^e              MXFP4 / MXFP8 (exact)
+//   err_t = sum (x_i - deq_i)^2, ref_t = sum x_i^2 per tensor t.
+//
+// Fixed summation order: every tensor is cut into chunks of kVerifyChunk
+// elements; one CTA reduces one chunk with a fixed thread -> element map,
+// fp32 partials per block of 16 / 32, fp64 across blocks, a fixed shuffle
+// tree and a fixed warp order.  The finalize kernel adds the chunk
+// partials of each tensor in chunk order.  Results do not depend on
+// scheduling, so repeated runs are bit-identical.
+#include "mxq_device.cuh"
+#include "mxq_internal.h"
+#include "mxq.h"
+
+namespace mxq {
+
+__device__ __forceinline__ void accum_sq(float2 x, float2 deq, float2 &err, float2 &ref)
+{
+    const float2 e = __fadd2_rn(x, make_float2(-deq.x, -deq.y));
+    err = __ffma2_rn(e, e, err);
+    ref = __ffma2_rn(x, x, ref);
+}
+
+// One NVFP4 block of 16: x (2 x uint4), codes (uint2), scale byte, s2.
+__device__ __forceinline__ void nvfp4_block_sq(uint4 v0, uint4 v1, uint2 c, uint32_t sbyte, float s2,
+                                               double &err, double &ref)
+{
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    const uint32_t dh = e4m3x2_to_f16x2(sbyte);          // D in the low half
+    const uint32_t dd = __byte_perm(dh, 0, 0x1010);      // D in both halves
+    const float2 s22 = make_float2(s2, s2);
+    float2 e2 = make_float2(0.f, 0.f), r2 = make_float2(0.f, 0.f);
+    uint32_t q[8];
+    q[0] = e2m1x2_to_f16x2<0>(c.x);
+    q[1] = e2m1x2_to_f16x2<1>(c.x);
+    q[2] = e2m1x2_to_f16x2<2>(c.x);
+    q[3] = e2m1x2_to_f16x2<3>(c.x);
+    q[4] = e2m1x2_to_f16x2<0>(c.y);
+    q[5] = e2m1x2_to_f16x2<1>(c.y);
+    q[6] = e2m1x2_to_f16x2<2>(c.y);
+    q[7] = e2m1x2_to_f16x2<3>(c.y);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const float2 qd = f16x2_to_float2(hmul2_bits(q[j], dd));   // q * D, exact
+        const float2 deq = __fmul2_rn(qd, s22);
+        accum_sq(make_float2(bf16_lo(w[j]), bf16_hi(w[j])), deq, e2, r2);
+    }
+    err += (double)__fadd_rn(e2.x, e2.y);
+    ref += (double)__fadd_rn(r2.x, r2.y);
+}
+
+// One MX block of 32: x (4 x uint4), codes, scale byte.
+template <int FMT>
+__device__ __forceinline__ void mx_block_sq(const uint4 (&v)[4], const uint32_t *cw, uint32_t sbyte,
+                                            double &err, double &ref)
+{
+    // 2^(sbyte - 127); sbyte = 0 is the subnormal 2^-127
+    const float sc = sbyte ? __uint_as_float(sbyte << 23) : 0x1p-127f;
+    const float2 sc2 = make_float2(sc, sc);
+    const uint32_t w[16] = {v[0].x, v[0].y, v[0].z, v[0].w, v[1].x, v[1].y, v[1].z, v[1].w,
+                            v[2].x, v[2].y, v[2].z, v[2].w, v[3].x, v[3].y, v[3].z, v[3].w};
+    float2 e2 = make_float2(0.f, 0.f), r2 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        uint32_t qh;
+        if (FMT == MXQ_FMT_MXFP8) {
+            qh = e4m3x2_to_f16x2(j & 1 ? (cw[j >> 1] >> 16) : cw[j >> 1]);
+        } else {
+            const uint32_t word = cw[j >> 2];
+            switch (j & 3) {
+            case 0: qh = e2m1x2_to_f16x2<0>(word); break;
+            case 1: qh = e2m1x2_to_f16x2<1>(word); break;
+            case 2: qh = e2m1x2_to_f16x2<2>(word); break;
+            default: qh = e2m1x2_to_f16x2<3>(word); break;
+            }
+        }
+        const float2 deq = __fmul2_rn(f16x2_to_float2(qh), sc2);
+        accum_sq(make_float2(bf16_lo(w[j]), bf16_hi(w[j])), deq, e2, r2);
+    }
+    err += (double)__fadd_rn(e2.x, e2.y);
+    ref += (double)__fadd_rn(r2.x, r2.y);
+}
+
+__device__ __forceinline__ void cta_reduce_store(double err, double ref, double *out2)
+{
+    __shared__ double s_err[kVerifyThreads / 32], s_ref[kVerifyThreads / 32];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        err += __shfl_down_sync(0xFFFFFFFFu, err, off);
+        ref += __shfl_down_sync(0xFFFFFFFFu, ref, off);
+    }
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane == 0) {
+        s_err[warp] = err;
+        s_ref[warp] = ref;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double a = 0.0, b = 0.0;
+        for (int w = 0; w < kVerifyThreads / 32; ++w) {
+            a += s_err[w];
+            b += s_ref[w];
+        }
+        out2[0] = a;
+        out2[1] = b;
+    }
+    __syncthreads();
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(kVerifyThreads)
+verify_chunk_kernel(const uint16_t *__restrict__ x, const uint8_t *__restrict__ codes,
+                    const uint8_t *__restrict__ scales, const float *__restrict__ s2,
+                    int64_t n_tensors, int64_t tsize, int64_t chunks_per_tensor,
+                    int64_t tensors_per_scale, double *__restrict__ partials)
+{
+    constexpr int BLK = (FMT == MXQ_FMT_NVFP4) ? 16 : 32;
+    const int64_t n_chunks = n_tensors * chunks_per_tensor;
+    for (int64_t c = blockIdx.x; c < n_chunks; c += gridDim.x) {
+        const int64_t t = c / chunks_per_tensor;
+        const int64_t k = c - t * chunks_per_tensor;
+        const int64_t lo = k * kVerifyChunk;
+        const int64_t hi = min(lo + kVerifyChunk, tsize);
+        const int64_t nblk = (hi - lo) / BLK;
+        const int64_t first = (t * tsize + lo) / BLK;   // global block index
+        double err = 0.0, ref = 0.0;
+        for (int64_t i = threadIdx.x; i < nblk; i += kVerifyThreads) {
+            const int64_t gb = first + i;
+            if (FMT == MXQ_FMT_NVFP4) {
+                const uint4 *xv = reinterpret_cast<const uint4 *>(x) + gb * 2;
+                const uint4 v0 = __ldg(xv), v1 = __ldg(xv + 1);
+                const uint2 cc = __ldg(reinterpret_cast<const uint2 *>(codes) + gb);
+                const uint32_t sb = __ldg(scales + gb);
+                nvfp4_block_sq(v0, v1, cc, sb, __ldg(s2 + t / tensors_per_scale), err, ref);
+            } else {
+                const uint4 *xv = reinterpret_cast<const uint4 *>(x) + gb * 4;
+                uint4 v[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    v[q] = __ldg(xv + q);
+                uint32_t cw[8];
+                if (FMT == MXQ_FMT_MXFP8) {
+                    const uint4 *cv = reinterpret_cast<const uint4 *>(codes) + gb * 2;
+                    const uint4 c0 = __ldg(cv), c1 = __ldg(cv + 1);
+                    cw[0] = c0.x; cw[1] = c0.y; cw[2] = c0.z; cw[3] = c0.w;
+                    cw[4] = c1.x; cw[5] = c1.y; cw[6] = c1.z; cw[7] = c1.w;
+                } else {
+                    const uint4 c0 = __ldg(reinterpret_cast<const uint4 *>(codes) + gb);
+                    cw[0] = c0.x; cw[1] = c0.y; cw[2] = c0.z; cw[3] = c0.w;
+                }
+                mx_block_sq<FMT>(v, cw, __ldg(scales + gb), err, ref);
+            }
+        }
+        cta_reduce_store(err, ref, partials + 2 * c);
+    }
+}
+
+// One thread per tensor: chunk partials in chunk order.
+__global__ void verify_finalize_kernel(const double *__restrict__ partials, int64_t n_tensors,
+                                       int64_t chunks_per_tensor, double *__restrict__ sum_sq_err,
+                                       double *__restrict__ sum_sq_ref, double *__restrict__ relerr)
+{
+    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= n_tensors)
+        return;
+    double a = 0.0, b = 0.0;
+    const double *p = partials + 2 * t * chunks_per_tensor;
+    for (int64_t k = 0; k < chunks_per_tensor; ++k) {
+        a += p[2 * k];
+        b += p[2 * k + 1];
+    }
+    sum_sq_err[t] = a;
+    sum_sq_ref[t] = b;
+    if (relerr)
+        relerr[t] = (b > 0.0) ? sqrt(a) / sqrt(b) : (a > 0.0 ? __longlong_as_double(0x7FF0000000000000LL) : 0.0);
+}
+
+cudaError_t launch_verify(const uint16_t *x, const uint8_t *codes, const uint8_t *scales,
+                          const float *s2, int fmt, int64_t n_tensors, int64_t tsize,
+                          int64_t tensors_per_scale, double *partials, double *sum_sq_err,
+                          double *sum_sq_ref, double *relerr, cudaStream_t s)
+{
+    if (n_tensors == 0)
+        return cudaSuccess;
+    const int64_t cpt = tsize > 0 ? (tsize + kVerifyChunk - 1) / kVerifyChunk : 1;
+    int64_t n_chunks = n_tensors * cpt;
+    const unsigned grid = (unsigned)(n_chunks < 0x7FFFFFFF ? n_chunks : 0x7FFFFFFF);
+    if (fmt == MXQ_FMT_NVFP4)
+        verify_chunk_kernel<MXQ_FMT_NVFP4><<<grid, kVerifyThreads, 0, s>>>(
+            x, codes, scales, s2, n_tensors, tsize, cpt, tensors_per_scale, partials);
+    else if (fmt == MXQ_FMT_MXFP8)
+        verify_chunk_kernel<MXQ_FMT_MXFP8><<<grid, kVerifyThreads, 0, s>>>(
+            x, codes, scales, s2, n_tensors, tsize, cpt, tensors_per_scale, partials);
+    else
+        verify_chunk_kernel<MXQ_FMT_MXFP4><<<grid, kVerifyThreads, 0, s>>>(
+            x, codes, scales, s2, n_tensors, tsize, cpt, tensors_per_scale, partials);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return e;
+    const unsigned fgrid = (unsigned)((n_tensors + 127) / 128);
+    verify_finalize_kernel<<<fgrid, 128, 0, s>>>(partials, n_tensors, cpt, sum_sq_err, sum_sq_ref, relerr);
+    return cudaGetLastError();
+}
+
+} // namespace mxq

@@ -1,0 +1,207 @@
+"""Thin Python binding of libmxq.so (include/mxq.h).
+
+Argument marshalling only: every step of the quantizer and the verifier
+runs in the CUDA library.  Torch provides device memory and the current
+CUDA stream; tensors are passed by data pointer.  There is no fallback: if
+the library is missing the first call raises.
+
+Low-level functions carry the C names (``mxq_quantize_nvfp4`` ...) and take
+tensors for every buffer.  ``quantize_nvfp4``, ``quantize_mx``,
+``quantize_act`` and ``dequant_relerr`` allocate the outputs and workspace
+with torch and return them.
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmxq.so")
+
+MXQ_OK = 0
+STATUS_NAMES = {0: "ok", 1: "invalid argument", 2: "shape", 3: "align", 4: "workspace",
+                5: "cuda", 6: "unsupported"}
+DEV_NONFINITE_INPUT = 0x1
+DEV_WAIT_TIMEOUT = 0x2
+
+FMT = {"nvfp4": 0, "mxfp4": 1, "mxfp8": 2}
+SCALE_MODE = {"rtn": 0, "four_six": 1}
+OP = {"quantize_nvfp4": 0, "quantize_act": 1, "dequant_relerr": 2}
+
+EXPORTED = ("mxq_version", "mxq_status_string", "mxq_workspace_bytes", "mxq_quantize_nvfp4",
+            "mxq_quantize_mx", "mxq_quantize_act", "mxq_dequant_relerr")
+
+
+class MxqError(RuntimeError):
+    def __init__(self, fn, code):
+        super().__init__("%s failed: %s (%d)" % (fn, STATUS_NAMES.get(code, "?"), code))
+        self.code = code
+
+
+_lib = None
+
+
+def load(path=LIB_PATH):
+    """Load libmxq.so and declare its signatures (raises if missing)."""
+    global _lib
+    if _lib is not None and path == LIB_PATH:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError("libmxq.so is not built (%s): run `python -m mxfp_block_scaled_b200.build`"
+                           % path)
+    L = ctypes.CDLL(path)
+    vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+    L.mxq_version.restype = i32
+    L.mxq_version.argtypes = []
+    L.mxq_status_string.restype = ctypes.c_char_p
+    L.mxq_status_string.argtypes = [i32]
+    L.mxq_workspace_bytes.restype = sz
+    L.mxq_workspace_bytes.argtypes = [i32, i64, i64, i64]
+    L.mxq_quantize_nvfp4.restype = i32
+    L.mxq_quantize_nvfp4.argtypes = [vp, i64, i64, i64, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.mxq_quantize_mx.restype = i32
+    L.mxq_quantize_mx.argtypes = [vp, i64, i64, i32, i32, vp, vp, vp, vp]
+    L.mxq_quantize_act.restype = i32
+    L.mxq_quantize_act.argtypes = [vp, i64, i64, i32, vp, vp, vp, vp, vp, sz, vp]
+    L.mxq_dequant_relerr.restype = i32
+    L.mxq_dequant_relerr.argtypes = [vp, vp, vp, vp, i32, i64, i64, i64, i64, vp, vp, vp, vp, sz, vp]
+    if path == LIB_PATH:
+        _lib = L
+    return L
+
+
+def _p(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libmxq takes device tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(fn, rc):
+    if rc != MXQ_OK:
+        raise MxqError(fn, rc)
+
+
+def workspace_bytes(op, n, rows, cols):
+    return load().mxq_workspace_bytes(OP[op], n, rows, cols)
+
+
+def _workspace(op, n, rows, cols, device):
+    nbytes = workspace_bytes(op, n, rows, cols)
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device), nbytes
+
+
+# ---------------------------------------------------------------- C names --
+def mxq_quantize_nvfp4(x, n_groups, rows, cols, mode, codes, scales, s2, mbits, m4_count,
+                       status, workspace, stream=None):
+    rc = load().mxq_quantize_nvfp4(_p(x), n_groups, rows, cols, SCALE_MODE[mode], _p(codes),
+                                   _p(scales), _p(s2), _p(mbits), _p(m4_count), _p(status),
+                                   _p(workspace), workspace.numel() if workspace is not None else 0,
+                                   _stream(stream))
+    _check("mxq_quantize_nvfp4", rc)
+
+
+def mxq_quantize_mx(x, rows, cols, fmt, block, codes, scales, status, stream=None):
+    rc = load().mxq_quantize_mx(_p(x), rows, cols, FMT[fmt], block, _p(codes), _p(scales),
+                                _p(status), _stream(stream))
+    _check("mxq_quantize_mx", rc)
+
+
+def mxq_quantize_act(tokens, T, hidden, fmt, codes, scales, input_scale, status, workspace,
+                     stream=None):
+    rc = load().mxq_quantize_act(_p(tokens), T, hidden, FMT[fmt], _p(codes), _p(scales),
+                                 _p(input_scale), _p(status), _p(workspace),
+                                 workspace.numel() if workspace is not None else 0, _stream(stream))
+    _check("mxq_quantize_act", rc)
+
+
+def mxq_dequant_relerr(x, codes, scales, s2, fmt, n_tensors, rows, cols, tensors_per_scale,
+                       sum_sq_err, sum_sq_ref, relerr, workspace, stream=None):
+    rc = load().mxq_dequant_relerr(_p(x), _p(codes), _p(scales), _p(s2), FMT[fmt], n_tensors, rows,
+                                   cols, tensors_per_scale, _p(sum_sq_err), _p(sum_sq_ref),
+                                   _p(relerr), _p(workspace),
+                                   workspace.numel() if workspace is not None else 0,
+                                   _stream(stream))
+    _check("mxq_dequant_relerr", rc)
+
+
+# ------------------------------------------------------------ allocating --
+def _bf16(x):
+    if x.dtype != torch.bfloat16 or not x.is_contiguous():
+        raise ValueError("expected a contiguous bf16 tensor")
+    return x
+
+
+def quantize_nvfp4(x, mode="four_six", with_mbits=True, stream=None):
+    """x: bf16 [G, R, C] on the device.  Returns a dict of device tensors:
+    codes [G,R,C/2] u8, scales [G,R,C/16] u8, s2 [G] f32, mbits u32 words,
+    m4_count [G] i32-view of u32, status [1]."""
+    _bf16(x)
+    G, R, C = x.shape
+    dev = x.device
+    out = {
+        "codes": torch.empty((G, R, C // 2), dtype=torch.uint8, device=dev),
+        "scales": torch.empty((G, R, C // 16), dtype=torch.uint8, device=dev),
+        "s2": torch.empty(G, dtype=torch.float32, device=dev),
+        "mbits": torch.empty(((G * R * C // 16) + 31) // 32 or 1, dtype=torch.int32, device=dev)
+        if with_mbits else None,
+        "m4_count": torch.empty(max(G, 1), dtype=torch.int32, device=dev),
+        "status": torch.zeros(1, dtype=torch.int32, device=dev),
+    }
+    ws, _ = _workspace("quantize_nvfp4", G, R, C, dev)
+    mxq_quantize_nvfp4(x, G, R, C, mode, out["codes"], out["scales"], out["s2"], out["mbits"],
+                       out["m4_count"], out["status"], ws, stream)
+    return out
+
+
+def quantize_mx(x, fmt, stream=None):
+    """x: bf16 [..., C].  Returns dict codes, scales, status."""
+    _bf16(x)
+    C = x.shape[-1]
+    R = x.numel() // C if C else 0
+    dev = x.device
+    out = {
+        "codes": torch.empty(x.shape[:-1] + ((C // 2) if fmt == "mxfp4" else C,), dtype=torch.uint8,
+                             device=dev),
+        "scales": torch.empty(x.shape[:-1] + (C // 32,), dtype=torch.uint8, device=dev),
+        "status": torch.zeros(1, dtype=torch.int32, device=dev),
+    }
+    mxq_quantize_mx(x, R, C, fmt, 32, out["codes"], out["scales"], out["status"], stream)
+    return out
+
+
+def quantize_act(tokens, fmt, stream=None):
+    """tokens: bf16 [T, hidden].  NVFP4 returns input_scale too."""
+    _bf16(tokens)
+    T, H = tokens.shape
+    dev = tokens.device
+    blk = 16 if fmt == "nvfp4" else 32
+    out = {
+        "codes": torch.empty((T, H if fmt == "mxfp8" else H // 2), dtype=torch.uint8, device=dev),
+        "scales": torch.empty((T, H // blk), dtype=torch.uint8, device=dev),
+        "input_scale": torch.empty(1, dtype=torch.float32, device=dev),
+        "status": torch.zeros(1, dtype=torch.int32, device=dev),
+    }
+    ws, _ = _workspace("quantize_act", T, H, 0, dev)
+    mxq_quantize_act(tokens, T, H, fmt, out["codes"], out["scales"], out["input_scale"],
+                     out["status"], ws, stream)
+    return out
+
+
+def dequant_relerr(x, codes, scales, s2, fmt, n_tensors, rows, cols, tensors_per_scale=1,
+                   stream=None):
+    """Per-tensor fp64 (sum_sq_err, sum_sq_ref, relerr) on the device."""
+    dev = x.device
+    err = torch.empty(max(n_tensors, 1), dtype=torch.float64, device=dev)
+    ref = torch.empty_like(err)
+    rel = torch.empty_like(err)
+    ws, _ = _workspace("dequant_relerr", n_tensors, rows, cols, dev)
+    mxq_dequant_relerr(x, codes, scales, s2, fmt, n_tensors, rows, cols, tensors_per_scale, err,
+                       ref, rel, ws, stream)
+    return err[:n_tensors], ref[:n_tensors], rel[:n_tensors]

@@ -1,0 +1,108 @@
+"""The C-ABI library loads and exports every entry point include/mxq.h
+declares; host-side argument checks answer before any CUDA work (these
+calls need no GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from mxfp_block_scaled_b200 import build, mxq
+    build.build()
+    return mxq.load()
+
+
+def declared_functions():
+    with open(os.path.join(ROOT, "include", "mxq.h")) as f:
+        text = f.read()
+    return re.findall(r"MXQ_API\s+[\w\s\*]+?\b(mxq_\w+)\s*\(", text)
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("mxq_quantize_nvfp4", "mxq_quantize_mx", "mxq_quantize_act", "mxq_dequant_relerr",
+              "mxq_workspace_bytes", "mxq_status_string", "mxq_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from mxfp_block_scaled_b200 import mxq
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(mxq.EXPORTED) <= set(declared_functions())
+
+
+def test_version_and_status_strings(lib):
+    assert lib.mxq_version() >= 10000
+    for code in range(7):
+        s = lib.mxq_status_string(code)
+        assert s and isinstance(s, bytes)
+    assert lib.mxq_status_string(99) == b"unknown status"
+
+
+def test_workspace_sizes(lib):
+    # amax bits + arrival counters, each padded to 256 bytes
+    assert lib.mxq_workspace_bytes(0, 512, 1536, 2048) == 2 * 2048
+    assert lib.mxq_workspace_bytes(0, 1, 16, 16) == 512
+    assert lib.mxq_workspace_bytes(1, 4096, 2048, 0) == 512
+    # verifier: 16 bytes per chunk of 16384 elements per tensor
+    cpt = -(-768 * 2048 // 16384)
+    assert lib.mxq_workspace_bytes(2, 1024, 768, 2048) == (1024 * cpt * 16 + 255) // 256 * 256
+    assert lib.mxq_workspace_bytes(0, -1, 4, 16) == 0
+    assert lib.mxq_workspace_bytes(0, 1 << 40, 1 << 20, 1 << 20) == 0   # overflow
+
+
+def test_host_argument_errors_return_before_any_launch(lib):
+    vp = ctypes.c_void_p
+    fake = vp(0x1000)           # never dereferenced: every call below fails its checks first
+    # NVFP4: cols not a multiple of 16
+    assert lib.mxq_quantize_nvfp4(fake, 1, 4, 24, 1, fake, fake, fake, None, None, fake, fake,
+                                  4096, None) == 2
+    # negative sizes, bad mode
+    assert lib.mxq_quantize_nvfp4(fake, -1, 4, 16, 1, fake, fake, fake, None, None, fake, fake,
+                                  4096, None) == 1
+    assert lib.mxq_quantize_nvfp4(fake, 1, 4, 16, 7, fake, fake, fake, None, None, fake, fake,
+                                  4096, None) == 1
+    # null output / status
+    assert lib.mxq_quantize_nvfp4(fake, 1, 4, 16, 1, None, fake, fake, None, None, fake, fake,
+                                  4096, None) == 1
+    assert lib.mxq_quantize_nvfp4(fake, 1, 4, 16, 1, fake, fake, fake, None, None, None, fake,
+                                  4096, None) == 1
+    # misaligned input
+    assert lib.mxq_quantize_nvfp4(vp(0x1002), 1, 4, 16, 1, fake, fake, fake, None, None, fake,
+                                  fake, 4096, None) == 3
+    # workspace too small
+    assert lib.mxq_quantize_nvfp4(fake, 1, 4, 16, 1, fake, fake, fake, None, None, fake, fake,
+                                  8, None) == 4
+    # MX: block size other than 32, bad format, bad shape
+    assert lib.mxq_quantize_mx(fake, 4, 64, 2, 16, fake, fake, None, None) == 6
+    assert lib.mxq_quantize_mx(fake, 4, 64, 0, 32, fake, fake, None, None) == 1
+    assert lib.mxq_quantize_mx(fake, 4, 48, 2, 32, fake, fake, None, None) == 2
+    # verifier: missing s2 for NVFP4, tensors_per_scale < 1
+    assert lib.mxq_dequant_relerr(fake, fake, fake, None, 0, 2, 4, 16, 1, fake, fake, None, fake,
+                                  4096, None) == 1
+    assert lib.mxq_dequant_relerr(fake, fake, fake, fake, 0, 2, 4, 16, 0, fake, fake, None, fake,
+                                  4096, None) == 1
+    # activation: status required; NVFP4 needs input_scale
+    assert lib.mxq_quantize_act(fake, 4, 64, 0, fake, fake, fake, None, fake, 4096, None) == 1
+    assert lib.mxq_quantize_act(fake, 4, 64, 0, fake, fake, None, fake, fake, 4096, None) == 1
+
+
+def test_empty_inputs_are_no_ops(lib):
+    # zero groups / zero rows: nothing to do, success without touching memory
+    assert lib.mxq_quantize_nvfp4(None, 0, 4, 16, 1, None, None, None, None, None, None, None, 0,
+                                  None) == 0
+    assert lib.mxq_quantize_mx(None, 0, 64, 2, 32, None, None, None, None) == 0
+    assert lib.mxq_dequant_relerr(None, None, None, None, 2, 0, 4, 64, 1, None, None, None, None, 0,
+                                  None) == 0
+
+
+def test_product_path_refuses_to_run_without_the_library(tmp_path):
+    from mxfp_block_scaled_b200 import mxq
+    with pytest.raises(RuntimeError, match="not built"):
+        mxq.load(str(tmp_path / "missing.so"))

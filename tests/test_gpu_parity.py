@@ -1,0 +1,261 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle on the
+same seeded inputs.  Bit-exact on codes, scale bytes, global scales and the
+per-block M choice; verifier sums within 1e-6 relative."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mxfp_block_scaled_b200 import mxq, workloads
+
+pytestmark = pytest.mark.gpu
+
+RTOL_STATS = 1e-6
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _setup():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from mxfp_block_scaled_b200 import build
+    build.build()
+    mxq.load()
+    oracle.build()
+
+
+def bits(t):
+    return workloads.bf16_bits(t)
+
+
+def from_bits_np(b):
+    return (np.asarray(b, np.uint32) << 16).view(np.float32)
+
+
+def to_dev_bf16(bits_np):
+    return torch.from_numpy(np.ascontiguousarray(bits_np).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def mbits_to_bytes(words, n_blocks):
+    w = words.cpu().numpy().view(np.uint32)
+    b = np.unpackbits(w.view(np.uint8), bitorder="little")
+    return b[:n_blocks]
+
+
+def check_nvfp4(x_dev, mode="four_six", label=""):
+    G, R, C = x_dev.shape
+    out = mxq.quantize_nvfp4(x_dev, mode=mode)
+    torch.cuda.synchronize()
+    assert int(out["status"].item()) == 0
+    xb = bits(x_dev).reshape(G, R, C)
+    c, s, s2, m4 = oracle.quantize_nvfp4(xb, mode=1 if mode == "four_six" else 0)
+    gc = out["codes"].cpu().numpy()
+    gs = out["scales"].cpu().numpy()
+    gs2 = out["s2"].cpu().numpy()
+    assert np.array_equal(gs2.view(np.uint32), s2.view(np.uint32)), label + " s2"
+    bad = np.nonzero(gs.reshape(-1) != s.reshape(-1))[0]
+    assert bad.size == 0, "%s scales differ at blocks %s" % (label, bad[:10])
+    badc = np.nonzero((gc.reshape(-1, 8) != c.reshape(-1, 8)).any(1))[0]
+    assert badc.size == 0, "%s codes differ at blocks %s" % (label, badc[:10])
+    gm = mbits_to_bytes(out["mbits"], G * R * C // 16)
+    assert np.array_equal(gm, m4.reshape(-1)), label + " M bits"
+    cnt = out["m4_count"].cpu().numpy()[:G]
+    if mode == "four_six":
+        assert np.array_equal(cnt, m4.reshape(G, -1).sum(1)), label + " m4 count"
+    return out, (c, s, s2, m4)
+
+
+def check_verify(x_dev, codes, scales, s2, fmt, n_tensors, rows, cols, tps=1):
+    err, ref, rel = mxq.dequant_relerr(x_dev, codes, scales, s2, fmt, n_tensors, rows, cols, tps)
+    torch.cuda.synchronize()
+    oe, orf = oracle.dequant_relerr(bits(x_dev), codes.cpu().numpy(), scales.cpu().numpy(),
+                                    None if s2 is None else s2.cpu().numpy(), fmt, n_tensors,
+                                    rows, cols, tps)
+    err, ref, rel = err.cpu().numpy(), ref.cpu().numpy(), rel.cpu().numpy()
+    np.testing.assert_allclose(err, oe, rtol=RTOL_STATS, atol=0)
+    np.testing.assert_allclose(ref, orf, rtol=RTOL_STATS, atol=0)
+    np.testing.assert_allclose(rel, oracle.relerr_from_sums(oe, orf), rtol=RTOL_STATS, atol=0)
+    return err, ref, rel
+
+
+# ---------------------------------------------------------------- NVFP4 --
+def test_tiny_moe_layer_four_six_bit_exact_and_verified():
+    gu, dn = workloads.tiny_moe_layer(seed=0)
+    gu, dn = gu.cuda(), dn.cuda()
+    o1, _ = check_nvfp4(gu, label="gate_up")
+    o2, (_, _, _, m4) = check_nvfp4(dn, label="down")
+    E, R, H = gu.shape
+    check_verify(gu, o1["codes"], o1["scales"], o1["s2"], "nvfp4", 2 * E, R // 2, H, tps=2)
+    check_verify(dn, o2["codes"], o2["scales"], o2["s2"], "nvfp4", E, dn.shape[1], dn.shape[2])
+    assert 0.2 < m4.mean() < 0.7
+
+
+def test_tiny_moe_layer_rtn():
+    gu, _ = workloads.tiny_moe_layer(seed=1)
+    check_nvfp4(gu.cuda(), mode="rtn", label="rtn")
+
+
+@pytest.mark.parametrize("shape", [(3, 5, 48), (1, 1, 16), (2, 70, 256), (5, 3, 32 * 16),
+                                   (1, 33, 16 * 33), (7, 64, 64)])
+def test_ragged_shapes(shape):
+    g = torch.Generator().manual_seed(sum(shape))
+    x = (torch.randn(shape, generator=g) * 0.05).to(torch.bfloat16).cuda()
+    out, _ = check_nvfp4(x, label=str(shape))
+    G, R, C = shape
+    check_verify(x, out["codes"], out["scales"], out["s2"], "nvfp4", G, R, C)
+
+
+def test_degenerate_values():
+    G, R, C = 6, 4, 64
+    g = torch.Generator().manual_seed(7)
+    x = torch.randn((G, R, C), generator=g) * 0.02
+    x[0] = 0.0                                     # all-zero group: s2 = 0
+    x[1] = -0.0                                    # negative zeros
+    x[2] = x[2] * 1e-36                            # tiny: subnormal s2, slow path
+    x[3, 0, 0] = 3.0e38                            # huge: s2 outside the fast range
+    x[4, :, :16] = 0.0                             # zero blocks inside a normal group
+    x[4, 1, 16:32] = 1e-40                         # subnormal bf16 values
+    x[5] = torch.round(x[5] * 1000) / 1000         # many exact ties
+    x = x.to(torch.bfloat16)
+    xb = bits(x)
+    xb[1] = 0x8000
+    check_nvfp4(to_dev_bf16(xb), label="degenerate")
+    check_nvfp4(to_dev_bf16(xb), mode="rtn", label="degenerate rtn")
+
+
+def test_nonfinite_input_sets_status():
+    x = torch.randn((2, 4, 32)).to(torch.bfloat16).cuda()
+    x[1, 2, 5] = float("inf")
+    out = mxq.quantize_nvfp4(x)
+    torch.cuda.synchronize()
+    assert int(out["status"].item()) & mxq.DEV_NONFINITE_INPUT
+    x[1, 2, 5] = float("nan")
+    o2 = mxq.quantize_mx(x.view(8, 32), "mxfp8")
+    torch.cuda.synchronize()
+    assert int(o2["status"].item()) & mxq.DEV_NONFINITE_INPUT
+
+
+def test_deterministic_and_canaries():
+    gu, _ = workloads.tiny_moe_layer(seed=2)
+    gu = gu.cuda()
+    G, R, C = gu.shape
+    n = G * R * C
+    pad = 256
+    codes = torch.full((n // 2 + 2 * pad,), 0xA5, dtype=torch.uint8, device="cuda")
+    scales = torch.full((n // 16 + 2 * pad,), 0x5A, dtype=torch.uint8, device="cuda")
+    s2 = torch.full((G + 64,), -7.0, dtype=torch.float32, device="cuda")
+    mb = torch.full(((n // 16) // 32 + 64,), -1, dtype=torch.int32, device="cuda")
+    m4 = torch.full((G + 64,), -1, dtype=torch.int32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws, _ = mxq._workspace("quantize_nvfp4", G, R, C, "cuda")
+    results = []
+    for _ in range(2):
+        mxq.mxq_quantize_nvfp4(gu, G, R, C, "four_six", codes[pad:pad + n // 2],
+                               scales[pad:pad + n // 16], s2[:G], mb[:(n // 16) // 32], m4[:G], st, ws)
+        torch.cuda.synchronize()
+        results.append((codes.clone(), scales.clone(), s2.clone(), mb.clone()))
+    for a, b in zip(results[0], results[1]):
+        assert torch.equal(a, b)
+    assert torch.all(codes[:pad] == 0xA5) and torch.all(codes[pad + n // 2:] == 0xA5)
+    assert torch.all(scales[:pad] == 0x5A) and torch.all(scales[pad + n // 16:] == 0x5A)
+    assert torch.all(s2[G:] == -7.0) and torch.all(mb[(n // 16) // 32:] == -1) and torch.all(m4[G:] == -1)
+    # verifier: bit-identical across runs
+    e1 = mxq.dequant_relerr(gu, codes[pad:pad + n // 2], scales[pad:pad + n // 16], s2[:G], "nvfp4",
+                            2 * G, R // 2, C, 2)
+    e2 = mxq.dequant_relerr(gu, codes[pad:pad + n // 2], scales[pad:pad + n // 16], s2[:G], "nvfp4",
+                            2 * G, R // 2, C, 2)
+    for a, b in zip(e1, e2):
+        assert torch.equal(a, b)
+
+
+# ------------------------------------------------------------------- MX --
+@pytest.mark.parametrize("fmt", ["mxfp8", "mxfp4"])
+def test_shared_expert_mx_bit_exact_dense_and_padded(fmt):
+    for padded in (False, True):
+        gu, dn = workloads.shared_expert_layer(seed=4, inter=320, hidden=512, pad_from=160,
+                                               padded=padded)
+        for t in (gu, dn):
+            td = t.cuda()
+            out = mxq.quantize_mx(td, fmt)
+            torch.cuda.synchronize()
+            c, s = oracle.quantize_mx(bits(td), fmt)
+            assert np.array_equal(out["codes"].cpu().numpy(), c)
+            assert np.array_equal(out["scales"].cpu().numpy(), s)
+            check_verify(td, out["codes"], out["scales"], None, fmt, 1, *td.shape)
+        if padded:
+            o = mxq.quantize_mx(gu.cuda(), fmt)
+            assert not o["codes"][160:320].any() and not o["scales"][160:320].any()
+
+
+def _all_bf16_in(lo, hi):
+    b = np.arange(0, 0x7F80, dtype=np.uint32)
+    f = (b << 16).view(np.float32)
+    sel = (f >= lo) & (f <= hi)
+    return b[sel].astype(np.uint16)
+
+
+@pytest.mark.parametrize("fmt,qmax", [("mxfp8", 448.0), ("mxfp4", 6.0)])
+def test_every_bf16_value_converts_like_the_oracle(fmt, qmax):
+    """Blocks whose first element is qmax (so e = 0) carry every bf16 value
+    in [0, qmax] and its negative: the hardware conversion of every such
+    input equals the oracle's nearest-even rounding."""
+    vals = _all_bf16_in(0.0, qmax)
+    vals = np.concatenate([vals, vals | 0x8000])
+    per = 31
+    nblk = -(-vals.size // per)
+    x = np.zeros((nblk, 32), np.uint16)
+    qbits = np.float32(qmax).view(np.uint32) >> 16
+    x[:, 0] = qbits
+    flat = x[:, 1:].reshape(-1)
+    flat[:vals.size] = vals
+    x[:, 1:] = flat.reshape(nblk, per)
+    xd = to_dev_bf16(x)
+    out = mxq.quantize_mx(xd, fmt)
+    torch.cuda.synchronize()
+    c, s = oracle.quantize_mx(x, fmt)
+    assert np.all(s == 127)
+    assert np.array_equal(out["scales"].cpu().numpy(), s)
+    assert np.array_equal(out["codes"].cpu().numpy(), c)
+
+
+@pytest.mark.parametrize("fmt", ["mxfp8", "mxfp4"])
+def test_every_bf16_amax_gives_the_exponent_rule(fmt):
+    """One block per positive finite bf16 value (and the subnormals): block
+    amax = that value; scale bytes equal the oracle's for all of them."""
+    vals = np.arange(1, 0x7F80, dtype=np.uint16)
+    x = np.zeros((vals.size, 32), np.uint16)
+    x[:, 3] = vals
+    x[:, 7] = vals | 0x8000
+    xd = to_dev_bf16(x)
+    out = mxq.quantize_mx(xd, fmt)
+    torch.cuda.synchronize()
+    c, s = oracle.quantize_mx(x, fmt)
+    assert np.array_equal(out["scales"].cpu().numpy(), s)
+    assert np.array_equal(out["codes"].cpu().numpy(), c)
+
+
+# ---------------------------------------------------------- activations --
+@pytest.mark.parametrize("T", [1, 16, 256])
+def test_activation_tiles(T):
+    a = workloads.activation_tile(T, seed=T).cuda()
+    o = mxq.quantize_act(a, "nvfp4")
+    torch.cuda.synchronize()
+    assert int(o["status"].item()) == 0
+    c, s, s2, _ = oracle.quantize_nvfp4(bits(a).reshape(1, T, -1), mode=0)
+    assert o["input_scale"].cpu().numpy().view(np.uint32)[0] == s2.view(np.uint32)[0]
+    assert np.array_equal(o["codes"].cpu().numpy(), c.reshape(T, -1))
+    assert np.array_equal(o["scales"].cpu().numpy(), s.reshape(T, -1))
+    for fmt in ("mxfp8", "mxfp4"):
+        o = mxq.quantize_act(a, fmt)
+        torch.cuda.synchronize()
+        c, s = oracle.quantize_mx(bits(a), fmt)
+        assert np.array_equal(o["codes"].cpu().numpy(), c)
+        assert np.array_equal(o["scales"].cpu().numpy(), s)
+
+
+def test_activation_input_scale_is_amax_over_2688_not_amax_over_6():
+    a = workloads.activation_tile(16, seed=3).cuda()
+    o = mxq.quantize_act(a, "nvfp4")
+    amax = a.float().abs().max().item()
+    got = float(o["input_scale"].item())
+    assert got == float(np.float32(amax) / np.float32(2688.0))
+    assert abs(got - amax / 6) > 0.1 * amax / 6
