@@ -159,10 +159,10 @@ def device_uuid():
 class Layer:
     """Device-resident layer and preallocated outputs."""
 
-    def __init__(self, seed, device):
+    def __init__(self, seed, device, experts=EXPERTS):
         from mxfp_block_scaled_b200 import mxq, workloads
         self.mxq = mxq
-        self.gu, self.dn, _ = workloads.full_moe_layer(seed=seed, device=device, experts=EXPERTS,
+        self.gu, self.dn, _ = workloads.full_moe_layer(seed=seed, device=device, experts=experts,
                                                         hidden=HIDDEN, inter=INTER)
         self.n_elems = self.gu.numel() + self.dn.numel()
         self.out = {}
@@ -339,6 +339,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the e2e and CPU-baseline legs (profiling runs)")
+    ap.add_argument("--experts", type=int, default=EXPERTS,
+                    help="experts in the layer; fewer than 512 only for small profiling captures")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "mine" else args.warmup
 
@@ -360,7 +362,7 @@ def main():
     build.build()
     mxq.load()
 
-    layer = Layer(seed=rank, device=device)
+    layer = Layer(seed=rank, device=device, experts=args.experts)
     torch.cuda.synchronize()
 
     def barrier():
@@ -414,7 +416,9 @@ def main():
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "experts": EXPERTS, "hidden": HIDDEN, "inter": INTER,
+        "config": {"workload": WORKLOAD if args.experts == EXPERTS else
+                   "PROFILING CASE, %d experts (not the headline workload)" % args.experts,
+                   "experts": args.experts, "hidden": HIDDEN, "inter": INTER,
                    "elements_per_gpu": layer.n_elems, "algorithmic_bytes_per_element": STEP_BYTES_PER_ELEM,
                    "l2": "inputs 4.8 GB per GPU, larger than L2; no flush",
                    "fraction_of_peak": value / peak, "peak_gbs": peak, "peak_kind": peak_kind,

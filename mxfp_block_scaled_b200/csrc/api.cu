@@ -108,12 +108,28 @@ mxq_status mxq_quantize_nvfp4(const uint16_t *x, int64_t n_groups, int64_t rows,
     const int64_t nb = gsize / 16;
     const int64_t total_blocks = total / 16;
     uint32_t *amax_bits = static_cast<uint32_t *>(workspace);
-    cudaError_t e = cudaMemsetAsync(amax_bits, 0, (size_t)n_groups * sizeof(uint32_t), stream);
+    uint32_t *arrive = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(workspace) +
+                                                    need / 2);
+    // amax bits and arrival counters start at zero
+    cudaError_t e = cudaMemsetAsync(workspace, 0, need, stream);
     if (e == cudaSuccess && m4_count)
         e = cudaMemsetAsync(m4_count, 0, (size_t)n_groups * sizeof(uint32_t), stream);
+    if (e != cudaSuccess)
+        return MXQ_ERR_CUDA;
+    // single pass (one HBM read of x) when the shape allows it
+    e = launch_nvfp4_fused(x, n_groups, nb, mode == MXQ_SCALE_FOUR_SIX, amax_bits, arrive, codes,
+                           scales, s2, mbits, m4_count, status, stream);
+    if (e == cudaSuccess)
+        return MXQ_OK;
+    if (e != cudaErrorNotSupported)
+        return MXQ_ERR_CUDA;
+    (void)cudaGetLastError();
+    // two passes: group amax, then the block quantizer
     const int mbits_atomic = (nb % 32) != 0;
-    if (e == cudaSuccess && mbits && (mbits_atomic || nb == 0 || total_blocks % 32 != 0))
+    if (mbits && mbits_atomic)
         e = cudaMemsetAsync(mbits, 0, (size_t)((total_blocks + 31) / 32) * sizeof(uint32_t), stream);
+    else
+        e = cudaSuccess;
     if (e == cudaSuccess)
         e = launch_group_amax(x, n_groups, nb, amax_bits, status, stream);
     if (e == cudaSuccess)

@@ -27,32 +27,49 @@ __device__ __forceinline__ uint32_t abs_max_bits(uint32_t acc, uint32_t w)
 __device__ __forceinline__ uint32_t fold_halves(uint32_t m) { return max(m & 0xFFFFu, m >> 16); }
 
 // ---- packed conversions (PTX ISA: cvt with .e2m1x2 / .e4m3x2) ------------
-// Eight fp32 values -> eight E2M1 codes in one word, element 2j in the low
-// nibble of byte j.  Round to nearest even, saturating at +-6, sign kept.
-__device__ __forceinline__ uint32_t e2m1x8(float2 p0, float2 p1, float2 p2, float2 p3)
+// Two fp32 values -> one byte of two E2M1 codes (lo in the low nibble),
+// round to nearest even, saturating at +-6, sign kept; zero-extended.
+// Bytes move between .b8 and 32-bit registers only with cvt.u8.u32 /
+// cvt.u32.u8: vector moves of .b8 registers ({b0, b1, ...}) corrupted
+// bytes when a packed word was unpacked again in the same kernel.
+__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi)
 {
     uint32_t out;
-    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
-        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
-        : "=r"(out)
-        : "f"(p0.x), "f"(p0.y), "f"(p1.x), "f"(p1.y), "f"(p2.x), "f"(p2.y), "f"(p3.x), "f"(p3.y));
+    asm("{\n\t.reg .b8 t;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t, %2, %1;\n\t"
+        "cvt.u32.u8 %0, t;\n\t}"
+        : "=r"(out) : "f"(lo), "f"(hi));
     return out;
 }
 
-// Byte j of `w` (two E2M1 codes) -> f16x2 values, low nibble in the low half.
-template <int J>
-__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t w)
+// Eight fp32 values -> eight E2M1 codes in one word, element 2j in the low
+// nibble of byte j.
+__device__ __forceinline__ uint32_t e2m1x8(float2 p0, float2 p1, float2 p2, float2 p3)
+{
+    const uint32_t b0 = e2m1x2(p0.x, p0.y), b1 = e2m1x2(p1.x, p1.y);
+    const uint32_t b2 = e2m1x2(p2.x, p2.y), b3 = e2m1x2(p3.x, p3.y);
+    return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
+}
+
+// Low byte of `v` (two E2M1 codes) -> f16x2, low nibble in the low half.
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t v)
 {
     uint32_t out;
-    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-        "mov.b32 {b0, b1, b2, b3}, %1;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %0, b" "%2" ";\n\t}"
-        : "=r"(out) : "r"(w), "n"(J));
+    asm("{\n\t.reg .b8 t;\n\t"
+        "cvt.u8.u32 t, %1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+        : "=r"(out) : "r"(v));
     return out;
+}
+
+// The four bytes of `w` (eight E2M1 codes) -> four f16x2 values; pair j
+// holds the codes of byte j.  Exact.
+__device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t (&h)[4])
+{
+    h[0] = e2m1x2_to_f16x2(w);
+    h[1] = e2m1x2_to_f16x2(w >> 8);
+    h[2] = e2m1x2_to_f16x2(w >> 16);
+    h[3] = e2m1x2_to_f16x2(w >> 24);
 }
 
 // Two fp32 -> two E4M3 bytes (lo from `lo`, hi from `hi`), round to nearest
@@ -125,6 +142,60 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p)
 __device__ __forceinline__ void red_release_add_u32(uint32_t *p, uint32_t v)
 {
     asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// ---- shared-memory barriers and bulk copies (PTX ISA, sm_90+) -----------
+__device__ __forceinline__ uint32_t smem_addr(const void *p)
+{
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+                 ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
+}
+
+// One bulk copy global -> shared (16-byte aligned, size a multiple of 16),
+// completing `bytes` transactions on `bar`.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
+
+// Wait for phase `parity` of `bar`, giving up after `limit` polls.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, uint32_t limit)
+{
+    for (uint32_t i = 0; i < limit; ++i)
+        if (mbar_try_wait(bar, parity))
+            return true;
+    return false;
 }
 
 } // namespace mxq

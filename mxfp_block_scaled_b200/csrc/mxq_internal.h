@@ -14,6 +14,9 @@ constexpr float kGlobalDivisor = 2688.0f;  // 6 * 448: weight_scale_2 / input_sc
 constexpr int kNvThreads = 256;
 constexpr int kNvTileBlocks = 512;
 
+// Single-pass NVFP4 schedule: one cooperative CTA per SM.
+constexpr int kFusedThreads = 512;
+
 // Verifier: one CTA reduces one chunk of a tensor.
 constexpr int kVerifyThreads = 256;
 constexpr int64_t kVerifyChunk = 16384;  // elements per chunk (multiple of 32)
@@ -30,6 +33,10 @@ cudaError_t launch_nvfp4_quant(const uint16_t *x, int64_t n_groups, int64_t nb, 
                                const uint32_t *amax_bits, uint8_t *codes, uint8_t *scales,
                                float *s2, uint32_t *mbits, int mbits_atomic,
                                uint32_t *m4_count, cudaStream_t s);
+cudaError_t launch_nvfp4_fused(const uint16_t *x, int64_t n_groups, int64_t nb, int four_six,
+                               uint32_t *amax_bits, uint32_t *arrive, uint8_t *codes,
+                               uint8_t *scales, float *s2, uint32_t *mbits, uint32_t *m4_count,
+                               uint32_t *status, cudaStream_t s);
 cudaError_t launch_mx_quant(const uint16_t *x, int64_t nblk32, int fmt, uint8_t *codes,
                             uint8_t *scales, uint32_t *status, cudaStream_t s);
 cudaError_t launch_verify(const uint16_t *x, const uint8_t *codes, const uint8_t *scales,

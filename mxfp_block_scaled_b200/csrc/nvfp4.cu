@@ -103,12 +103,10 @@ struct Plan {
     float b;       // sum q_i^2 (exact)
 };
 
-// q pair (f16x2) of byte J of `w`: accumulate B in f16 (exact: <= 8 terms of
-// quarter-integers <= 36 per half) and -A in fp32 pairs.
-template <int J>
-__device__ __forceinline__ void accum_pair(uint32_t w, float2 nx, float2 &acc, uint32_t &bh)
+// q pair (f16x2): accumulate B in f16 (exact: <= 8 terms of quarter-
+// integers <= 36 per half) and -A in fp32 pairs.
+__device__ __forceinline__ void accum_pair(uint32_t qh, float2 nx, float2 &acc, uint32_t &bh)
 {
-    const uint32_t qh = e2m1x2_to_f16x2<J>(w);
     bh = hfma2_bits(qh, qh, bh);
     acc = __ffma2_rn(nx, f16x2_to_float2(qh), acc);
 }
@@ -139,14 +137,12 @@ __device__ __forceinline__ Plan make_plan(const float2 (&nx)[8], float D, float 
     p.codes.y = e2m1x8(y[4], y[5], y[6], y[7]);
     float2 acc = make_float2(0.0f, 0.0f);
     uint32_t bh = 0u;
-    accum_pair<0>(p.codes.x, nx[0], acc, bh);
-    accum_pair<1>(p.codes.x, nx[1], acc, bh);
-    accum_pair<2>(p.codes.x, nx[2], acc, bh);
-    accum_pair<3>(p.codes.x, nx[3], acc, bh);
-    accum_pair<0>(p.codes.y, nx[4], acc, bh);
-    accum_pair<1>(p.codes.y, nx[5], acc, bh);
-    accum_pair<2>(p.codes.y, nx[6], acc, bh);
-    accum_pair<3>(p.codes.y, nx[7], acc, bh);
+    uint32_t q[8];
+    e2m1x8_to_f16x2(p.codes.x, *reinterpret_cast<uint32_t(*)[4]>(&q[0]));
+    e2m1x8_to_f16x2(p.codes.y, *reinterpret_cast<uint32_t(*)[4]>(&q[4]));
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        accum_pair(q[j], nx[j], acc, bh);
     p.a_neg = __fadd_rn(acc.x, acc.y);
     const float2 bf = f16x2_to_float2(bh);
     p.b = __fadd_rn(bf.x, bf.y);
@@ -287,6 +283,189 @@ nvfp4_quant_kernel(const uint4 *__restrict__ x, int64_t n_groups, int64_t nb,
     }
 }
 
+// ---------------------------------------------------------------------------
+// Single-pass schedule: nvfp4_fused_kernel.
+//
+// A cooperative persistent grid of one CTA per SM.  Every group's blocks are
+// cut into one contiguous slice per CTA (a multiple of 32 blocks, so a warp's
+// M bits fill one word).  Each CTA walks the groups in order with a ring of
+// `stages` shared-memory buffers filled by bulk copies:
+//   iteration i:  (A) wait for slice i in smem, reduce its amax, publish it
+//                     (atomicMax, then a release increment of arrive[i]);
+//                 (B) for j = i - lookahead: wait until all CTAs published
+//                     group j (acquire, bounded), derive s2, quantize slice j
+//                     from smem, then refill its buffer with slice j+stages.
+// W is read from HBM once; the amax dependency of a group is resolved
+// `lookahead` iterations after its data arrived, so the wait is normally
+// already satisfied.  Every wait is bounded: on time-out the CTA sets
+// MXQ_DEV_WAIT_TIMEOUT, waits (bounded) for its own copies in flight and
+// returns.
+// ---------------------------------------------------------------------------
+struct FusedArgs {
+    const uint16_t *x;
+    int64_t n_groups, nb, slice;   // blocks per group, blocks per CTA slice
+    int stages, lookahead;
+    uint32_t *amax_bits, *arrive, *status;
+    uint2 *codes;
+    uint8_t *scales;
+    float *s2_out;
+    uint32_t *mbits, *m4_count;
+};
+
+constexpr uint32_t kSpinLimit = 1u << 22;   // polls of a flag / barrier before giving up
+
+template <bool FOUR_SIX>
+__global__ void __launch_bounds__(kFusedThreads, 1)
+nvfp4_fused_kernel(const FusedArgs a)
+{
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
+    uint8_t *buf = smem + 128;
+    __shared__ uint32_t s_red[kFusedThreads / 32];
+    __shared__ GroupConst s_gc;
+    __shared__ uint32_t s_m4;
+    __shared__ int s_abort;
+
+    const int tid = threadIdx.x, lane = tid & 31;
+    const uint32_t P = gridDim.x;
+    const int64_t my_lo = (int64_t)blockIdx.x * a.slice;
+    const int64_t my_n = max((int64_t)0, min(a.slice, a.nb - my_lo));
+    const uint32_t bytes = (uint32_t)(my_n * 32);
+    const int64_t stage_bytes = a.slice * 32;
+    const int L = a.stages, LA = a.lookahead;
+    const int64_t G = a.n_groups;
+
+    if (tid == 0) {
+        for (int k = 0; k < L; ++k)
+            mbar_init(bars + k, 1);
+        fence_mbar_init();
+        s_abort = 0;
+        s_m4 = 0;
+    }
+    __syncthreads();
+
+    auto issue = [&](int64_t g) {   // thread 0: load slice of group g into stage g % L
+        if (bytes == 0)
+            return;
+        const int st = (int)(g % L);
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(bars + st, bytes);
+        bulk_g2s(buf + st * stage_bytes, a.x + (g * a.nb + my_lo) * 16, bytes, bars + st);
+    };
+    if (tid == 0)
+        for (int64_t g = 0; g < G && g < L; ++g)
+            issue(g);
+    int64_t issued = G < L ? G : L;   // groups whose slice load was issued
+    int64_t landed = 0;               // groups whose slice load was waited for
+
+    for (int64_t i = 0; i < G + LA; ++i) {
+        // (A) amax of my slice of group i, published to the other CTAs
+        if (i < G) {
+            const int st = (int)(i % L);
+            uint32_t m = 0;
+            if (bytes) {
+                if (!mbar_wait_bounded(bars + st, (uint32_t)((i / L) & 1), kSpinLimit))
+                    s_abort = 1;
+                else
+                    landed = i + 1;
+                const uint4 *v = reinterpret_cast<const uint4 *>(buf + st * stage_bytes);
+                for (int64_t k = tid; k < my_n * 2; k += kFusedThreads) {
+                    const uint4 q = v[k];
+                    m = abs_max_bits(m, q.x);
+                    m = abs_max_bits(m, q.y);
+                    m = abs_max_bits(m, q.z);
+                    m = abs_max_bits(m, q.w);
+                }
+            }
+            const uint32_t r = __reduce_max_sync(0xFFFFFFFFu, fold_halves(m));
+            if (lane == 0)
+                s_red[tid >> 5] = r;
+            __syncthreads();
+            if (tid == 0) {
+                uint32_t mx = 0;
+                for (int w = 0; w < kFusedThreads / 32; ++w)
+                    mx = max(mx, s_red[w]);
+                if (mx)
+                    atomicMax(a.amax_bits + i, mx);
+                if (mx >= 0x7F80u)
+                    atomicOr(a.status, MXQ_DEV_NONFINITE_INPUT);
+                red_release_add_u32(a.arrive + i, 1u);
+            }
+        }
+        // (B) quantize my slice of group j once every CTA published it
+        const int64_t j = i - LA;
+        if (j >= 0) {
+            if (tid == 0) {
+                uint32_t spins = 0;
+                while (ld_acquire_u32(a.arrive + j) < P) {
+                    if (++spins > kSpinLimit) {
+                        s_abort = 1;
+                        break;
+                    }
+                    __nanosleep(64);
+                }
+                const uint32_t am = *reinterpret_cast<volatile uint32_t *>(a.amax_bits + j);
+                s_gc = make_group_const(am);
+                if (blockIdx.x == 0)
+                    a.s2_out[j] = s_gc.s2;
+            }
+            __syncthreads();
+            if (s_abort)
+                break;
+            const GroupConst gc = s_gc;
+            const int st = (int)(j % L);
+            const uint4 *v = reinterpret_cast<const uint4 *>(buf + st * stage_bytes);
+            uint32_t my_m4 = 0;
+            for (int64_t k0 = 0; k0 < my_n; k0 += kFusedThreads) {
+                const int64_t k = k0 + tid;
+                const bool live = k < my_n;
+                BlockOut o;
+                o.m4 = false;
+                const int64_t gb = j * a.nb + my_lo + k;
+                if (live) {
+                    o = quantize_block<FOUR_SIX>(v[2 * k], v[2 * k + 1], gc);
+                    a.codes[gb] = o.codes;
+                    a.scales[gb] = (uint8_t)o.scale;
+                }
+                if (a.mbits) {
+                    const uint32_t word = __ballot_sync(0xFFFFFFFFu, o.m4);
+                    if (lane == 0 && k0 + tid - lane < my_n)
+                        a.mbits[(gb - lane) >> 5] = word;
+                }
+                my_m4 += o.m4 ? 1u : 0u;
+            }
+            if (FOUR_SIX && a.m4_count) {
+                const uint32_t wsum = __reduce_add_sync(0xFFFFFFFFu, my_m4);
+                if (lane == 0 && wsum)
+                    atomicAdd(&s_m4, wsum);
+            }
+            __syncthreads();   // every thread is done with stage st
+            if (tid == 0) {
+                if (FOUR_SIX && a.m4_count && s_m4) {
+                    atomicAdd(a.m4_count + j, s_m4);
+                    s_m4 = 0;
+                }
+                if (j + L < G)
+                    issue(j + L);
+            }
+            if (j + L < G)
+                ++issued;
+        }
+        if (i < G) {
+            __syncthreads();
+            if (s_abort)
+                break;
+        }
+    }
+    if (s_abort && tid == 0) {
+        atomicOr(a.status, MXQ_DEV_WAIT_TIMEOUT);
+        // let this CTA's copies in flight land before its smem is released
+        if (bytes)
+            for (int64_t g = landed; g < issued; ++g)
+                mbar_wait_bounded(bars + (g % L), (uint32_t)((g / L) & 1), kSpinLimit);
+    }
+}
+
 cudaError_t launch_group_amax(const uint16_t *x, int64_t n_groups, int64_t nb,
                               uint32_t *amax_bits, uint32_t *status, cudaStream_t s)
 {
@@ -298,6 +477,76 @@ cudaError_t launch_group_amax(const uint16_t *x, int64_t n_groups, int64_t nb,
     group_amax_kernel<<<grid, kNvThreads, 0, s>>>(reinterpret_cast<const uint4 *>(x), n_groups, nb,
                                                   amax_bits, status);
     return cudaGetLastError();
+}
+
+static int sm_count()
+{
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 0;
+    return n;
+}
+
+// Returns cudaErrorNotSupported (and launches nothing) when the shape or the
+// device does not suit the single-pass schedule; the caller then takes the
+// two-pass path.
+cudaError_t launch_nvfp4_fused(const uint16_t *x, int64_t n_groups, int64_t nb, int four_six,
+                               uint32_t *amax_bits, uint32_t *arrive, uint8_t *codes,
+                               uint8_t *scales, float *s2, uint32_t *mbits, uint32_t *m4_count,
+                               uint32_t *status, cudaStream_t s)
+{
+    if (n_groups <= 0 || nb <= 0 || nb % 32 != 0)
+        return cudaErrorNotSupported;
+    int dev = 0, coop = 0, max_optin = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+        return cudaErrorNotSupported;
+    const int sms = sm_count();
+    if (!coop || sms <= 0)
+        return cudaErrorNotSupported;
+    int64_t slice = (nb + sms - 1) / sms;
+    slice = (slice + 31) / 32 * 32;
+    const int64_t slice_bytes = slice * 32;
+    const int64_t avail = (int64_t)max_optin - 128 - 1024;   // barriers + static smem margin
+    int64_t L = avail / slice_bytes;
+    if (L < 1)
+        return cudaErrorNotSupported;
+    if (L > 8)
+        L = 8;
+    if (L > n_groups)
+        L = n_groups;
+    const int LA = L >= 4 ? 2 : (L >= 2 ? 1 : 0);
+    const size_t dyn = 128 + (size_t)(L * slice_bytes);
+    const void *fn = four_six ? (const void *)nvfp4_fused_kernel<true> : (const void *)nvfp4_fused_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
+    if (e != cudaSuccess)
+        return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kFusedThreads, dyn);
+    if (e != cudaSuccess)
+        return e;
+    if (per_sm < 1)
+        return cudaErrorNotSupported;
+    FusedArgs args;
+    args.x = x;
+    args.n_groups = n_groups;
+    args.nb = nb;
+    args.slice = slice;
+    args.stages = (int)L;
+    args.lookahead = LA;
+    args.amax_bits = amax_bits;
+    args.arrive = arrive;
+    args.status = status;
+    args.codes = reinterpret_cast<uint2 *>(codes);
+    args.scales = scales;
+    args.s2_out = s2;
+    args.mbits = mbits;
+    args.m4_count = four_six ? m4_count : nullptr;
+    void *params[] = {&args};
+    return cudaLaunchCooperativeKernel(fn, dim3((unsigned)sms), dim3(kFusedThreads), params, dyn, s);
 }
 
 cudaError_t launch_nvfp4_quant(const uint16_t *x, int64_t n_groups, int64_t nb, int four_six,

@@ -37,14 +37,8 @@ __device__ __forceinline__ void nvfp4_block_sq(uint4 v0, uint4 v1, uint2 c, uint
     const float2 s22 = make_float2(s2, s2);
     float2 e2 = make_float2(0.f, 0.f), r2 = make_float2(0.f, 0.f);
     uint32_t q[8];
-    q[0] = e2m1x2_to_f16x2<0>(c.x);
-    q[1] = e2m1x2_to_f16x2<1>(c.x);
-    q[2] = e2m1x2_to_f16x2<2>(c.x);
-    q[3] = e2m1x2_to_f16x2<3>(c.x);
-    q[4] = e2m1x2_to_f16x2<0>(c.y);
-    q[5] = e2m1x2_to_f16x2<1>(c.y);
-    q[6] = e2m1x2_to_f16x2<2>(c.y);
-    q[7] = e2m1x2_to_f16x2<3>(c.y);
+    e2m1x8_to_f16x2(c.x, *reinterpret_cast<uint32_t(*)[4]>(&q[0]));
+    e2m1x8_to_f16x2(c.y, *reinterpret_cast<uint32_t(*)[4]>(&q[4]));
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         const float2 qd = f16x2_to_float2(hmul2_bits(q[j], dd));   // q * D, exact
@@ -66,20 +60,17 @@ __device__ __forceinline__ void mx_block_sq(const uint4 (&v)[4], const uint32_t 
     const uint32_t w[16] = {v[0].x, v[0].y, v[0].z, v[0].w, v[1].x, v[1].y, v[1].z, v[1].w,
                             v[2].x, v[2].y, v[2].z, v[2].w, v[3].x, v[3].y, v[3].z, v[3].w};
     float2 e2 = make_float2(0.f, 0.f), r2 = make_float2(0.f, 0.f);
+    uint32_t q4[16];
+    if (FMT == MXQ_FMT_MXFP4) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            e2m1x8_to_f16x2(cw[k], *reinterpret_cast<uint32_t(*)[4]>(&q4[4 * k]));
+    }
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
-        uint32_t qh;
-        if (FMT == MXQ_FMT_MXFP8) {
-            qh = e4m3x2_to_f16x2(j & 1 ? (cw[j >> 1] >> 16) : cw[j >> 1]);
-        } else {
-            const uint32_t word = cw[j >> 2];
-            switch (j & 3) {
-            case 0: qh = e2m1x2_to_f16x2<0>(word); break;
-            case 1: qh = e2m1x2_to_f16x2<1>(word); break;
-            case 2: qh = e2m1x2_to_f16x2<2>(word); break;
-            default: qh = e2m1x2_to_f16x2<3>(word); break;
-            }
-        }
+        const uint32_t qh = (FMT == MXQ_FMT_MXFP8)
+                                ? e4m3x2_to_f16x2(j & 1 ? (cw[j >> 1] >> 16) : cw[j >> 1])
+                                : q4[j];
         const float2 deq = __fmul2_rn(f16x2_to_float2(qh), sc2);
         accum_sq(make_float2(bf16_lo(w[j]), bf16_hi(w[j])), deq, e2, r2);
     }
