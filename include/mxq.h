@@ -205,6 +205,31 @@ MXQ_API mxq_status mxq_dequant_relerr(const uint16_t *x, const uint8_t *codes,
                               double *sum_sq_ref, double *relerr, void *workspace,
                               size_t workspace_bytes, cudaStream_t stream);
 
+/* The verifier above, for callers that cannot allocate device memory.
+ * The pages have no counterpart to this entry point; it exists for callers
+ * that reserve their whole device-memory budget up front (and so cannot
+ * cudaMalloc a workspace) or must not risk the synchronisation a cudaMalloc
+ * can cause.  It takes no workspace: the per-chunk partial sums live in a
+ * fixed 2 MiB array inside the library's device image, which every GPU that
+ * loads the library holds until the process exits.  Arguments, outputs and
+ * results are those of mxq_dequant_relerr.
+ *   Limit: n_tensors * ceil(rows * cols / 16384) <= 131072 chunks (for
+ *   example 1024 tensors of 768 x 2048, or 512 of 2048 x 768); larger
+ *   requests return MXQ_ERR_WORKSPACE before anything is enqueued.
+ *   The first call on a device looks up the array's device address on that
+ *   device (cudaGetSymbolAddress) and caches it; make that first call before
+ *   any stream capture.  It allocates nothing: no cudaMalloc, no cudaFree.
+ *   Every call on a device uses the same array and leaves its last contents
+ *   there (each call writes every partial it reads, so nothing needs to
+ *   start at zero); calls whose GPU work overlaps in time, on any streams,
+ *   race on it and give undefined results. */
+MXQ_API mxq_status mxq_dequant_relerr_noalloc(const uint16_t *x, const uint8_t *codes,
+                                              const uint8_t *scales, const float *s2,
+                                              mxq_fmt fmt, int64_t n_tensors, int64_t rows,
+                                              int64_t cols, int64_t tensors_per_scale,
+                                              double *sum_sq_err, double *sum_sq_ref,
+                                              double *relerr, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -11,7 +11,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libmxq.so")
-SOURCES = ["api.cu", "nvfp4.cu", "mx.cu", "verify.cu"]
+SOURCES = ["api.cu", "nvfp4.cu", "mx.cu", "verify.cu", "noalloc.cu"]
 HEADERS = ["mxq_device.cuh", "mxq_internal.h"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

@@ -29,7 +29,8 @@ SCALE_MODE = {"rtn": 0, "four_six": 1}
 OP = {"quantize_nvfp4": 0, "quantize_act": 1, "dequant_relerr": 2}
 
 EXPORTED = ("mxq_version", "mxq_status_string", "mxq_workspace_bytes", "mxq_quantize_nvfp4",
-            "mxq_quantize_mx", "mxq_quantize_act", "mxq_dequant_relerr")
+            "mxq_quantize_mx", "mxq_quantize_act", "mxq_dequant_relerr",
+            "mxq_dequant_relerr_noalloc")
 
 
 class MxqError(RuntimeError):
@@ -65,6 +66,8 @@ def load(path=LIB_PATH):
     L.mxq_quantize_act.argtypes = [vp, i64, i64, i32, vp, vp, vp, vp, vp, sz, vp]
     L.mxq_dequant_relerr.restype = i32
     L.mxq_dequant_relerr.argtypes = [vp, vp, vp, vp, i32, i64, i64, i64, i64, vp, vp, vp, vp, sz, vp]
+    L.mxq_dequant_relerr_noalloc.restype = i32
+    L.mxq_dequant_relerr_noalloc.argtypes = [vp, vp, vp, vp, i32, i64, i64, i64, i64, vp, vp, vp, vp]
     if path == LIB_PATH:
         _lib = L
     return L
@@ -129,6 +132,19 @@ def mxq_dequant_relerr(x, codes, scales, s2, fmt, n_tensors, rows, cols, tensors
                                    workspace.numel() if workspace is not None else 0,
                                    _stream(stream))
     _check("mxq_dequant_relerr", rc)
+
+
+def mxq_dequant_relerr_noalloc(x, codes, scales, s2, fmt, n_tensors, rows, cols,
+                               tensors_per_scale, sum_sq_err, sum_sq_ref, relerr, stream=None):
+    """The verifier without a workspace, for callers that cannot allocate
+    device memory: its partial sums live in a fixed 2 MiB array inside the
+    library (at most 131072 chunks of 16384 elements per call).  Calls whose
+    GPU work overlaps in time share that array and race."""
+    rc = load().mxq_dequant_relerr_noalloc(_p(x), _p(codes), _p(scales), _p(s2), FMT[fmt],
+                                           n_tensors, rows, cols, tensors_per_scale,
+                                           _p(sum_sq_err), _p(sum_sq_ref), _p(relerr),
+                                           _stream(stream))
+    _check("mxq_dequant_relerr_noalloc", rc)
 
 
 # ------------------------------------------------------------ allocating --
