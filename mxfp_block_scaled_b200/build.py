@@ -52,7 +52,9 @@ def build(force=False, verbose=False):
         subprocess.check_call(cmd)
         objs.append(obj)
     tmp = LIB + ".tmp%d" % os.getpid()
-    cmd = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *objs]
+    # -z defs: an unresolved symbol fails the link instead of the first dlopen
+    cmd = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-Xlinker", "-z,defs",
+           "-o", tmp, *objs]
     if verbose:
         print(" ".join(cmd))
     subprocess.check_call(cmd)

@@ -10,9 +10,15 @@ namespace mxq {
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+size_t nvfp4_slots_offset(int64_t n_groups)
+{
+    return align_up((size_t)n_groups * sizeof(uint32_t), 256);
+}
+
 size_t nvfp4_workspace_bytes(int64_t n_groups)
 {
-    return 2 * align_up((size_t)n_groups * sizeof(uint32_t), 256);
+    return nvfp4_slots_offset(n_groups) +
+           align_up((size_t)n_groups * kMaxFusedCtas * sizeof(unsigned long long), 256);
 }
 
 static size_t verify_workspace_bytes(int64_t n_tensors, int64_t rows, int64_t cols)
@@ -108,17 +114,17 @@ mxq_status mxq_quantize_nvfp4(const uint16_t *x, int64_t n_groups, int64_t rows,
     const int64_t nb = gsize / 16;
     const int64_t total_blocks = total / 16;
     uint32_t *amax_bits = static_cast<uint32_t *>(workspace);
-    uint32_t *arrive = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(workspace) +
-                                                    need / 2);
-    // amax bits and arrival counters start at zero
+    unsigned long long *slots = reinterpret_cast<unsigned long long *>(
+        static_cast<uint8_t *>(workspace) + nvfp4_slots_offset(n_groups));
+    // amax bits and amax slots start at zero (a slot's tag is its group + 1)
     cudaError_t e = cudaMemsetAsync(workspace, 0, need, stream);
     if (e == cudaSuccess && m4_count)
         e = cudaMemsetAsync(m4_count, 0, (size_t)n_groups * sizeof(uint32_t), stream);
     if (e != cudaSuccess)
         return MXQ_ERR_CUDA;
     // single pass (one HBM read of x) when the shape allows it
-    e = launch_nvfp4_fused(x, n_groups, nb, mode == MXQ_SCALE_FOUR_SIX, amax_bits, arrive, codes,
-                           scales, s2, mbits, m4_count, status, stream);
+    e = launch_nvfp4_fused(x, n_groups, nb, mode == MXQ_SCALE_FOUR_SIX, slots, codes, scales, s2,
+                           mbits, m4_count, status, stream);
     if (e == cudaSuccess)
         return MXQ_OK;
     if (e != cudaErrorNotSupported)

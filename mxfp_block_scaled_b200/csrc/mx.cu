@@ -47,7 +47,7 @@ mx_quant_kernel(const uint4 *__restrict__ x, int64_t nblk, uint8_t *__restrict__
         uint32_t m = 0;
 #pragma unroll
         for (int j = 0; j < 16; ++j)
-            m = abs_max_bits(m, w[j]);
+            m = absmax_bf16x2(m, w[j]);
         const uint32_t a = fold_halves(m);
         if (a >= 0x7F80u && status)
             atomicOr(status, MXQ_DEV_NONFINITE_INPUT);

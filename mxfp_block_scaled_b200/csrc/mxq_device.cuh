@@ -16,14 +16,17 @@ namespace mxq {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// Largest |x| of the 16-bit halves of `words` as bf16 magnitude bits.  Bit
-// patterns of non-negative bf16 values order like the values, and Inf / NaN
-// patterns (exponent all ones) sort above every finite value, so the result
-// is >= 0x7F80 exactly when some element is not finite.
-__device__ __forceinline__ uint32_t abs_max_bits(uint32_t acc, uint32_t w)
+// Running max of |x| over bf16x2 words, as bf16x2 bits (both halves >= 0).
+// NaN propagates, so a non-finite element leaves bits >= 0x7F80 (Inf or NaN)
+// in its half.
+__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t acc, uint32_t w)
 {
-    return __vmaxu2(acc, w & 0x7FFF7FFFu);
+    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162 *>(&acc);
+    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162 *>(&w);
+    const __nv_bfloat162 r = __hmax2_nan(a, __habs2(b));
+    return *reinterpret_cast<const uint32_t *>(&r);
 }
+// Larger half of non-negative bf16x2 bits (bit patterns order like values).
 __device__ __forceinline__ uint32_t fold_halves(uint32_t m) { return max(m & 0xFFFFu, m >> 16); }
 
 // ---- packed conversions (PTX ISA: cvt with .e2m1x2 / .e4m3x2) ------------
@@ -42,13 +45,53 @@ __device__ __forceinline__ uint32_t e2m1x2(float lo, float hi)
     return out;
 }
 
+// As e2m1x2, also returning the two decoded values as f16x2 (exact), taken
+// from the same byte register.
+__device__ __forceinline__ uint32_t e2m1x2_enc_dec(float lo, float hi, uint32_t &q)
+{
+    uint32_t out;
+    asm("{\n\t.reg .b8 t;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t, %3, %2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, t;\n\t"
+        "cvt.u32.u8 %0, t;\n\t}"
+        : "=r"(out), "=r"(q) : "f"(lo), "f"(hi));
+    return out;
+}
+
+// Eight fp32 values (four pairs) -> one word of eight E2M1 codes (pair j in
+// byte j, element 2j in its low nibble) and the four decoded pairs as f16x2,
+// decoded from the same byte registers.  The bytes are only ever packed into
+// the word here, never unpacked from it.
+__device__ __forceinline__ uint32_t e2m1x8_enc_dec(float2 p0, float2 p1, float2 p2, float2 p3,
+                                                   uint32_t (&q)[4])
+{
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %8, %7;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %10, %9;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %12, %11;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %4, b3;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(out), "=r"(q[0]), "=r"(q[1]), "=r"(q[2]), "=r"(q[3])
+        : "f"(p0.x), "f"(p0.y), "f"(p1.x), "f"(p1.y), "f"(p2.x), "f"(p2.y), "f"(p3.x), "f"(p3.y));
+    return out;
+}
+
+// Four zero-extended bytes -> one word, b0 lowest.
+__device__ __forceinline__ uint32_t pack4(uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3)
+{
+    return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
+}
+
 // Eight fp32 values -> eight E2M1 codes in one word, element 2j in the low
 // nibble of byte j.
 __device__ __forceinline__ uint32_t e2m1x8(float2 p0, float2 p1, float2 p2, float2 p3)
 {
-    const uint32_t b0 = e2m1x2(p0.x, p0.y), b1 = e2m1x2(p1.x, p1.y);
-    const uint32_t b2 = e2m1x2(p2.x, p2.y), b3 = e2m1x2(p3.x, p3.y);
-    return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
+    return pack4(e2m1x2(p0.x, p0.y), e2m1x2(p1.x, p1.y), e2m1x2(p2.x, p2.y), e2m1x2(p3.x, p3.y));
 }
 
 // Low byte of `v` (two E2M1 codes) -> f16x2, low nibble in the low half.
@@ -121,14 +164,13 @@ __device__ __forceinline__ float div_bf16(float x, float d, float r)
     return __fmaf_rn(-e, r, q0);
 }
 
-// Pairwise form on -x (nx), with nr = -r: returns x/d for both lanes.  The
-// operations are the same IEEE operations as div_bf16 with the negations
-// moved onto operands, so each lane's result is bit-identical to it.
-__device__ __forceinline__ float2 div2_bf16_neg(float2 nx, float2 d, float2 nr)
+// Pairwise form of div_bf16 with nr = -r: the same IEEE operations, the
+// negations moved onto operands, so each lane is bit-identical to it.
+__device__ __forceinline__ float2 div2_bf16(float2 x, float2 d, float2 nr)
 {
-    float2 q0 = __fmul2_rn(nx, nr);          // x * r
-    float2 e = __ffma2_rn(q0, d, nx);        // q0 * d - x
-    return __ffma2_rn(e, nr, q0);            // q0 - e * r
+    const float2 q0 = __fmul2_rn(x, make_float2(-nr.x, -nr.y));        // x * r
+    const float2 e = __ffma2_rn(q0, d, make_float2(-x.x, -x.y));        // q0 * d - x
+    return __ffma2_rn(e, nr, q0);                                       // q0 - e * r
 }
 
 // Bounded spin for inter-CTA flags: returns false after `limit` polls.
@@ -137,6 +179,18 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p)
     uint32_t v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
+}
+
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long *p)
+{
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long *p, unsigned long long v)
+{
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
 __device__ __forceinline__ void red_release_add_u32(uint32_t *p, uint32_t v)
@@ -165,6 +219,11 @@ __device__ __forceinline__ void fence_proxy_async_smem()
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes)
 {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
@@ -186,6 +245,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
                  "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
                  "selp.u32 %0, 1, 0, p;\n\t}"
                  : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
+
+// As mbar_try_wait, letting the hardware suspend the thread for up to about
+// `ns` nanoseconds while the phase is incomplete (fewer polling instructions).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t ns)
+{
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity), "r"(ns) : "memory");
     return ok != 0;
 }
 

@@ -15,7 +15,10 @@ constexpr int kNvThreads = 256;
 constexpr int kNvTileBlocks = 512;
 
 // Single-pass NVFP4 schedule: one cooperative CTA per SM.
-constexpr int kFusedThreads = 512;
+// 21 compute warps (2 and 1 full rounds over the gate_up / down slices of
+// the full-size layer), one publisher warp and one loader warp.
+constexpr int kFusedComputeWarps = 21;
+constexpr int kFusedThreads = 32 * (kFusedComputeWarps + 2);
 
 // Verifier: one CTA reduces one chunk of a tensor.
 constexpr int kVerifyThreads = 256;
@@ -23,9 +26,14 @@ constexpr int64_t kVerifyChunk = 16384;  // elements per chunk (multiple of 32)
 
 size_t align_up(size_t v, size_t a);
 
-// Workspace of the NVFP4 quantizer: per-group amax bits and per-group
-// arrival counters, each padded to 256 bytes.
+// Largest grid of the single-pass NVFP4 schedule (one CTA per SM).
+constexpr int kMaxFusedCtas = 256;
+
+// Workspace of the NVFP4 quantizer: per-group amax bits (two-pass schedule)
+// and per-group, per-CTA amax slots (single-pass schedule), each region
+// padded to 256 bytes.
 size_t nvfp4_workspace_bytes(int64_t n_groups);
+size_t nvfp4_slots_offset(int64_t n_groups);
 
 cudaError_t launch_group_amax(const uint16_t *x, int64_t n_groups, int64_t nb,
                               uint32_t *amax_bits, uint32_t *status, cudaStream_t s);
@@ -34,9 +42,9 @@ cudaError_t launch_nvfp4_quant(const uint16_t *x, int64_t n_groups, int64_t nb, 
                                float *s2, uint32_t *mbits, int mbits_atomic,
                                uint32_t *m4_count, cudaStream_t s);
 cudaError_t launch_nvfp4_fused(const uint16_t *x, int64_t n_groups, int64_t nb, int four_six,
-                               uint32_t *amax_bits, uint32_t *arrive, uint8_t *codes,
-                               uint8_t *scales, float *s2, uint32_t *mbits, uint32_t *m4_count,
-                               uint32_t *status, cudaStream_t s);
+                               unsigned long long *slots, uint8_t *codes, uint8_t *scales,
+                               float *s2, uint32_t *mbits, uint32_t *m4_count, uint32_t *status,
+                               cudaStream_t s);
 cudaError_t launch_mx_quant(const uint16_t *x, int64_t nblk32, int fmt, uint8_t *codes,
                             uint8_t *scales, uint32_t *status, cudaStream_t s);
 cudaError_t launch_verify(const uint16_t *x, const uint8_t *codes, const uint8_t *scales,

@@ -50,10 +50,10 @@ group_amax_kernel(const uint4 *__restrict__ x, int64_t n_groups, int64_t nb,
                 int64_t i = base + threadIdx.x + k * kNvThreads;
                 if (i < vec_per_group) {
                     uint4 v = __ldg(xg + i);
-                    m = abs_max_bits(m, v.x);
-                    m = abs_max_bits(m, v.y);
-                    m = abs_max_bits(m, v.z);
-                    m = abs_max_bits(m, v.w);
+                    m = absmax_bf16x2(m, v.x);
+                    m = absmax_bf16x2(m, v.y);
+                    m = absmax_bf16x2(m, v.z);
+                    m = absmax_bf16x2(m, v.w);
                 }
             }
         }
@@ -99,61 +99,73 @@ __device__ __forceinline__ GroupConst make_group_const(uint32_t amax_bits)
 
 struct Plan {
     uint2 codes;   // 16 E2M1 nibbles
-    float a_neg;   // -sum x_i q_i (exact)
+    float a;       // sum x_i q_i (exact)
     float b;       // sum q_i^2 (exact)
 };
 
-// q pair (f16x2): accumulate B in f16 (exact: <= 8 terms of quarter-
-// integers <= 36 per half) and -A in fp32 pairs.
-__device__ __forceinline__ void accum_pair(uint32_t qh, float2 nx, float2 &acc, uint32_t &bh)
-{
-    bh = hfma2_bits(qh, qh, bh);
-    acc = __ffma2_rn(nx, f16x2_to_float2(qh), acc);
-}
-
-__device__ __forceinline__ Plan make_plan(const float2 (&nx)[8], float D, float s2)
+// One plan's codes and the exact sums A and B from the quotients y.  The
+// decoded pair q comes from the same byte register the code was written to.
+// B is accumulated in f16 (<= 8 quarter-integers <= 36 per half: exact), A
+// in fp32 pairs (exact).
+__device__ __forceinline__ Plan plan_from_quotients(const float2 (&x)[8], const float2 (&y)[8])
 {
     Plan p;
-    const float d = __fmul_rn(D, s2);
-    if (!(d > 0.0f)) {  // D == 0, or D * s2 underflowed: all codes 0
-        p.codes = make_uint2(0u, 0u);
-        p.a_neg = 0.0f;
-        p.b = 0.0f;
-        return p;
-    }
-    float2 y[8];
-    if (d >= 0x1p-60f && d <= 0x1p60f) {
-        const float r = __frcp_rn(d);
-        const float2 d2 = make_float2(d, d), nr2 = make_float2(-r, -r);
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-            y[j] = div2_bf16_neg(nx[j], d2, nr2);
-    } else {
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-            y[j] = make_float2(__fdiv_rn(-nx[j].x, d), __fdiv_rn(-nx[j].y, d));
-    }
-    p.codes.x = e2m1x8(y[0], y[1], y[2], y[3]);
-    p.codes.y = e2m1x8(y[4], y[5], y[6], y[7]);
+    uint32_t q[8];
+    p.codes.x = e2m1x8_enc_dec(y[0], y[1], y[2], y[3], *reinterpret_cast<uint32_t(*)[4]>(&q[0]));
+    p.codes.y = e2m1x8_enc_dec(y[4], y[5], y[6], y[7], *reinterpret_cast<uint32_t(*)[4]>(&q[4]));
     float2 acc = make_float2(0.0f, 0.0f);
     uint32_t bh = 0u;
-    uint32_t q[8];
-    e2m1x8_to_f16x2(p.codes.x, *reinterpret_cast<uint32_t(*)[4]>(&q[0]));
-    e2m1x8_to_f16x2(p.codes.y, *reinterpret_cast<uint32_t(*)[4]>(&q[4]));
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-        accum_pair(q[j], nx[j], acc, bh);
-    p.a_neg = __fadd_rn(acc.x, acc.y);
+    for (int j = 0; j < 8; ++j) {
+        bh = hfma2_bits(q[j], q[j], bh);
+        acc = __ffma2_rn(x[j], f16x2_to_float2(q[j]), acc);
+    }
+    p.a = __fadd_rn(acc.x, acc.y);
     const float2 bf = f16x2_to_float2(bh);
     p.b = __fadd_rn(bf.x, bf.y);
     return p;
+}
+
+// y = RN32(x / d) with the reciprocal + FMA quotient, exact for d in
+// [2^-60, 2^60] (see div_bf16).
+__device__ __forceinline__ Plan make_plan_fast(const float2 (&x)[8], float d)
+{
+    const float r = __frcp_rn(d);
+    const float2 d2 = make_float2(d, d), nr2 = make_float2(-r, -r);
+    float2 y[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        y[j] = div2_bf16(x[j], d2, nr2);
+    return plan_from_quotients(x, y);
+}
+
+__device__ __forceinline__ bool fast_scale(float d) { return d >= 0x1p-60f && d <= 0x1p60f; }
+
+// Any d: all codes 0 when d is 0 (D == 0, or D * s2 underflowed), IEEE
+// division outside the fast range.  Taken for rare blocks only.
+__device__ __noinline__ Plan make_plan_any(const float2 (&x)[8], float d)
+{
+    if (!(d > 0.0f)) {
+        Plan p;
+        p.codes = make_uint2(0u, 0u);
+        p.a = 0.0f;
+        p.b = 0.0f;
+        return p;
+    }
+    if (fast_scale(d))
+        return make_plan_fast(x, d);
+    float2 y[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        y[j] = make_float2(__fdiv_rn(x[j].x, d), __fdiv_rn(x[j].y, d));
+    return plan_from_quotients(x, y);
 }
 
 // G_M = D (D s2 B - 2 A) in fp64, exact (see the file comment).
 __device__ __forceinline__ double plan_g(float D, float s2, const Plan &p)
 {
     const double dS = (double)D * (double)s2;
-    const double P = fma(dS, (double)p.b, 2.0 * (double)p.a_neg);
+    const double P = fma(dS, (double)p.b, -2.0 * (double)p.a);
     return (double)D * P;
 }
 
@@ -171,7 +183,7 @@ __device__ __forceinline__ BlockOut quantize_block(uint4 v0, uint4 v1, const Gro
     uint32_t m = 0;
 #pragma unroll
     for (int j = 0; j < 8; ++j)
-        m = abs_max_bits(m, w[j]);
+        m = absmax_bf16x2(m, w[j]);
     const float amax_b = __uint_as_float(fold_halves(m) << 16);
     if (!(gc.s2 > 0.0f)) {  // all-zero group
         o.codes = make_uint2(0u, 0u);
@@ -179,12 +191,10 @@ __device__ __forceinline__ BlockOut quantize_block(uint4 v0, uint4 v1, const Gro
         o.m4 = false;
         return o;
     }
-    float2 nx[8];
+    float2 x[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const uint32_t n = w[j] ^ 0x80008000u;
-        nx[j] = make_float2(bf16_lo(n), bf16_hi(n));
-    }
+    for (int j = 0; j < 8; ++j)
+        x[j] = make_float2(bf16_lo(w[j]), bf16_hi(w[j]));
     float t6, t4;
     if (gc.fast) {
         t6 = div_bf16(amax_b, gc.den6, gc.r6);
@@ -195,14 +205,24 @@ __device__ __forceinline__ BlockOut quantize_block(uint4 v0, uint4 v1, const Gro
     }
     const uint32_t sb = e4m3x2(t6, FOUR_SIX ? t4 : 0.0f);   // S6 low byte, S4 high
     const float2 D = f16x2_to_float2(e4m3x2_to_f16x2(sb));
-    const Plan p6 = make_plan(nx, D.x, gc.s2);
+    const float d6 = __fmul_rn(D.x, gc.s2), d4 = __fmul_rn(D.y, gc.s2);
+    // Both plans straight-line on the fast path (so their independent work
+    // interleaves); blocks whose scale is 0 or outside the fast range redo
+    // the affected plan exactly.
+    Plan p6 = make_plan_fast(x, d6);
     if (!FOUR_SIX) {
+        if (!fast_scale(d6))
+            p6 = make_plan_any(x, d6);
         o.codes = p6.codes;
         o.scale = sb & 0xFFu;
         o.m4 = false;
         return o;
     }
-    const Plan p4 = make_plan(nx, D.y, gc.s2);
+    Plan p4 = make_plan_fast(x, d4);
+    if (!fast_scale(d6) || !fast_scale(d4)) {
+        p6 = make_plan_any(x, d6);
+        p4 = make_plan_any(x, d4);
+    }
     const bool use4 = plan_g(D.y, gc.s2, p4) < plan_g(D.x, gc.s2, p6);
     o.codes = use4 ? p4.codes : p6.codes;
     o.scale = use4 ? (sb >> 8) : (sb & 0xFFu);
@@ -288,24 +308,29 @@ nvfp4_quant_kernel(const uint4 *__restrict__ x, int64_t n_groups, int64_t nb,
 //
 // A cooperative persistent grid of one CTA per SM.  Every group's blocks are
 // cut into one contiguous slice per CTA (a multiple of 32 blocks, so a warp's
-// M bits fill one word).  Each CTA walks the groups in order with a ring of
-// `stages` shared-memory buffers filled by bulk copies:
-//   iteration i:  (A) wait for slice i in smem, reduce its amax, publish it
-//                     (atomicMax, then a release increment of arrive[i]);
-//                 (B) for j = i - lookahead: wait until all CTAs published
-//                     group j (acquire, bounded), derive s2, quantize slice j
-//                     from smem, then refill its buffer with slice j+stages.
-// W is read from HBM once; the amax dependency of a group is resolved
-// `lookahead` iterations after its data arrived, so the wait is normally
-// already satisfied.  Every wait is bounded: on time-out the CTA sets
-// MXQ_DEV_WAIT_TIMEOUT, waits (bounded) for its own copies in flight and
-// returns.
+// M bits fill one word).  The slices of successive groups stream through a
+// ring of `stages` shared-memory buffers filled by bulk copies.  W is read
+// from HBM once.
+//
+// Warp roles.  A publisher thread (warp 0) publishes this CTA's slice amax
+// of each group (atomicMax, then a release increment of arrive[g]) and, as
+// soon as every CTA published group j (acquire, bounded), hands the group
+// amax to the compute warps.  A loader thread (warp 1) refills each buffer
+// with a bulk copy as soon as the compute warps freed it.  The compute warps,
+// at step t, reduce the amax of their share of slice t and quantize their
+// share of slice t - lookahead, deriving the group constants themselves.
+// Roles hand over through mbarriers only (full: copy landed; amaxd: partial
+// amax written; ready: group amax known; freed: slice consumed), so no warp
+// waits for another except through the data it needs.  Every wait is
+// bounded: on time-out the CTA sets MXQ_DEV_WAIT_TIMEOUT, lets its copies in
+// flight land (bounded) and returns.
 // ---------------------------------------------------------------------------
 struct FusedArgs {
     const uint16_t *x;
     int64_t n_groups, nb, slice;   // blocks per group, blocks per CTA slice
     int stages, lookahead;
-    uint32_t *amax_bits, *arrive, *status;
+    uint32_t *status;
+    unsigned long long *slots;     // [n_groups][kMaxFusedCtas] (tag << 32 | slice amax bits)
     uint2 *codes;
     uint8_t *scales;
     float *s2_out;
@@ -313,156 +338,220 @@ struct FusedArgs {
 };
 
 constexpr uint32_t kSpinLimit = 1u << 22;   // polls of a flag / barrier before giving up
+constexpr int kMaxStages = 8;
+
+// Bounded wait on an mbarrier phase that also gives up once another role of
+// the CTA has aborted.
+__device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity, volatile int *abort_flag)
+{
+    for (uint32_t i = 0; i < kSpinLimit; ++i) {
+        if (mbar_try_wait_sleep(bar, parity, 20000u))
+            return true;
+        if (*abort_flag)
+            return false;
+    }
+    *abort_flag = 1;
+    return false;
+}
 
 template <bool FOUR_SIX>
 __global__ void __launch_bounds__(kFusedThreads, 1)
 nvfp4_fused_kernel(const FusedArgs a)
 {
     extern __shared__ __align__(128) uint8_t smem[];
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
-    uint8_t *buf = smem + 128;
-    __shared__ uint32_t s_red[kFusedThreads / 32];
-    __shared__ GroupConst s_gc;
-    __shared__ uint32_t s_m4;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem);   // copy of the slice landed
+    uint64_t *amaxd = full + kMaxStages;                   // all compute warps wrote their amax
+    uint64_t *ready = amaxd + kMaxStages;                  // every CTA published the group
+    uint64_t *freed = ready + kMaxStages;                  // all compute warps done with the slice
+    uint8_t *buf = smem + 256;
+    __shared__ uint32_t s_amax[kMaxStages];                // group amax bits, set before ready
+    __shared__ uint32_t s_part[kMaxStages][kFusedComputeWarps];
+    __shared__ uint32_t s_m4[kMaxStages];
     __shared__ int s_abort;
+    volatile int *abort_flag = &s_abort;
 
-    const int tid = threadIdx.x, lane = tid & 31;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t P = gridDim.x;
     const int64_t my_lo = (int64_t)blockIdx.x * a.slice;
-    const int64_t my_n = max((int64_t)0, min(a.slice, a.nb - my_lo));
+    const int64_t my_n = max((int64_t)0, min(a.slice, a.nb - my_lo));   // multiple of 32
     const uint32_t bytes = (uint32_t)(my_n * 32);
     const int64_t stage_bytes = a.slice * 32;
     const int L = a.stages, LA = a.lookahead;
     const int64_t G = a.n_groups;
 
-    if (tid == 0) {
-        for (int k = 0; k < L; ++k)
-            mbar_init(bars + k, 1);
-        fence_mbar_init();
+    if (threadIdx.x == 0) {
+        for (int k = 0; k < L; ++k) {
+            mbar_init(full + k, 1);
+            mbar_init(amaxd + k, kFusedComputeWarps);
+            mbar_init(ready + k, 1);
+            mbar_init(freed + k, kFusedComputeWarps);
+            s_m4[k] = 0;
+        }
         s_abort = 0;
-        s_m4 = 0;
+        fence_mbar_init();
     }
     __syncthreads();
 
-    auto issue = [&](int64_t g) {   // thread 0: load slice of group g into stage g % L
-        if (bytes == 0)
+    if (warp == 0) {
+        // -------------------------------------------------------- publisher
+        // Publishes this CTA's slice amax of each group as soon as the compute
+        // warps reduced it: one 64-bit store of (group tag, amax bits) into
+        // the CTA's slot, so value and tag become visible together and no
+        // fence is needed.  Group j is released to the compute warps once all
+        // P slots of j carry j's tag; the group amax is the max over slots.
+        int64_t next_pub = 0, next_ready = 0;
+        uint32_t idle = 0;
+        while (next_ready < G) {
+            bool progress = false;
+            int got = 0;
+            if (next_pub < G && lane == 0)
+                got = mbar_try_wait(amaxd + next_pub % L, (uint32_t)((next_pub / L) & 1)) ? 1 : 0;
+            if (__shfl_sync(0xFFFFFFFFu, got, 0)) {   // warp-uniform from here
+                if (lane == 0) {
+                    const int st = (int)(next_pub % L);
+                    uint32_t mx = 0;
+                    for (int w = 0; w < kFusedComputeWarps; ++w)
+                        mx = max(mx, s_part[st][w]);
+                    if (mx >= 0x7F80u)
+                        atomicOr(a.status, MXQ_DEV_NONFINITE_INPUT);
+                    const unsigned long long v = ((unsigned long long)(next_pub + 1) << 32) | mx;
+                    st_relaxed_u64(a.slots + next_pub * kMaxFusedCtas + blockIdx.x, v);
+                }
+                ++next_pub;
+                progress = true;
+            }
+            if (next_ready < next_pub) {
+                const unsigned long long *sl = a.slots + next_ready * kMaxFusedCtas;
+                const uint32_t tag = (uint32_t)(next_ready + 1);
+                bool all = true;
+                uint32_t mx = 0;
+                for (uint32_t c = lane; c < P; c += 32) {
+                    const unsigned long long v = ld_relaxed_u64(sl + c);
+                    all = all && ((uint32_t)(v >> 32) == tag);
+                    mx = max(mx, (uint32_t)v);
+                }
+                if (__all_sync(0xFFFFFFFFu, all)) {
+                    mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+                    if (lane == 0) {
+                        const int st = (int)(next_ready % L);
+                        s_amax[st] = mx;
+                        if (blockIdx.x == 0)
+                            a.s2_out[next_ready] = __fdiv_rn(__uint_as_float(mx << 16), kGlobalDivisor);
+                        mbar_arrive(ready + st);
+                    }
+                    ++next_ready;
+                    progress = true;
+                }
+            }
+            if (!progress)
+                __nanosleep(200);
+            if (progress) {
+                idle = 0;
+            } else if (__any_sync(0xFFFFFFFFu, ++idle > (kSpinLimit >> 4) || *abort_flag)) {
+                if (lane == 0) {
+                    *abort_flag = 1;
+                    atomicOr(a.status, MXQ_DEV_WAIT_TIMEOUT);
+                }
+                break;
+            }
+        }
+        return;
+    }
+    if (warp == 1) {
+        // ----------------------------------------------------------- loader
+        if (lane != 0)
             return;
-        const int st = (int)(g % L);
-        fence_proxy_async_smem();
-        mbar_arrive_expect_tx(bars + st, bytes);
-        bulk_g2s(buf + st * stage_bytes, a.x + (g * a.nb + my_lo) * 16, bytes, bars + st);
-    };
-    if (tid == 0)
+        int64_t last_issued[kMaxStages];
+        for (int k = 0; k < kMaxStages; ++k)
+            last_issued[k] = -1;
+        auto issue = [&](int64_t g) {
+            if (bytes == 0)
+                return;
+            const int st = (int)(g % L);
+            fence_proxy_async_smem();
+            mbar_arrive_expect_tx(full + st, bytes);
+            bulk_g2s(buf + st * stage_bytes, a.x + (g * a.nb + my_lo) * 16, bytes, full + st);
+            last_issued[st] = g;
+        };
         for (int64_t g = 0; g < G && g < L; ++g)
             issue(g);
-    int64_t issued = G < L ? G : L;   // groups whose slice load was issued
-    int64_t landed = 0;               // groups whose slice load was waited for
+        for (int64_t j = 0; j < G; ++j) {
+            const int st = (int)(j % L);
+            if (!wait_phase(freed + st, (uint32_t)((j / L) & 1), abort_flag))
+                break;
+            if (a.m4_count && s_m4[st])
+                atomicAdd(a.m4_count + j, s_m4[st]);
+            s_m4[st] = 0;
+            if (j + L < G)
+                issue(j + L);
+        }
+        if (*abort_flag) {
+            atomicOr(a.status, MXQ_DEV_WAIT_TIMEOUT);
+            // let this CTA's copies in flight land before its smem is released
+            for (int k = 0; k < L; ++k)
+                if (last_issued[k] >= 0)
+                    for (uint32_t n = 0; n < kSpinLimit; ++n)
+                        if (mbar_try_wait(full + k, (uint32_t)((last_issued[k] / L) & 1)))
+                            break;
+        }
+        return;
+    }
 
-    for (int64_t i = 0; i < G + LA; ++i) {
-        // (A) amax of my slice of group i, published to the other CTAs
+    // -------------------------------------------------------- compute warps
+    const int cw = warp - 2;
+    const int64_t n32 = my_n / 32;
+    for (int64_t t = 0; t < G + LA; ++t) {
+        const int64_t i = t, j = t - LA;
         if (i < G) {
             const int st = (int)(i % L);
             uint32_t m = 0;
             if (bytes) {
-                if (!mbar_wait_bounded(bars + st, (uint32_t)((i / L) & 1), kSpinLimit))
-                    s_abort = 1;
-                else
-                    landed = i + 1;
+                const bool ok = __all_sync(0xFFFFFFFFu, wait_phase(full + st, (uint32_t)((i / L) & 1), abort_flag));
+                if (!ok)
+                    break;
                 const uint4 *v = reinterpret_cast<const uint4 *>(buf + st * stage_bytes);
-                for (int64_t k = tid; k < my_n * 2; k += kFusedThreads) {
-                    const uint4 q = v[k];
-                    m = abs_max_bits(m, q.x);
-                    m = abs_max_bits(m, q.y);
-                    m = abs_max_bits(m, q.z);
-                    m = abs_max_bits(m, q.w);
+                for (int64_t u = lane + 32 * cw; u < my_n * 2; u += 32 * kFusedComputeWarps) {
+                    const uint4 q = v[u];
+                    m = absmax_bf16x2(m, q.x);
+                    m = absmax_bf16x2(m, q.y);
+                    m = absmax_bf16x2(m, q.z);
+                    m = absmax_bf16x2(m, q.w);
                 }
             }
             const uint32_t r = __reduce_max_sync(0xFFFFFFFFu, fold_halves(m));
-            if (lane == 0)
-                s_red[tid >> 5] = r;
-            __syncthreads();
-            if (tid == 0) {
-                uint32_t mx = 0;
-                for (int w = 0; w < kFusedThreads / 32; ++w)
-                    mx = max(mx, s_red[w]);
-                if (mx)
-                    atomicMax(a.amax_bits + i, mx);
-                if (mx >= 0x7F80u)
-                    atomicOr(a.status, MXQ_DEV_NONFINITE_INPUT);
-                red_release_add_u32(a.arrive + i, 1u);
+            if (lane == 0) {
+                s_part[st][cw] = r;
+                mbar_arrive(amaxd + st);
             }
         }
-        // (B) quantize my slice of group j once every CTA published it
-        const int64_t j = i - LA;
         if (j >= 0) {
-            if (tid == 0) {
-                uint32_t spins = 0;
-                while (ld_acquire_u32(a.arrive + j) < P) {
-                    if (++spins > kSpinLimit) {
-                        s_abort = 1;
-                        break;
-                    }
-                    __nanosleep(64);
-                }
-                const uint32_t am = *reinterpret_cast<volatile uint32_t *>(a.amax_bits + j);
-                s_gc = make_group_const(am);
-                if (blockIdx.x == 0)
-                    a.s2_out[j] = s_gc.s2;
-            }
-            __syncthreads();
-            if (s_abort)
-                break;
-            const GroupConst gc = s_gc;
             const int st = (int)(j % L);
-            const uint4 *v = reinterpret_cast<const uint4 *>(buf + st * stage_bytes);
-            uint32_t my_m4 = 0;
-            for (int64_t k0 = 0; k0 < my_n; k0 += kFusedThreads) {
-                const int64_t k = k0 + tid;
-                const bool live = k < my_n;
-                BlockOut o;
-                o.m4 = false;
-                const int64_t gb = j * a.nb + my_lo + k;
-                if (live) {
-                    o = quantize_block<FOUR_SIX>(v[2 * k], v[2 * k + 1], gc);
-                    a.codes[gb] = o.codes;
-                    a.scales[gb] = (uint8_t)o.scale;
-                }
-                if (a.mbits) {
-                    const uint32_t word = __ballot_sync(0xFFFFFFFFu, o.m4);
-                    if (lane == 0 && k0 + tid - lane < my_n)
-                        a.mbits[(gb - lane) >> 5] = word;
-                }
-                my_m4 += o.m4 ? 1u : 0u;
-            }
-            if (FOUR_SIX && a.m4_count) {
-                const uint32_t wsum = __reduce_add_sync(0xFFFFFFFFu, my_m4);
-                if (lane == 0 && wsum)
-                    atomicAdd(&s_m4, wsum);
-            }
-            __syncthreads();   // every thread is done with stage st
-            if (tid == 0) {
-                if (FOUR_SIX && a.m4_count && s_m4) {
-                    atomicAdd(a.m4_count + j, s_m4);
-                    s_m4 = 0;
-                }
-                if (j + L < G)
-                    issue(j + L);
-            }
-            if (j + L < G)
-                ++issued;
-        }
-        if (i < G) {
-            __syncthreads();
-            if (s_abort)
+            const bool ok = __all_sync(0xFFFFFFFFu, wait_phase(ready + st, (uint32_t)((j / L) & 1), abort_flag));
+            if (!ok)
                 break;
+            const GroupConst gc = make_group_const(s_amax[st]);
+            const uint4 *v = reinterpret_cast<const uint4 *>(buf + st * stage_bytes);
+            uint32_t cnt = 0;
+            for (int64_t k32 = cw; k32 < n32; k32 += kFusedComputeWarps) {
+                const int64_t k = k32 * 32 + lane;
+                const BlockOut o = quantize_block<FOUR_SIX>(v[2 * k], v[2 * k + 1], gc);
+                const int64_t gb = j * a.nb + my_lo + k;
+                a.codes[gb] = o.codes;
+                a.scales[gb] = (uint8_t)o.scale;
+                const uint32_t word = __ballot_sync(0xFFFFFFFFu, o.m4);
+                if (lane == 0) {
+                    if (a.mbits)
+                        a.mbits[(gb - lane) >> 5] = word;
+                    cnt += __popc(word);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) {
+                if (cnt)
+                    atomicAdd(&s_m4[st], cnt);
+                mbar_arrive(freed + st);
+            }
         }
-    }
-    if (s_abort && tid == 0) {
-        atomicOr(a.status, MXQ_DEV_WAIT_TIMEOUT);
-        // let this CTA's copies in flight land before its smem is released
-        if (bytes)
-            for (int64_t g = landed; g < issued; ++g)
-                mbar_wait_bounded(bars + (g % L), (uint32_t)((g / L) & 1), kSpinLimit);
     }
 }
 
@@ -493,9 +582,9 @@ static int sm_count()
 // device does not suit the single-pass schedule; the caller then takes the
 // two-pass path.
 cudaError_t launch_nvfp4_fused(const uint16_t *x, int64_t n_groups, int64_t nb, int four_six,
-                               uint32_t *amax_bits, uint32_t *arrive, uint8_t *codes,
-                               uint8_t *scales, float *s2, uint32_t *mbits, uint32_t *m4_count,
-                               uint32_t *status, cudaStream_t s)
+                               unsigned long long *slots, uint8_t *codes, uint8_t *scales,
+                               float *s2, uint32_t *mbits, uint32_t *m4_count, uint32_t *status,
+                               cudaStream_t s)
 {
     if (n_groups <= 0 || nb <= 0 || nb % 32 != 0)
         return cudaErrorNotSupported;
@@ -505,12 +594,12 @@ cudaError_t launch_nvfp4_fused(const uint16_t *x, int64_t n_groups, int64_t nb, 
         cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
         return cudaErrorNotSupported;
     const int sms = sm_count();
-    if (!coop || sms <= 0)
+    if (!coop || sms <= 0 || sms > kMaxFusedCtas || !slots)
         return cudaErrorNotSupported;
     int64_t slice = (nb + sms - 1) / sms;
     slice = (slice + 31) / 32 * 32;
     const int64_t slice_bytes = slice * 32;
-    const int64_t avail = (int64_t)max_optin - 128 - 1024;   // barriers + static smem margin
+    const int64_t avail = (int64_t)max_optin - 256 - 2048;   // barriers + static smem margin
     int64_t L = avail / slice_bytes;
     if (L < 1)
         return cudaErrorNotSupported;
@@ -519,7 +608,7 @@ cudaError_t launch_nvfp4_fused(const uint16_t *x, int64_t n_groups, int64_t nb, 
     if (L > n_groups)
         L = n_groups;
     const int LA = L >= 4 ? 2 : (L >= 2 ? 1 : 0);
-    const size_t dyn = 128 + (size_t)(L * slice_bytes);
+    const size_t dyn = 256 + (size_t)(L * slice_bytes);
     const void *fn = four_six ? (const void *)nvfp4_fused_kernel<true> : (const void *)nvfp4_fused_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
     if (e != cudaSuccess)
@@ -537,8 +626,7 @@ cudaError_t launch_nvfp4_fused(const uint16_t *x, int64_t n_groups, int64_t nb, 
     args.slice = slice;
     args.stages = (int)L;
     args.lookahead = LA;
-    args.amax_bits = amax_bits;
-    args.arrive = arrive;
+    args.slots = slots;
     args.status = status;
     args.codes = reinterpret_cast<uint2 *>(codes);
     args.scales = scales;

@@ -112,6 +112,11 @@ verify_chunk_kernel(const uint16_t *__restrict__ x, const uint8_t *__restrict__ 
                     int64_t tensors_per_scale, double *__restrict__ partials)
 {
     constexpr int BLK = (FMT == MXQ_FMT_NVFP4) ? 16 : 32;
+    // blocks per thread per chunk; all of a thread's loads are issued before
+    // any of its arithmetic, so each thread keeps PER blocks in flight
+    constexpr int PER = (int)(kVerifyChunk / BLK / kVerifyThreads);
+    constexpr int XV = BLK / 8;                                   // uint4 of x per block
+    constexpr int CV = (FMT == MXQ_FMT_MXFP8) ? 2 : 1;            // uint4 of codes (MX)
     const int64_t n_chunks = n_tensors * chunks_per_tensor;
     for (int64_t c = blockIdx.x; c < n_chunks; c += gridDim.x) {
         const int64_t t = c / chunks_per_tensor;
@@ -120,32 +125,48 @@ verify_chunk_kernel(const uint16_t *__restrict__ x, const uint8_t *__restrict__ 
         const int64_t hi = min(lo + kVerifyChunk, tsize);
         const int64_t nblk = (hi - lo) / BLK;
         const int64_t first = (t * tsize + lo) / BLK;   // global block index
-        double err = 0.0, ref = 0.0;
-        for (int64_t i = threadIdx.x; i < nblk; i += kVerifyThreads) {
-            const int64_t gb = first + i;
-            if (FMT == MXQ_FMT_NVFP4) {
-                const uint4 *xv = reinterpret_cast<const uint4 *>(x) + gb * 2;
-                const uint4 v0 = __ldg(xv), v1 = __ldg(xv + 1);
-                const uint2 cc = __ldg(reinterpret_cast<const uint2 *>(codes) + gb);
-                const uint32_t sb = __ldg(scales + gb);
-                nvfp4_block_sq(v0, v1, cc, sb, __ldg(s2 + t / tensors_per_scale), err, ref);
-            } else {
-                const uint4 *xv = reinterpret_cast<const uint4 *>(x) + gb * 4;
-                uint4 v[4];
+        const float sv = (FMT == MXQ_FMT_NVFP4) ? __ldg(s2 + t / tensors_per_scale) : 0.0f;
+        uint4 xv[PER][XV];
+        uint4 cv[PER][CV];
+        uint2 c2[PER];
+        uint32_t sb[PER];
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    v[q] = __ldg(xv + q);
-                uint32_t cw[8];
-                if (FMT == MXQ_FMT_MXFP8) {
-                    const uint4 *cv = reinterpret_cast<const uint4 *>(codes) + gb * 2;
-                    const uint4 c0 = __ldg(cv), c1 = __ldg(cv + 1);
-                    cw[0] = c0.x; cw[1] = c0.y; cw[2] = c0.z; cw[3] = c0.w;
-                    cw[4] = c1.x; cw[5] = c1.y; cw[6] = c1.z; cw[7] = c1.w;
+        for (int u = 0; u < PER; ++u) {
+            const int64_t i = threadIdx.x + (int64_t)u * kVerifyThreads;
+            if (i < nblk) {
+                const int64_t gb = first + i;
+                const uint4 *src = reinterpret_cast<const uint4 *>(x) + gb * XV;
+#pragma unroll
+                for (int q = 0; q < XV; ++q)
+                    xv[u][q] = __ldg(src + q);
+                if (FMT == MXQ_FMT_NVFP4) {
+                    c2[u] = __ldg(reinterpret_cast<const uint2 *>(codes) + gb);
                 } else {
-                    const uint4 c0 = __ldg(reinterpret_cast<const uint4 *>(codes) + gb);
-                    cw[0] = c0.x; cw[1] = c0.y; cw[2] = c0.z; cw[3] = c0.w;
+#pragma unroll
+                    for (int q = 0; q < CV; ++q)
+                        cv[u][q] = __ldg(reinterpret_cast<const uint4 *>(codes) + gb * CV + q);
                 }
-                mx_block_sq<FMT>(v, cw, __ldg(scales + gb), err, ref);
+                sb[u] = __ldg(scales + gb);
+            }
+        }
+        double err = 0.0, ref = 0.0;
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+            const int64_t i = threadIdx.x + (int64_t)u * kVerifyThreads;
+            if (i < nblk) {
+                if (FMT == MXQ_FMT_NVFP4) {
+                    nvfp4_block_sq(xv[u][0], xv[u][1], c2[u], sb[u], sv, err, ref);
+                } else {
+                    uint32_t cw[8];
+                    cw[0] = cv[u][0].x; cw[1] = cv[u][0].y; cw[2] = cv[u][0].z; cw[3] = cv[u][0].w;
+                    if (CV == 2) {
+                        cw[4] = cv[u][CV - 1].x; cw[5] = cv[u][CV - 1].y;
+                        cw[6] = cv[u][CV - 1].z; cw[7] = cv[u][CV - 1].w;
+                    }
+                    const uint4 v4[4] = {xv[u][0], xv[u][XV > 1 ? 1 : 0], xv[u][XV > 2 ? 2 : 0],
+                                         xv[u][XV > 3 ? 3 : 0]};
+                    mx_block_sq<FMT>(v4, cw, sb[u], err, ref);
+                }
             }
         }
         cta_reduce_store(err, ref, partials + 2 * c);

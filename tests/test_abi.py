@@ -46,10 +46,11 @@ def test_version_and_status_strings(lib):
 
 
 def test_workspace_sizes(lib):
-    # amax bits + arrival counters, each padded to 256 bytes
-    assert lib.mxq_workspace_bytes(0, 512, 1536, 2048) == 2 * 2048
-    assert lib.mxq_workspace_bytes(0, 1, 16, 16) == 512
-    assert lib.mxq_workspace_bytes(1, 4096, 2048, 0) == 512
+    # amax bits + per-group, per-CTA amax slots (256 x 8 bytes), each padded
+    # to 256 bytes
+    assert lib.mxq_workspace_bytes(0, 512, 1536, 2048) == 2048 + 512 * 256 * 8
+    assert lib.mxq_workspace_bytes(0, 1, 16, 16) == 256 + 2048
+    assert lib.mxq_workspace_bytes(1, 4096, 2048, 0) == 256 + 2048
     # verifier: 16 bytes per chunk of 16384 elements per tensor
     cpt = -(-768 * 2048 // 16384)
     assert lib.mxq_workspace_bytes(2, 1024, 768, 2048) == (1024 * cpt * 16 + 255) // 256 * 256
