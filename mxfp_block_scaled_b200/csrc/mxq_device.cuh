@@ -173,6 +173,12 @@ __device__ __forceinline__ float2 div2_bf16(float2 x, float2 d, float2 nr)
     return __ffma2_rn(e, nr, q0);                                       // q0 - e * r
 }
 
+// Barrier `id` (1..15) among `count` threads (a multiple of 32).
+__device__ __forceinline__ void named_barrier_sync(int id, int count)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // Bounded spin for inter-CTA flags: returns false after `limit` polls.
 __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p)
 {

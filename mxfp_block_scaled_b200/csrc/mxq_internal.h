@@ -16,9 +16,9 @@ constexpr int kNvTileBlocks = 512;
 
 // Single-pass NVFP4 schedule: one cooperative CTA per SM.
 // 21 compute warps (2 and 1 full rounds over the gate_up / down slices of
-// the full-size layer), one publisher warp and one loader warp.
+// the full-size layer), a publisher warp, a loader warp and two scout warps.
 constexpr int kFusedComputeWarps = 21;
-constexpr int kFusedThreads = 32 * (kFusedComputeWarps + 2);
+constexpr int kFusedThreads = 32 * (kFusedComputeWarps + 4);
 
 // Verifier: one CTA reduces one chunk of a tensor.
 constexpr int kVerifyThreads = 256;

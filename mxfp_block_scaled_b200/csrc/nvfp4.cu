@@ -308,27 +308,28 @@ nvfp4_quant_kernel(const uint4 *__restrict__ x, int64_t n_groups, int64_t nb,
 //
 // A cooperative persistent grid of one CTA per SM.  Every group's blocks are
 // cut into one contiguous slice per CTA (a multiple of 32 blocks, so a warp's
-// M bits fill one word).  The slices of successive groups stream through a
-// ring of `stages` shared-memory buffers filled by bulk copies.  W is read
-// from HBM once.
-//
-// Warp roles.  A publisher thread (warp 0) publishes this CTA's slice amax
-// of each group (atomicMax, then a release increment of arrive[g]) and, as
-// soon as every CTA published group j (acquire, bounded), hands the group
-// amax to the compute warps.  A loader thread (warp 1) refills each buffer
-// with a bulk copy as soon as the compute warps freed it.  The compute warps,
-// at step t, reduce the amax of their share of slice t and quantize their
-// share of slice t - lookahead, deriving the group constants themselves.
-// Roles hand over through mbarriers only (full: copy landed; amaxd: partial
-// amax written; ready: group amax known; freed: slice consumed), so no warp
-// waits for another except through the data it needs.  Every wait is
-// bounded: on time-out the CTA sets MXQ_DEV_WAIT_TIMEOUT, lets its copies in
-// flight land (bounded) and returns.
+// M bits fill one word).  Each CTA walks the groups in order; its slice of
+// a group is brought into shared memory twice by bulk copies:
+//   scout copy     (ring of `sstages`): two scout warps reduce the slice
+//                  amax and publish it as one tagged 64-bit slot per group
+//                  and CTA (tag and value land together: no fence needed);
+//   quantize copy  (ring of `qstages`), issued only after the scouts are
+//                  done with that group, `distance` groups behind them, so
+//                  it normally hits the L2 copy the scout read left behind:
+//                  21 compute warps quantize it once a publisher warp has
+//                  seen every CTA's slot for the group.
+// The grid-wide amax of a group is therefore resolved while the compute
+// warps work on earlier groups; its latency is off the critical path.
+// Roles hand over through mbarriers (sfull / sfreed: scout ring, qfull /
+// qfreed: quantize ring, ready: group amax known) and one shared counter
+// (groups scouted).  Every wait is bounded: on time-out the CTA sets
+// MXQ_DEV_WAIT_TIMEOUT, lets its copies in flight land (bounded) and
+// returns.
 // ---------------------------------------------------------------------------
 struct FusedArgs {
     const uint16_t *x;
     int64_t n_groups, nb, slice;   // blocks per group, blocks per CTA slice
-    int stages, lookahead;
+    int sstages, qstages, distance;
     uint32_t *status;
     unsigned long long *slots;     // [n_groups][kMaxFusedCtas] (tag << 32 | slice amax bits)
     uint2 *codes;
@@ -339,13 +340,18 @@ struct FusedArgs {
 
 constexpr uint32_t kSpinLimit = 1u << 22;   // polls of a flag / barrier before giving up
 constexpr int kMaxStages = 8;
+constexpr int kReadyRing = 16;   // > distance + qstages: ready phases never run a lap ahead
+constexpr int kPollGroups = 4;   // groups whose readiness one publisher poll tests
 
 // Bounded wait on an mbarrier phase that also gives up once another role of
 // the CTA has aborted.
-__device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity, volatile int *abort_flag)
+// The hardware may suspend the waiting thread for up to about `sleep_ns`
+// while the phase is incomplete, so idle roles do not spin.
+__device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                           uint32_t sleep_ns = 0)
 {
     for (uint32_t i = 0; i < kSpinLimit; ++i) {
-        if (mbar_try_wait_sleep(bar, parity, 20000u))
+        if (sleep_ns ? mbar_try_wait_sleep(bar, parity, sleep_ns) : mbar_try_wait(bar, parity))
             return true;
         if (*abort_flag)
             return false;
@@ -359,16 +365,19 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 nvfp4_fused_kernel(const FusedArgs a)
 {
     extern __shared__ __align__(128) uint8_t smem[];
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem);   // copy of the slice landed
-    uint64_t *amaxd = full + kMaxStages;                   // all compute warps wrote their amax
-    uint64_t *ready = amaxd + kMaxStages;                  // every CTA published the group
-    uint64_t *freed = ready + kMaxStages;                  // all compute warps done with the slice
-    uint8_t *buf = smem + 256;
-    __shared__ uint32_t s_amax[kMaxStages];                // group amax bits, set before ready
-    __shared__ uint32_t s_part[kMaxStages][kFusedComputeWarps];
-    __shared__ uint32_t s_m4[kMaxStages];
+    uint64_t *sfull = reinterpret_cast<uint64_t *>(smem);
+    uint64_t *sfreed = sfull + kMaxStages;
+    uint64_t *qfull = sfreed + kMaxStages;
+    uint64_t *qfreed = qfull + kMaxStages;
+    uint64_t *ready = qfreed + kMaxStages;              // kReadyRing barriers
+    uint8_t *buf = smem + 512;
+    __shared__ uint32_t s_amax[kReadyRing];             // group amax bits, set before ready
+    __shared__ uint32_t s_scout_part[2];
+    __shared__ int s_scout_stop;
+    __shared__ int s_scouted;                           // groups whose slot this CTA published
     __shared__ int s_abort;
     volatile int *abort_flag = &s_abort;
+    volatile int *scouted = &s_scouted;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t P = gridDim.x;
@@ -376,141 +385,163 @@ nvfp4_fused_kernel(const FusedArgs a)
     const int64_t my_n = max((int64_t)0, min(a.slice, a.nb - my_lo));   // multiple of 32
     const uint32_t bytes = (uint32_t)(my_n * 32);
     const int64_t stage_bytes = a.slice * 32;
-    const int L = a.stages, LA = a.lookahead;
+    const int LS = a.sstages, LQ = a.qstages, D = a.distance;
     const int64_t G = a.n_groups;
+    uint8_t *sbuf = buf;                                // scout ring
+    uint8_t *qbuf = buf + LS * stage_bytes;             // quantize ring
 
     if (threadIdx.x == 0) {
-        for (int k = 0; k < L; ++k) {
-            mbar_init(full + k, 1);
-            mbar_init(amaxd + k, kFusedComputeWarps);
-            mbar_init(ready + k, 1);
-            mbar_init(freed + k, kFusedComputeWarps);
-            s_m4[k] = 0;
+        for (int k = 0; k < kMaxStages; ++k) {
+            mbar_init(sfull + k, 1);
+            mbar_init(sfreed + k, 2);                   // both scout warps
+            mbar_init(qfull + k, 1);
+            mbar_init(qfreed + k, kFusedComputeWarps);
         }
+        for (int k = 0; k < kReadyRing; ++k)
+            mbar_init(ready + k, 1);
+        s_scouted = 0;
         s_abort = 0;
         fence_mbar_init();
     }
     __syncthreads();
 
+    const unsigned long long *src0 = reinterpret_cast<const unsigned long long *>(a.x);
+    (void)src0;
+
     if (warp == 0) {
         // -------------------------------------------------------- publisher
-        // Publishes this CTA's slice amax of each group as soon as the compute
-        // warps reduced it: one 64-bit store of (group tag, amax bits) into
-        // the CTA's slot, so value and tag become visible together and no
-        // fence is needed.  Group j is released to the compute warps once all
-        // P slots of j carry j's tag; the group amax is the max over slots.
-        int64_t next_pub = 0, next_ready = 0;
+        // Releases group j to the compute warps once all P slots of j carry
+        // j's tag; the group amax is the max over the slots.
+        if (bytes == 0)
+            return;                                     // no compute here to release
+        int64_t next_ready = 0;
         uint32_t idle = 0;
         while (next_ready < G) {
             bool progress = false;
-            int got = 0;
-            if (next_pub < G && lane == 0)
-                got = mbar_try_wait(amaxd + next_pub % L, (uint32_t)((next_pub / L) & 1)) ? 1 : 0;
-            if (__shfl_sync(0xFFFFFFFFu, got, 0)) {   // warp-uniform from here
-                if (lane == 0) {
-                    const int st = (int)(next_pub % L);
-                    uint32_t mx = 0;
-                    for (int w = 0; w < kFusedComputeWarps; ++w)
-                        mx = max(mx, s_part[st][w]);
-                    if (mx >= 0x7F80u)
-                        atomicOr(a.status, MXQ_DEV_NONFINITE_INPUT);
-                    const unsigned long long v = ((unsigned long long)(next_pub + 1) << 32) | mx;
-                    st_relaxed_u64(a.slots + next_pub * kMaxFusedCtas + blockIdx.x, v);
+            const int npoll = (int)min((int64_t)kPollGroups, (int64_t)*scouted - next_ready);
+            if (npoll > 0) {
+                uint32_t mx[kPollGroups];
+                bool all[kPollGroups];
+#pragma unroll
+                for (int q = 0; q < kPollGroups; ++q) {
+                    mx[q] = 0;
+                    all[q] = true;
+                    if (q < npoll) {
+                        const unsigned long long *sl = a.slots + (next_ready + q) * kMaxFusedCtas;
+                        const uint32_t tag = (uint32_t)(next_ready + q + 1);
+                        for (uint32_t c = lane; c < P; c += 32) {
+                            const unsigned long long v = ld_relaxed_u64(sl + c);
+                            all[q] = all[q] && ((uint32_t)(v >> 32) == tag);
+                            mx[q] = max(mx[q], (uint32_t)v);
+                        }
+                    }
                 }
-                ++next_pub;
-                progress = true;
-            }
-            if (next_ready < next_pub) {
-                const unsigned long long *sl = a.slots + next_ready * kMaxFusedCtas;
-                const uint32_t tag = (uint32_t)(next_ready + 1);
-                bool all = true;
-                uint32_t mx = 0;
-                for (uint32_t c = lane; c < P; c += 32) {
-                    const unsigned long long v = ld_relaxed_u64(sl + c);
-                    all = all && ((uint32_t)(v >> 32) == tag);
-                    mx = max(mx, (uint32_t)v);
-                }
-                if (__all_sync(0xFFFFFFFFu, all)) {
-                    mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+#pragma unroll
+                for (int q = 0; q < kPollGroups; ++q) {
+                    if (q >= npoll || !__all_sync(0xFFFFFFFFu, all[q]))
+                        break;
+                    const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, mx[q]);
                     if (lane == 0) {
-                        const int st = (int)(next_ready % L);
-                        s_amax[st] = mx;
+                        const int rs = (int)(next_ready % kReadyRing);
+                        s_amax[rs] = m;
                         if (blockIdx.x == 0)
-                            a.s2_out[next_ready] = __fdiv_rn(__uint_as_float(mx << 16), kGlobalDivisor);
-                        mbar_arrive(ready + st);
+                            a.s2_out[next_ready] = __fdiv_rn(__uint_as_float(m << 16), kGlobalDivisor);
+                        mbar_arrive(ready + rs);
                     }
                     ++next_ready;
                     progress = true;
                 }
             }
-            if (!progress)
-                __nanosleep(200);
             if (progress) {
                 idle = 0;
-            } else if (__any_sync(0xFFFFFFFFu, ++idle > (kSpinLimit >> 4) || *abort_flag)) {
-                if (lane == 0) {
-                    *abort_flag = 1;
-                    atomicOr(a.status, MXQ_DEV_WAIT_TIMEOUT);
+            } else {
+                if (__any_sync(0xFFFFFFFFu, ++idle > (kSpinLimit >> 4) || *abort_flag)) {
+                    if (lane == 0) {
+                        *abort_flag = 1;
+                        atomicOr(a.status, MXQ_DEV_WAIT_TIMEOUT);
+                    }
+                    break;
                 }
-                break;
+                __nanosleep(256);
             }
         }
         return;
     }
     if (warp == 1) {
         // ----------------------------------------------------------- loader
-        if (lane != 0)
+        // Scout copies run up to `distance` groups ahead of quantize copies;
+        // a group's quantize copy waits until the scouts are done with it.
+        if (lane != 0 || bytes == 0)
             return;
-        int64_t last_issued[kMaxStages];
+        int64_t s_next = 0, q_next = 0;
+        int64_t s_last[kMaxStages], q_last[kMaxStages];
         for (int k = 0; k < kMaxStages; ++k)
-            last_issued[k] = -1;
-        auto issue = [&](int64_t g) {
-            if (bytes == 0)
-                return;
-            const int st = (int)(g % L);
-            fence_proxy_async_smem();
-            mbar_arrive_expect_tx(full + st, bytes);
-            bulk_g2s(buf + st * stage_bytes, a.x + (g * a.nb + my_lo) * 16, bytes, full + st);
-            last_issued[st] = g;
-        };
-        for (int64_t g = 0; g < G && g < L; ++g)
-            issue(g);
-        for (int64_t j = 0; j < G; ++j) {
-            const int st = (int)(j % L);
-            if (!wait_phase(freed + st, (uint32_t)((j / L) & 1), abort_flag))
+            s_last[k] = q_last[k] = -1;
+        uint32_t idle = 0;
+        while (q_next < G) {
+            bool progress = false;
+            if (s_next < G && s_next < q_next + D) {
+                const int st = (int)(s_next % LS);
+                if (s_next < LS || mbar_try_wait(sfreed + st, (uint32_t)(((s_next / LS) - 1) & 1))) {
+                    fence_proxy_async_smem();
+                    mbar_arrive_expect_tx(sfull + st, bytes);
+                    bulk_g2s(sbuf + st * stage_bytes, a.x + (s_next * a.nb + my_lo) * 16, bytes, sfull + st);
+                    s_last[st] = s_next;
+                    ++s_next;
+                    progress = true;
+                }
+            }
+            if (q_next < *scouted) {
+                const int st = (int)(q_next % LQ);
+                if (q_next < LQ || mbar_try_wait(qfreed + st, (uint32_t)(((q_next / LQ) - 1) & 1))) {
+                    fence_proxy_async_smem();
+                    mbar_arrive_expect_tx(qfull + st, bytes);
+                    bulk_g2s(qbuf + st * stage_bytes, a.x + (q_next * a.nb + my_lo) * 16, bytes, qfull + st);
+                    q_last[st] = q_next;
+                    ++q_next;
+                    progress = true;
+                }
+            }
+            if (progress) {
+                idle = 0;
+            } else if (++idle > kSpinLimit || *abort_flag) {
+                *abort_flag = 1;
+                atomicOr(a.status, MXQ_DEV_WAIT_TIMEOUT);
                 break;
-            if (a.m4_count && s_m4[st])
-                atomicAdd(a.m4_count + j, s_m4[st]);
-            s_m4[st] = 0;
-            if (j + L < G)
-                issue(j + L);
+            } else {
+                __nanosleep(200);
+            }
         }
         if (*abort_flag) {
-            atomicOr(a.status, MXQ_DEV_WAIT_TIMEOUT);
             // let this CTA's copies in flight land before its smem is released
-            for (int k = 0; k < L; ++k)
-                if (last_issued[k] >= 0)
+            for (int k = 0; k < kMaxStages; ++k) {
+                if (s_last[k] >= 0)
                     for (uint32_t n = 0; n < kSpinLimit; ++n)
-                        if (mbar_try_wait(full + k, (uint32_t)((last_issued[k] / L) & 1)))
+                        if (mbar_try_wait(sfull + k, (uint32_t)((s_last[k] / LS) & 1)))
                             break;
+                if (q_last[k] >= 0)
+                    for (uint32_t n = 0; n < kSpinLimit; ++n)
+                        if (mbar_try_wait(qfull + k, (uint32_t)((q_last[k] / LQ) & 1)))
+                            break;
+            }
         }
         return;
     }
-
-    // -------------------------------------------------------- compute warps
-    const int cw = warp - 2;
-    const int64_t n32 = my_n / 32;
-    for (int64_t t = 0; t < G + LA; ++t) {
-        const int64_t i = t, j = t - LA;
-        if (i < G) {
-            const int st = (int)(i % L);
+    if (warp < 4) {
+        // ----------------------------------------------------------- scouts
+        // The two scout warps meet at a named barrier twice per group; the
+        // decision to stop is taken from a flag snapshot written before the
+        // first meeting, so both warps always make the same choice.
+        const int sw = warp - 2;
+        for (int64_t g = 0; g < G; ++g) {
+            const int st = (int)(g % LS);
+            bool ok = true;
+            if (bytes)
+                ok = __all_sync(0xFFFFFFFFu, wait_phase(sfull + st, (uint32_t)((g / LS) & 1), abort_flag, 4000u));
             uint32_t m = 0;
-            if (bytes) {
-                const bool ok = __all_sync(0xFFFFFFFFu, wait_phase(full + st, (uint32_t)((i / L) & 1), abort_flag));
-                if (!ok)
-                    break;
-                const uint4 *v = reinterpret_cast<const uint4 *>(buf + st * stage_bytes);
-                for (int64_t u = lane + 32 * cw; u < my_n * 2; u += 32 * kFusedComputeWarps) {
+            if (ok && bytes) {
+                const uint4 *v = reinterpret_cast<const uint4 *>(sbuf + st * stage_bytes);
+                for (int64_t u = lane + 32 * sw; u < my_n * 2; u += 64) {
                     const uint4 q = v[u];
                     m = absmax_bf16x2(m, q.x);
                     m = absmax_bf16x2(m, q.y);
@@ -520,37 +551,64 @@ nvfp4_fused_kernel(const FusedArgs a)
             }
             const uint32_t r = __reduce_max_sync(0xFFFFFFFFu, fold_halves(m));
             if (lane == 0) {
-                s_part[st][cw] = r;
-                mbar_arrive(amaxd + st);
+                s_scout_part[sw] = r;
+                if (!ok)
+                    *abort_flag = 1;
+            }
+            if (sw == 0 && lane == 0)
+                s_scout_stop = *abort_flag;
+            named_barrier_sync(1, 64);                  // both parts written, stop decided
+            const int stop = s_scout_stop;
+            if (!stop && sw == 0 && lane == 0) {
+                const uint32_t mx = max(s_scout_part[0], s_scout_part[1]);
+                if (mx >= 0x7F80u)
+                    atomicOr(a.status, MXQ_DEV_NONFINITE_INPUT);
+                st_relaxed_u64(a.slots + g * kMaxFusedCtas + blockIdx.x,
+                               ((unsigned long long)(g + 1) << 32) | mx);
+                *scouted = (int)(g + 1);
+            }
+            named_barrier_sync(1, 64);                  // parts and snapshot may be rewritten
+            if (stop)
+                break;
+            if (lane == 0 && bytes)
+                mbar_arrive(sfreed + st);
+        }
+        return;
+    }
+
+    // -------------------------------------------------------- compute warps
+    if (bytes == 0)
+        return;
+    const int cw = warp - 4;
+    const int64_t n32 = my_n / 32;
+    for (int64_t j = 0; j < G; ++j) {
+        const int st = (int)(j % LQ);
+        const int rs = (int)(j % kReadyRing);
+        bool ok = wait_phase(ready + rs, (uint32_t)((j / kReadyRing) & 1), abort_flag, 500u);
+        ok = ok && wait_phase(qfull + st, (uint32_t)((j / LQ) & 1), abort_flag, 500u);
+        if (!__all_sync(0xFFFFFFFFu, ok))
+            break;
+        const GroupConst gc = make_group_const(s_amax[rs]);
+        const uint4 *v = reinterpret_cast<const uint4 *>(qbuf + st * stage_bytes);
+        uint32_t cnt = 0;
+        for (int64_t k32 = cw; k32 < n32; k32 += kFusedComputeWarps) {
+            const int64_t k = k32 * 32 + lane;
+            const BlockOut o = quantize_block<FOUR_SIX>(v[2 * k], v[2 * k + 1], gc);
+            const int64_t gb = j * a.nb + my_lo + k;
+            a.codes[gb] = o.codes;
+            a.scales[gb] = (uint8_t)o.scale;
+            const uint32_t word = __ballot_sync(0xFFFFFFFFu, o.m4);
+            if (lane == 0) {
+                if (a.mbits)
+                    a.mbits[(gb - lane) >> 5] = word;
+                cnt += __popc(word);
             }
         }
-        if (j >= 0) {
-            const int st = (int)(j % L);
-            const bool ok = __all_sync(0xFFFFFFFFu, wait_phase(ready + st, (uint32_t)((j / L) & 1), abort_flag));
-            if (!ok)
-                break;
-            const GroupConst gc = make_group_const(s_amax[st]);
-            const uint4 *v = reinterpret_cast<const uint4 *>(buf + st * stage_bytes);
-            uint32_t cnt = 0;
-            for (int64_t k32 = cw; k32 < n32; k32 += kFusedComputeWarps) {
-                const int64_t k = k32 * 32 + lane;
-                const BlockOut o = quantize_block<FOUR_SIX>(v[2 * k], v[2 * k + 1], gc);
-                const int64_t gb = j * a.nb + my_lo + k;
-                a.codes[gb] = o.codes;
-                a.scales[gb] = (uint8_t)o.scale;
-                const uint32_t word = __ballot_sync(0xFFFFFFFFu, o.m4);
-                if (lane == 0) {
-                    if (a.mbits)
-                        a.mbits[(gb - lane) >> 5] = word;
-                    cnt += __popc(word);
-                }
-            }
-            __syncwarp();
-            if (lane == 0) {
-                if (cnt)
-                    atomicAdd(&s_m4[st], cnt);
-                mbar_arrive(freed + st);
-            }
+        __syncwarp();
+        if (lane == 0) {
+            if (a.m4_count && cnt)
+                atomicAdd(a.m4_count + j, cnt);
+            mbar_arrive(qfreed + st);
         }
     }
 }
@@ -599,16 +657,19 @@ cudaError_t launch_nvfp4_fused(const uint16_t *x, int64_t n_groups, int64_t nb, 
     int64_t slice = (nb + sms - 1) / sms;
     slice = (slice + 31) / 32 * 32;
     const int64_t slice_bytes = slice * 32;
-    const int64_t avail = (int64_t)max_optin - 256 - 2048;   // barriers + static smem margin
-    int64_t L = avail / slice_bytes;
-    if (L < 1)
+    const int64_t avail = (int64_t)max_optin - 512 - 2048;   // barriers + static smem margin
+    const int64_t stages = avail / slice_bytes;               // scout + quantize buffers
+    if (stages < 2)
         return cudaErrorNotSupported;
-    if (L > 8)
-        L = 8;
-    if (L > n_groups)
-        L = n_groups;
-    const int LA = L >= 4 ? 2 : (L >= 2 ? 1 : 0);
-    const size_t dyn = 256 + (size_t)(L * slice_bytes);
+    // Split the buffers between the two rings; the scouts run `distance`
+    // groups ahead of the compute warps.
+    int LS = (int)(stages / 2), LQ = (int)(stages - stages / 2);
+    if (LS > kMaxStages)
+        LS = kMaxStages;
+    if (LQ > kMaxStages)
+        LQ = kMaxStages;
+    const int D = LQ + 2 <= kReadyRing - 1 - LQ ? LQ + 2 : kReadyRing - 1 - LQ;
+    const size_t dyn = 512 + (size_t)(LS + LQ) * (size_t)slice_bytes;
     const void *fn = four_six ? (const void *)nvfp4_fused_kernel<true> : (const void *)nvfp4_fused_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
     if (e != cudaSuccess)
@@ -624,8 +685,9 @@ cudaError_t launch_nvfp4_fused(const uint16_t *x, int64_t n_groups, int64_t nb, 
     args.n_groups = n_groups;
     args.nb = nb;
     args.slice = slice;
-    args.stages = (int)L;
-    args.lookahead = LA;
+    args.sstages = LS;
+    args.qstages = LQ;
+    args.distance = D;
     args.slots = slots;
     args.status = status;
     args.codes = reinterpret_cast<uint2 *>(codes);
