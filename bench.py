@@ -39,7 +39,7 @@ Q_BYTES = 2.0 + 0.5 + 1.0 / 16
 V_BYTES = 2.0 + 0.5 + 1.0 / 16
 STEP_BYTES_PER_ELEM = Q_BYTES + V_BYTES
 # Kernels of this library launched per call (cudaMemsetAsync not counted).
-KERNELS_PER_QUANTIZE_NVFP4 = 2   # group amax, block quantizer
+KERNELS_PER_QUANTIZE_NVFP4 = 1   # the single-pass kernel (full-size stacks)
 KERNELS_PER_VERIFY = 2           # chunk reduction, per-tensor finalize
 METRIC = "NVFP4 4/6-optimal quantize+verify HBM GB/s and % of B200 peak (1 GPU)"
 WORKLOAD = ("one full-size routed-expert layer, NVFP4 4/6-optimal quantize + verify: "
@@ -332,7 +332,7 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
@@ -428,7 +428,8 @@ def main():
                    "quality": quality},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "kernel": "mxq_quantize_nvfp4 on gate_up (group amax + block quantizer)",
+                     "kernel": "nvfp4_fused_kernel (mxq_quantize_nvfp4 on the gate_up stack)",
+                     "algorithmic_bytes_per_launch": gu_elems * Q_BYTES,
                      "peak_kind": peak_kind},
         "gpu_launches": args.steps * 2 * (KERNELS_PER_QUANTIZE_NVFP4 + KERNELS_PER_VERIFY),
         "clocks": clk.summary(),

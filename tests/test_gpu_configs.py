@@ -1,0 +1,165 @@
+"""Full-size and sweep parity for every workload of the quantizer, through
+the C ABI, against the CPU oracle: bit-exact codes / scales / global
+scales / M bits on sampled experts, layers or rows the oracle computes, and
+properties that hold at any size.
+
+Workloads (shapes of the model cards; synthetic values):
+* routed-expert layer, NVFP4 4/6: gate_up [512, 1536, 2048] + down
+  [512, 2048, 768], per-expert sigma log-uniform in [0.005, 0.05], 0.05 %
+  outliers at 8 sigma (the benchmark's configuration);
+* shared-expert MXFP8 rewrite: gate/up [2560, 2048] + down [2048, 1280],
+  dense and MTP-style zero-padded 640 -> 1280;
+* mixed-format layers: NVFP4 4/6 and MXFP4 layers side by side, Student-t
+  tail mix;
+* dynamic activations: token tiles [T, 2048], T in {1, 16, 256, 4096, 65536}.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mxfp_block_scaled_b200 import layers, mxq, workloads
+
+pytestmark = pytest.mark.gpu
+
+RTOL_STATS = 1e-6
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _setup():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from mxfp_block_scaled_b200 import build
+    build.build()
+    mxq.load()
+    oracle.build()
+
+
+def bits(t):
+    return workloads.bf16_bits(t)
+
+
+def unpack_mbits(words, n):
+    w = words.cpu().numpy().view(np.uint32)
+    return np.unpackbits(w.view(np.uint8), bitorder="little")[:n]
+
+
+def test_full_size_routed_layer_sampled_experts():
+    """The benchmark's exact launch: full 512-expert stacks through
+    mxq_quantize_nvfp4 and mxq_dequant_relerr; experts 0, 255 and 511 (and
+    their unstacked tensors) checked against the oracle."""
+    gu, dn, _ = workloads.full_moe_layer(seed=0, device="cuda")
+    res = layers.quantize_routed_layer(gu, dn, fmt="nvfp4", mode="four_six")
+    torch.cuda.synchronize()
+    for name, x in (("gate_up", gu), ("down", dn)):
+        q = res[name]
+        assert int(q["status"].item()) == 0
+        E, R, C = x.shape
+        nb = R * C // 16
+        gm = unpack_mbits(q["mbits"], E * nb).reshape(E, nb)
+        tps = 2 if name == "gate_up" else 1
+        for e in (0, 255, 511):
+            xb = bits(x[e:e + 1])
+            c, s, s2, m4 = oracle.quantize_nvfp4(xb, mode=1)
+            assert np.array_equal(q["codes"][e].cpu().numpy(), c[0]), (name, e)
+            assert np.array_equal(q["scales"][e].cpu().numpy(), s[0]), (name, e)
+            assert q["s2"][e].cpu().numpy().view(np.uint32) == s2.view(np.uint32)[0]
+            assert np.array_equal(gm[e], m4[0]), (name, e)
+            assert q["m4_count"][e].item() == int(m4.sum())
+            oe, orf = oracle.dequant_relerr(xb, c, s, s2, "nvfp4", tps, R // tps, C, tps)
+            got_e = q["sum_sq_err"][e * tps:(e + 1) * tps].cpu().numpy()
+            got_r = q["sum_sq_ref"][e * tps:(e + 1) * tps].cpu().numpy()
+            np.testing.assert_allclose(got_e, oe, rtol=RTOL_STATS)
+            np.testing.assert_allclose(got_r, orf, rtol=RTOL_STATS)
+    # census over all 1536 unstacked tensors; gate/up of an expert share s2
+    mean, mx, n = layers.relerr_census([res])
+    assert n == 512 * 3
+    assert 0.05 < mean < 0.12 and mx < 0.2
+    ex = layers.unstack_expert(res, 7)
+    assert ex["gate"][0].shape == (768, 1024) and ex["up"][1].shape == (768, 128)
+    assert ex["gate"][0].data_ptr() == res["gate_up"]["codes"][7].data_ptr()
+
+
+@pytest.mark.parametrize("pad_up", [True, False])
+def test_shared_expert_mxfp8_full_size_dense_and_padded(pad_up):
+    for padded in (False, True):
+        gu, dn = workloads.shared_expert_layer(seed=11, device="cuda", padded=padded,
+                                               pad_up=pad_up)
+        for t, name in ((gu, "gate_up"), (dn, "down")):
+            q = mxq.quantize_mx(t, "mxfp8")
+            torch.cuda.synchronize()
+            assert int(q["status"].item()) == 0
+            c, s = oracle.quantize_mx(bits(t), "mxfp8")
+            assert np.array_equal(q["codes"].cpu().numpy(), c), (name, padded)
+            assert np.array_equal(q["scales"].cpu().numpy(), s), (name, padded)
+            err, ref, rel = mxq.dequant_relerr(t, q["codes"], q["scales"], None, "mxfp8", 1,
+                                               *t.shape)
+            assert 0.025 < float(rel[0]) < 0.028      # the pages' MXFP8 sanity band
+        if padded:
+            qg = mxq.quantize_mx(gu, "mxfp8")
+            qd = mxq.quantize_mx(dn, "mxfp8")
+            assert not qg["codes"][640:1280].any() and not qg["scales"][640:1280].any()
+            if pad_up:
+                assert not qg["codes"][1920:].any() and not qg["scales"][1920:].any()
+            assert not qd["codes"][:, 640:].any() and not qd["scales"][:, 20:].any()
+
+
+def test_mixed_format_layers_reduced_experts():
+    """Two layers, one NVFP4 4/6 and one MXFP4 (reduced expert count so the
+    oracle covers every byte), Student-t tail mix."""
+    lay = [workloads.student_t_mix_layer(seed=s, device="cuda", experts=4) for s in (0, 1)]
+    res = layers.quantize_mixed(lay, ["nvfp4", "mxfp4"])
+    torch.cuda.synchronize()
+    for (gu, dn), fmt, r in zip(lay, ["nvfp4", "mxfp4"], res):
+        for name, x in (("gate_up", gu), ("down", dn)):
+            q = r[name]
+            xb = bits(x)
+            if fmt == "nvfp4":
+                c, s, s2, _ = oracle.quantize_nvfp4(xb, mode=1)
+                assert np.array_equal(q["s2"].cpu().numpy().view(np.uint32), s2.view(np.uint32))
+            else:
+                c, s = oracle.quantize_mx(xb, "mxfp4")
+            assert np.array_equal(q["codes"].cpu().numpy(), c), (fmt, name)
+            assert np.array_equal(q["scales"].cpu().numpy(), s), (fmt, name)
+    mean, mx, n = layers.relerr_census(res)
+    assert n == 2 * 4 * 3 and mx < 0.25
+
+
+@pytest.mark.parametrize("T", [1, 16, 256, 4096])
+def test_activation_sweep_exact(T):
+    a = workloads.activation_tile(T, seed=100 + T, device="cuda")
+    o = mxq.quantize_act(a, "nvfp4")
+    o8 = mxq.quantize_act(a, "mxfp8")
+    torch.cuda.synchronize()
+    c, s, s2, _ = oracle.quantize_nvfp4(bits(a).reshape(1, T, -1), mode=0)
+    assert o["input_scale"].cpu().numpy().view(np.uint32)[0] == s2.view(np.uint32)[0]
+    assert np.array_equal(o["codes"].cpu().numpy(), c.reshape(T, -1))
+    assert np.array_equal(o["scales"].cpu().numpy(), s.reshape(T, -1))
+    c8, s8 = oracle.quantize_mx(bits(a), "mxfp8")
+    assert np.array_equal(o8["codes"].cpu().numpy(), c8)
+    assert np.array_equal(o8["scales"].cpu().numpy(), s8)
+
+
+def test_activation_65536_tokens_sampled_rows():
+    """The largest tile (268 MB, beyond L2): input_scale from the closed form,
+    and sampled rows bit-exact: the oracle quantizes the sampled rows together
+    with the row that holds the tile amax, which fixes the same input_scale."""
+    T = 65536
+    a = workloads.activation_tile(T, seed=7, device="cuda")
+    o = mxq.quantize_act(a, "nvfp4")
+    o8 = mxq.quantize_act(a, "mxfp8")
+    torch.cuda.synchronize()
+    assert int(o["status"].item()) == 0
+    absmax = a.abs().amax(dim=1)
+    r_amax = int(torch.argmax(absmax).item())
+    amax = float(absmax[r_amax].float().item())
+    assert o["input_scale"].cpu().numpy()[0] == np.float32(amax) / np.float32(2688.0)
+    rows = sorted({0, 1, 4097, 33333, T - 1, r_amax})
+    sub = bits(a[rows])
+    c, s, s2, _ = oracle.quantize_nvfp4(sub.reshape(1, len(rows), -1), mode=0)
+    assert s2[0] == o["input_scale"].cpu().numpy()[0]
+    assert np.array_equal(o["codes"][rows].cpu().numpy(), c.reshape(len(rows), -1))
+    assert np.array_equal(o["scales"][rows].cpu().numpy(), s.reshape(len(rows), -1))
+    c8, s8 = oracle.quantize_mx(sub, "mxfp8")
+    assert np.array_equal(o8["codes"][rows].cpu().numpy(), c8)
+    assert np.array_equal(o8["scales"][rows].cpu().numpy(), s8)
