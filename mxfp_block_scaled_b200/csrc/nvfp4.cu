@@ -371,7 +371,7 @@ nvfp4_fused_kernel(const FusedArgs a)
     uint64_t *qfreed = qfull + kMaxStages;
     uint64_t *ready = qfreed + kMaxStages;              // kReadyRing barriers
     uint8_t *buf = smem + 512;
-    __shared__ uint32_t s_amax[kReadyRing];             // group amax bits, set before ready
+    __shared__ GroupConst s_gc[kReadyRing];             // group constants, set before ready
     __shared__ uint32_t s_scout_part[2];
     __shared__ int s_scout_stop;
     __shared__ int s_scouted;                           // groups whose slot this CTA published
@@ -443,9 +443,9 @@ nvfp4_fused_kernel(const FusedArgs a)
                     const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, mx[q]);
                     if (lane == 0) {
                         const int rs = (int)(next_ready % kReadyRing);
-                        s_amax[rs] = m;
+                        s_gc[rs] = make_group_const(m);
                         if (blockIdx.x == 0)
-                            a.s2_out[next_ready] = __fdiv_rn(__uint_as_float(m << 16), kGlobalDivisor);
+                            a.s2_out[next_ready] = s_gc[rs].s2;
                         mbar_arrive(ready + rs);
                     }
                     ++next_ready;
@@ -588,19 +588,22 @@ nvfp4_fused_kernel(const FusedArgs a)
         ok = ok && wait_phase(qfull + st, (uint32_t)((j / LQ) & 1), abort_flag, 500u);
         if (!__all_sync(0xFFFFFFFFu, ok))
             break;
-        const GroupConst gc = make_group_const(s_amax[rs]);
+        const GroupConst gc = s_gc[rs];
         const uint4 *v = reinterpret_cast<const uint4 *>(qbuf + st * stage_bytes);
+        const int64_t gb0 = j * a.nb + my_lo;             // first block of the slice
+        uint2 *codes = a.codes + gb0;
+        uint8_t *scales = a.scales + gb0;
+        uint32_t *mbits = a.mbits ? a.mbits + (gb0 >> 5) : nullptr;
         uint32_t cnt = 0;
-        for (int64_t k32 = cw; k32 < n32; k32 += kFusedComputeWarps) {
-            const int64_t k = k32 * 32 + lane;
+        for (int k32 = cw; k32 < (int)n32; k32 += kFusedComputeWarps) {
+            const int k = k32 * 32 + lane;
             const BlockOut o = quantize_block<FOUR_SIX>(v[2 * k], v[2 * k + 1], gc);
-            const int64_t gb = j * a.nb + my_lo + k;
-            a.codes[gb] = o.codes;
-            a.scales[gb] = (uint8_t)o.scale;
+            codes[k] = o.codes;
+            scales[k] = (uint8_t)o.scale;
             const uint32_t word = __ballot_sync(0xFFFFFFFFu, o.m4);
             if (lane == 0) {
-                if (a.mbits)
-                    a.mbits[(gb - lane) >> 5] = word;
+                if (mbits)
+                    mbits[k32] = word;
                 cnt += __popc(word);
             }
         }
