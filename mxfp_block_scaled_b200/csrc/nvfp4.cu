@@ -329,6 +329,7 @@ nvfp4_quant_kernel(const uint4 *__restrict__ x, int64_t n_groups, int64_t nb,
 struct FusedArgs {
     const uint16_t *x;
     int64_t n_groups, nb, slice;   // blocks per group, blocks per CTA slice
+    int teams, team_size;          // the grid is `teams` teams of `team_size` CTAs
     int sstages, qstages, distance;
     uint32_t *status;
     unsigned long long *slots;     // [n_groups][kMaxFusedCtas] (tag << 32 | slice amax bits)
@@ -380,13 +381,19 @@ nvfp4_fused_kernel(const FusedArgs a)
     volatile int *scouted = &s_scouted;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t P = gridDim.x;
-    const int64_t my_lo = (int64_t)blockIdx.x * a.slice;
+    // Team `team` takes groups team, team + teams, ...; rank is this CTA's
+    // place in the team and picks its slice of each of those groups.
+    const int team = (int)blockIdx.x / a.team_size, rank = (int)blockIdx.x % a.team_size;
+    if (team >= a.teams)
+        return;                                         // spare CTA (whole CTA: no barrier missed)
+    const uint32_t P = (uint32_t)a.team_size;
+    const int64_t my_lo = (int64_t)rank * a.slice;
     const int64_t my_n = max((int64_t)0, min(a.slice, a.nb - my_lo));   // multiple of 32
     const uint32_t bytes = (uint32_t)(my_n * 32);
     const int64_t stage_bytes = a.slice * 32;
     const int LS = a.sstages, LQ = a.qstages, D = a.distance;
-    const int64_t G = a.n_groups;
+    const int64_t G = a.n_groups > team ? (a.n_groups - team + a.teams - 1) / a.teams : 0;
+    auto group_of = [&](int64_t i) -> int64_t { return team + i * a.teams; };
     uint8_t *sbuf = buf;                                // scout ring
     uint8_t *qbuf = buf + LS * stage_bytes;             // quantize ring
 
@@ -427,8 +434,9 @@ nvfp4_fused_kernel(const FusedArgs a)
                     mx[q] = 0;
                     all[q] = true;
                     if (q < npoll) {
-                        const unsigned long long *sl = a.slots + (next_ready + q) * kMaxFusedCtas;
-                        const uint32_t tag = (uint32_t)(next_ready + q + 1);
+                        const int64_t gq = group_of(next_ready + q);
+                        const unsigned long long *sl = a.slots + gq * kMaxFusedCtas;
+                        const uint32_t tag = (uint32_t)(gq + 1);
                         for (uint32_t c = lane; c < P; c += 32) {
                             const unsigned long long v = ld_relaxed_u64(sl + c);
                             all[q] = all[q] && ((uint32_t)(v >> 32) == tag);
@@ -444,8 +452,8 @@ nvfp4_fused_kernel(const FusedArgs a)
                     if (lane == 0) {
                         const int rs = (int)(next_ready % kReadyRing);
                         s_gc[rs] = make_group_const(m);
-                        if (blockIdx.x == 0)
-                            a.s2_out[next_ready] = s_gc[rs].s2;
+                        if (rank == 0)
+                            a.s2_out[group_of(next_ready)] = s_gc[rs].s2;
                         mbar_arrive(ready + rs);
                     }
                     ++next_ready;
@@ -485,7 +493,7 @@ nvfp4_fused_kernel(const FusedArgs a)
                 if (s_next < LS || mbar_try_wait(sfreed + st, (uint32_t)(((s_next / LS) - 1) & 1))) {
                     fence_proxy_async_smem();
                     mbar_arrive_expect_tx(sfull + st, bytes);
-                    bulk_g2s(sbuf + st * stage_bytes, a.x + (s_next * a.nb + my_lo) * 16, bytes, sfull + st);
+                    bulk_g2s(sbuf + st * stage_bytes, a.x + (group_of(s_next) * a.nb + my_lo) * 16, bytes, sfull + st);
                     s_last[st] = s_next;
                     ++s_next;
                     progress = true;
@@ -496,7 +504,7 @@ nvfp4_fused_kernel(const FusedArgs a)
                 if (q_next < LQ || mbar_try_wait(qfreed + st, (uint32_t)(((q_next / LQ) - 1) & 1))) {
                     fence_proxy_async_smem();
                     mbar_arrive_expect_tx(qfull + st, bytes);
-                    bulk_g2s(qbuf + st * stage_bytes, a.x + (q_next * a.nb + my_lo) * 16, bytes, qfull + st);
+                    bulk_g2s(qbuf + st * stage_bytes, a.x + (group_of(q_next) * a.nb + my_lo) * 16, bytes, qfull + st);
                     q_last[st] = q_next;
                     ++q_next;
                     progress = true;
@@ -563,8 +571,9 @@ nvfp4_fused_kernel(const FusedArgs a)
                 const uint32_t mx = max(s_scout_part[0], s_scout_part[1]);
                 if (mx >= 0x7F80u)
                     atomicOr(a.status, MXQ_DEV_NONFINITE_INPUT);
-                st_relaxed_u64(a.slots + g * kMaxFusedCtas + blockIdx.x,
-                               ((unsigned long long)(g + 1) << 32) | mx);
+                const int64_t gg = group_of(g);
+                st_relaxed_u64(a.slots + gg * kMaxFusedCtas + rank,
+                               ((unsigned long long)(gg + 1) << 32) | mx);
                 *scouted = (int)(g + 1);
             }
             named_barrier_sync(1, 64);                  // parts and snapshot may be rewritten
@@ -590,7 +599,8 @@ nvfp4_fused_kernel(const FusedArgs a)
             break;
         const GroupConst gc = s_gc[rs];
         const uint4 *v = reinterpret_cast<const uint4 *>(qbuf + st * stage_bytes);
-        const int64_t gb0 = j * a.nb + my_lo;             // first block of the slice
+        const int64_t gj = group_of(j);
+        const int64_t gb0 = gj * a.nb + my_lo;            // first block of the slice
         uint2 *codes = a.codes + gb0;
         uint8_t *scales = a.scales + gb0;
         uint32_t *mbits = a.mbits ? a.mbits + (gb0 >> 5) : nullptr;
@@ -610,7 +620,7 @@ nvfp4_fused_kernel(const FusedArgs a)
         __syncwarp();
         if (lane == 0) {
             if (a.m4_count && cnt)
-                atomicAdd(a.m4_count + j, cnt);
+                atomicAdd(a.m4_count + gj, cnt);
             mbar_arrive(qfreed + st);
         }
     }
@@ -655,12 +665,31 @@ cudaError_t launch_nvfp4_fused(const uint16_t *x, int64_t n_groups, int64_t nb, 
         cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
         return cudaErrorNotSupported;
     const int sms = sm_count();
-    if (!coop || sms <= 0 || sms > kMaxFusedCtas || !slots)
+    if (!coop || sms <= 0 || !slots)
         return cudaErrorNotSupported;
-    int64_t slice = (nb + sms - 1) / sms;
-    slice = (slice + 31) / 32 * 32;
-    const int64_t slice_bytes = slice * 32;
+    // Teams: the largest number of teams whose slices (one per CTA of a
+    // team) still fit four stage buffers; small groups then get larger
+    // slices and fewer, cheaper hand-overs.
     const int64_t avail = (int64_t)max_optin - 512 - 2048;   // barriers + static smem margin
+    const int64_t target = avail / 4;
+    int teams = 1, team_size = sms;
+    int64_t slice = 0;
+    for (int h = (int)min((int64_t)sms, n_groups); h >= 1; --h) {
+        const int ts = sms / h;
+        if (ts > kMaxFusedCtas)
+            continue;
+        int64_t sl = (nb + ts - 1) / ts;
+        sl = (sl + 31) / 32 * 32;
+        if (sl * 32 <= target || h == 1) {
+            teams = h;
+            team_size = ts;
+            slice = sl;
+            break;
+        }
+    }
+    if (team_size > kMaxFusedCtas)
+        return cudaErrorNotSupported;
+    const int64_t slice_bytes = slice * 32;
     const int64_t stages = avail / slice_bytes;               // scout + quantize buffers
     if (stages < 2)
         return cudaErrorNotSupported;
@@ -688,6 +717,8 @@ cudaError_t launch_nvfp4_fused(const uint16_t *x, int64_t n_groups, int64_t nb, 
     args.n_groups = n_groups;
     args.nb = nb;
     args.slice = slice;
+    args.teams = teams;
+    args.team_size = team_size;
     args.sstages = LS;
     args.qstages = LQ;
     args.distance = D;
