@@ -29,9 +29,10 @@ size_t align_up(size_t v, size_t a);
 // Largest grid of the single-pass NVFP4 schedule (one CTA per SM).
 constexpr int kMaxFusedCtas = 256;
 
-// Workspace of the NVFP4 quantizer: per-group amax bits (two-pass schedule)
-// and per-group, per-CTA amax slots (single-pass schedule), each region
-// padded to 256 bytes.
+// Workspace of the NVFP4 quantizer: one word per group (the amax bits of the
+// two-pass schedule, or the arrival count of the single-pass schedule) and
+// per-group, per-CTA amax slots (single-pass schedule), each region padded
+// to 256 bytes.
 size_t nvfp4_workspace_bytes(int64_t n_groups);
 size_t nvfp4_slots_offset(int64_t n_groups);
 
@@ -42,7 +43,7 @@ cudaError_t launch_nvfp4_quant(const uint16_t *x, int64_t n_groups, int64_t nb, 
                                float *s2, uint32_t *mbits, int mbits_atomic,
                                uint32_t *m4_count, cudaStream_t s);
 cudaError_t launch_nvfp4_fused(const uint16_t *x, int64_t n_groups, int64_t nb, int four_six,
-                               unsigned long long *slots, uint8_t *codes, uint8_t *scales,
+                               unsigned long long *slots, uint32_t *arrived, uint8_t *codes, uint8_t *scales,
                                float *s2, uint32_t *mbits, uint32_t *m4_count, uint32_t *status,
                                cudaStream_t s);
 cudaError_t launch_mx_quant(const uint16_t *x, int64_t nblk32, int fmt, uint8_t *codes,

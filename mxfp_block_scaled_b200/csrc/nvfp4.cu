@@ -79,9 +79,13 @@ group_amax_kernel(const uint4 *__restrict__ x, int64_t n_groups, int64_t nb,
 // ---------------------------------------------------------------------------
 struct GroupConst {
     float s2;        // global scale
-    float den6, r6;  // RN32(6 s2), RN32(1 / den6)
-    float den4, r4;  // 4 s2 (exact), RN32(1 / den4)
-    int fast;        // den in the range where div_bf16 is exact
+    float2 den;      // (RN32(6 s2), 4 s2): the divisors of the two plans' block scales
+    float2 nr;       // (-RN32(1 / den.x), -RN32(1 / den.y)) when `tfast`
+    double s2h;      // s2 / 2 (exact), for the decision
+    int tfast;       // den in the range where the reciprocal quotient is exact
+    int qfast;       // s2 in [2^-50, 2^50]: every non-zero block scale gives a
+                     // divisor d = RN32(D s2) in [2^-59, 2^59], where the
+                     // reciprocal quotient of the block values is exact
 };
 
 __device__ __forceinline__ GroupConst make_group_const(uint32_t amax_bits)
@@ -89,11 +93,11 @@ __device__ __forceinline__ GroupConst make_group_const(uint32_t amax_bits)
     GroupConst c;
     const float amax = __uint_as_float(amax_bits << 16);
     c.s2 = __fdiv_rn(amax, kGlobalDivisor);
-    c.den6 = __fmul_rn(6.0f, c.s2);
-    c.den4 = __fmul_rn(4.0f, c.s2);
-    c.fast = (c.s2 >= 0x1p-100f && c.s2 <= 0x1p100f) ? 1 : 0;
-    c.r6 = c.fast ? __frcp_rn(c.den6) : 0.0f;
-    c.r4 = c.fast ? __frcp_rn(c.den4) : 0.0f;
+    c.den = make_float2(__fmul_rn(6.0f, c.s2), __fmul_rn(4.0f, c.s2));
+    c.tfast = (c.s2 >= 0x1p-100f && c.s2 <= 0x1p100f) ? 1 : 0;
+    c.qfast = (c.s2 >= 0x1p-50f && c.s2 <= 0x1p50f) ? 1 : 0;
+    c.nr = c.tfast ? make_float2(-__frcp_rn(c.den.x), -__frcp_rn(c.den.y)) : make_float2(0.0f, 0.0f);
+    c.s2h = 0.5 * (double)c.s2;
     return c;
 }
 
@@ -126,11 +130,10 @@ __device__ __forceinline__ Plan plan_from_quotients(const float2 (&x)[8], const 
     return p;
 }
 
-// y = RN32(x / d) with the reciprocal + FMA quotient, exact for d in
-// [2^-60, 2^60] (see div_bf16).
-__device__ __forceinline__ Plan make_plan_fast(const float2 (&x)[8], float d)
+// y = RN32(x / d) from r = RN32(1 / d) with the reciprocal + FMA quotient,
+// exact for d in [2^-60, 2^60] (see div_bf16).
+__device__ __forceinline__ Plan make_plan_fast(const float2 (&x)[8], float d, float r)
 {
-    const float r = __frcp_rn(d);
     const float2 d2 = make_float2(d, d), nr2 = make_float2(-r, -r);
     float2 y[8];
 #pragma unroll
@@ -142,8 +145,8 @@ __device__ __forceinline__ Plan make_plan_fast(const float2 (&x)[8], float d)
 __device__ __forceinline__ bool fast_scale(float d) { return d >= 0x1p-60f && d <= 0x1p60f; }
 
 // Any d: all codes 0 when d is 0 (D == 0, or D * s2 underflowed), IEEE
-// division outside the fast range.  Taken for rare blocks only.
-__device__ __noinline__ Plan make_plan_any(const float2 (&x)[8], float d)
+// division outside the fast range.
+__device__ __forceinline__ Plan make_plan_any(const float2 (&x)[8], float d)
 {
     if (!(d > 0.0f)) {
         Plan p;
@@ -153,7 +156,7 @@ __device__ __noinline__ Plan make_plan_any(const float2 (&x)[8], float d)
         return p;
     }
     if (fast_scale(d))
-        return make_plan_fast(x, d);
+        return make_plan_fast(x, d, __frcp_rn(d));
     float2 y[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j)
@@ -161,12 +164,12 @@ __device__ __noinline__ Plan make_plan_any(const float2 (&x)[8], float d)
     return plan_from_quotients(x, y);
 }
 
-// G_M = D (D s2 B - 2 A) in fp64, exact (see the file comment).
-__device__ __forceinline__ double plan_g(float D, float s2, const Plan &p)
+// G_M / 2 = D (D (s2/2) B - A) in fp64, exact (see the file comment); the
+// factor 1/2 is common to both plans.
+__device__ __forceinline__ double plan_g(float D, double s2h, const Plan &p)
 {
-    const double dS = (double)D * (double)s2;
-    const double P = fma(dS, (double)p.b, -2.0 * (double)p.a);
-    return (double)D * P;
+    const double dD = (double)D;
+    return dD * fma(dD * s2h, (double)p.b, -(double)p.a);
 }
 
 struct BlockOut {
@@ -175,55 +178,88 @@ struct BlockOut {
     bool m4;
 };
 
-template <bool FOUR_SIX>
-__device__ __forceinline__ BlockOut quantize_block(uint4 v0, uint4 v1, const GroupConst &gc)
+__device__ __forceinline__ void unpack_x(const uint32_t (&w)[8], float2 (&x)[8])
 {
-    BlockOut o;
-    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    uint32_t m = 0;
 #pragma unroll
     for (int j = 0; j < 8; ++j)
-        m = absmax_bf16x2(m, w[j]);
-    const float amax_b = __uint_as_float(fold_halves(m) << 16);
+        x[j] = make_float2(bf16_lo(w[j]), bf16_hi(w[j]));
+}
+
+// The general block quantizer: any s2, any block scale (zero, or a divisor
+// outside the fast range).  Taken for whole groups whose s2 is outside
+// [2^-50, 2^50] and for blocks whose scale code is 0 in a plan.
+template <bool FOUR_SIX>
+__device__ __noinline__ BlockOut quantize_block_general(uint4 v0, uint4 v1, float amax_b, const GroupConst gc)
+{
+    BlockOut o;
     if (!(gc.s2 > 0.0f)) {  // all-zero group
         o.codes = make_uint2(0u, 0u);
         o.scale = 0u;
         o.m4 = false;
         return o;
     }
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
     float2 x[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-        x[j] = make_float2(bf16_lo(w[j]), bf16_hi(w[j]));
+    unpack_x(w, x);
     float t6, t4;
-    if (gc.fast) {
-        t6 = div_bf16(amax_b, gc.den6, gc.r6);
-        t4 = div_bf16(amax_b, gc.den4, gc.r4);
+    if (gc.tfast) {
+        t6 = div_bf16(amax_b, gc.den.x, -gc.nr.x);
+        t4 = div_bf16(amax_b, gc.den.y, -gc.nr.y);
     } else {
-        t6 = __fdiv_rn(amax_b, gc.den6);
-        t4 = __fdiv_rn(amax_b, gc.den4);
+        t6 = __fdiv_rn(amax_b, gc.den.x);
+        t4 = __fdiv_rn(amax_b, gc.den.y);
     }
     const uint32_t sb = e4m3x2(t6, FOUR_SIX ? t4 : 0.0f);   // S6 low byte, S4 high
     const float2 D = f16x2_to_float2(e4m3x2_to_f16x2(sb));
     const float d6 = __fmul_rn(D.x, gc.s2), d4 = __fmul_rn(D.y, gc.s2);
-    // Both plans straight-line on the fast path (so their independent work
-    // interleaves); blocks whose scale is 0 or outside the fast range redo
-    // the affected plan exactly.
-    Plan p6 = make_plan_fast(x, d6);
+    const Plan p6 = make_plan_any(x, d6);
     if (!FOUR_SIX) {
-        if (!fast_scale(d6))
-            p6 = make_plan_any(x, d6);
         o.codes = p6.codes;
         o.scale = sb & 0xFFu;
         o.m4 = false;
         return o;
     }
-    Plan p4 = make_plan_fast(x, d4);
-    if (!fast_scale(d6) || !fast_scale(d4)) {
-        p6 = make_plan_any(x, d6);
-        p4 = make_plan_any(x, d4);
+    const Plan p4 = make_plan_any(x, d4);
+    const bool use4 = plan_g(D.y, gc.s2h, p4) < plan_g(D.x, gc.s2h, p6);
+    o.codes = use4 ? p4.codes : p6.codes;
+    o.scale = use4 ? (sb >> 8) : (sb & 0xFFu);
+    o.m4 = use4;
+    return o;
+}
+
+// One block of 16.  With s2 in [2^-50, 2^50] (`qfast`, uniform over a group)
+// and both scale codes non-zero, every divisor lies in the exact range of
+// the reciprocal quotient, so the two plans run straight-line with no range
+// tests; the block amax quotients of both plans share packed operations.
+template <bool FOUR_SIX>
+__device__ __forceinline__ BlockOut quantize_block(uint4 v0, uint4 v1, const GroupConst &gc)
+{
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    uint32_t m = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        m = absmax_bf16x2(m, w[j]);
+    const float amax_b = __uint_as_float(fold_halves(m) << 16);
+    if (!gc.qfast)
+        return quantize_block_general<FOUR_SIX>(v0, v1, amax_b, gc);
+    const float2 t = div2_bf16(make_float2(amax_b, amax_b), gc.den, gc.nr);
+    const uint32_t sb = e4m3x2(t.x, FOUR_SIX ? t.y : 1.0f);   // S6 low byte, S4 high
+    if ((sb & 0xFFu) == 0u || (sb & 0xFF00u) == 0u)
+        return quantize_block_general<FOUR_SIX>(v0, v1, amax_b, gc);
+    const float2 D = f16x2_to_float2(e4m3x2_to_f16x2(sb));
+    const float2 d = __fmul2_rn(D, make_float2(gc.s2, gc.s2));
+    float2 x[8];
+    unpack_x(w, x);
+    BlockOut o;
+    const Plan p6 = make_plan_fast(x, d.x, __frcp_rn(d.x));
+    if (!FOUR_SIX) {
+        o.codes = p6.codes;
+        o.scale = sb & 0xFFu;
+        o.m4 = false;
+        return o;
     }
-    const bool use4 = plan_g(D.y, gc.s2, p4) < plan_g(D.x, gc.s2, p6);
+    const Plan p4 = make_plan_fast(x, d.y, __frcp_rn(d.y));
+    const bool use4 = plan_g(D.y, gc.s2h, p4) < plan_g(D.x, gc.s2h, p6);
     o.codes = use4 ? p4.codes : p6.codes;
     o.scale = use4 ? (sb >> 8) : (sb & 0xFFu);
     o.m4 = use4;
@@ -311,13 +347,17 @@ nvfp4_quant_kernel(const uint4 *__restrict__ x, int64_t n_groups, int64_t nb,
 // M bits fill one word).  Each CTA walks the groups in order; its slice of
 // a group is brought into shared memory twice by bulk copies:
 //   scout copy     (ring of `sstages`): two scout warps reduce the slice
-//                  amax and publish it as one tagged 64-bit slot per group
-//                  and CTA (tag and value land together: no fence needed);
+//                  amax, publish it as one tagged 64-bit slot per group
+//                  and CTA (tag and value land together: no fence needed)
+//                  and then count the group's arrivals up by one;
 //   quantize copy  (ring of `qstages`), issued only after the scouts are
 //                  done with that group, `distance` groups behind them, so
 //                  it normally hits the L2 copy the scout read left behind:
 //                  21 compute warps quantize it once a publisher warp has
-//                  seen every CTA's slot for the group.
+//                  seen every CTA's slot for the group.  The publisher polls
+//                  only the one arrival word of a group; it reads the slots
+//                  (and checks their tags) once the count is complete, so
+//                  the polling of every CTA stays off the slots' L2 lines.
 // The grid-wide amax of a group is therefore resolved while the compute
 // warps work on earlier groups; its latency is off the critical path.
 // Roles hand over through mbarriers (sfull / sfreed: scout ring, qfull /
@@ -333,6 +373,7 @@ struct FusedArgs {
     int sstages, qstages, distance;
     uint32_t *status;
     unsigned long long *slots;     // [n_groups][kMaxFusedCtas] (tag << 32 | slice amax bits)
+    uint32_t *arrived;             // [n_groups] slots stored so far (starts at 0)
     uint2 *codes;
     uint8_t *scales;
     float *s2_out;
@@ -345,17 +386,20 @@ constexpr int kReadyRing = 16;   // > distance + qstages: ready phases never run
 constexpr int kPollGroups = 4;   // groups whose readiness one publisher poll tests
 
 // Bounded wait on an mbarrier phase that also gives up once another role of
-// the CTA has aborted.
-// The hardware may suspend the waiting thread for up to about `sleep_ns`
-// while the phase is incomplete, so idle roles do not spin.
+// the CTA has aborted.  With `sleep_ns` the phase is tested without blocking
+// and the warp sleeps about that long between tests: a blocking try_wait
+// with a suspend-time hint keeps polling inside the instruction and takes
+// issue slots from the compute warps of the same SM.
 __device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                            uint32_t sleep_ns = 0)
 {
     for (uint32_t i = 0; i < kSpinLimit; ++i) {
-        if (sleep_ns ? mbar_try_wait_sleep(bar, parity, sleep_ns) : mbar_try_wait(bar, parity))
+        if (sleep_ns ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity))
             return true;
         if (*abort_flag)
             return false;
+        if (sleep_ns)
+            __nanosleep(sleep_ns);
     }
     *abort_flag = 1;
     return false;
@@ -392,7 +436,8 @@ nvfp4_fused_kernel(const FusedArgs a)
     const uint32_t bytes = (uint32_t)(my_n * 32);
     const int64_t stage_bytes = a.slice * 32;
     const int LS = a.sstages, LQ = a.qstages, D = a.distance;
-    const int64_t G = a.n_groups > team ? (a.n_groups - team + a.teams - 1) / a.teams : 0;
+    // groups of this team (the launch keeps n_groups below 2^31)
+    const int G = a.n_groups > team ? (int)((a.n_groups - team + a.teams - 1) / a.teams) : 0;
     auto group_of = [&](int64_t i) -> int64_t { return team + i * a.teams; };
     uint8_t *sbuf = buf;                                // scout ring
     uint8_t *qbuf = buf + LS * stage_bytes;             // quantize ring
@@ -417,43 +462,41 @@ nvfp4_fused_kernel(const FusedArgs a)
 
     if (warp == 0) {
         // -------------------------------------------------------- publisher
-        // Releases group j to the compute warps once all P slots of j carry
-        // j's tag; the group amax is the max over the slots.
+        // Releases group j to the compute warps once all P CTAs have counted
+        // their arrival for j and all P slots of j carry j's tag; the group
+        // amax is the max over the slots.
         if (bytes == 0)
             return;                                     // no compute here to release
-        int64_t next_ready = 0;
+        int next_ready = 0;
         uint32_t idle = 0;
         while (next_ready < G) {
             bool progress = false;
-            const int npoll = (int)min((int64_t)kPollGroups, (int64_t)*scouted - next_ready);
+            const int npoll = min(kPollGroups, *scouted - next_ready);
             if (npoll > 0) {
-                uint32_t mx[kPollGroups];
-                bool all[kPollGroups];
-#pragma unroll
-                for (int q = 0; q < kPollGroups; ++q) {
-                    mx[q] = 0;
-                    all[q] = true;
-                    if (q < npoll) {
-                        const int64_t gq = group_of(next_ready + q);
-                        const unsigned long long *sl = a.slots + gq * kMaxFusedCtas;
-                        const uint32_t tag = (uint32_t)(gq + 1);
-                        for (uint32_t c = lane; c < P; c += 32) {
-                            const unsigned long long v = ld_relaxed_u64(sl + c);
-                            all[q] = all[q] && ((uint32_t)(v >> 32) == tag);
-                            mx[q] = max(mx[q], (uint32_t)v);
-                        }
+                uint32_t cnt = 0;
+                if (lane < npoll)
+                    cnt = ld_relaxed_u32(a.arrived + group_of(next_ready + lane));
+                const uint32_t full = __ballot_sync(0xFFFFFFFFu, lane < npoll && cnt >= P);
+                const int nfull = __ffs(~full) - 1;     // complete groups, in order
+                for (int q = 0; q < nfull; ++q) {
+                    const int64_t gq = group_of(next_ready);
+                    const unsigned long long *sl = a.slots + gq * kMaxFusedCtas;
+                    const uint32_t tag = (uint32_t)(gq + 1);
+                    bool all = true;
+                    uint32_t mx = 0;
+                    for (uint32_t c = lane; c < P; c += 32) {
+                        const unsigned long long v = ld_relaxed_u64(sl + c);
+                        all = all && ((uint32_t)(v >> 32) == tag);
+                        mx = max(mx, (uint32_t)v);
                     }
-                }
-#pragma unroll
-                for (int q = 0; q < kPollGroups; ++q) {
-                    if (q >= npoll || !__all_sync(0xFFFFFFFFu, all[q]))
-                        break;
-                    const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, mx[q]);
+                    if (!__all_sync(0xFFFFFFFFu, all))
+                        break;                          // a slot not visible yet: poll again
+                    const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, mx);
                     if (lane == 0) {
-                        const int rs = (int)(next_ready % kReadyRing);
+                        const int rs = next_ready & (kReadyRing - 1);
                         s_gc[rs] = make_group_const(m);
                         if (rank == 0)
-                            a.s2_out[group_of(next_ready)] = s_gc[rs].s2;
+                            a.s2_out[gq] = s_gc[rs].s2;
                         mbar_arrive(ready + rs);
                     }
                     ++next_ready;
@@ -481,32 +524,42 @@ nvfp4_fused_kernel(const FusedArgs a)
         // a group's quantize copy waits until the scouts are done with it.
         if (lane != 0 || bytes == 0)
             return;
-        int64_t s_next = 0, q_next = 0;
-        int64_t s_last[kMaxStages], q_last[kMaxStages];
+        // Stages and phase parities advance incrementally (no division).
+        int s_next = 0, q_next = 0, s_st = 0, q_st = 0;
+        uint32_t s_par = 0, q_par = 0;                  // parity of (next / ring size)
+        int s_last[kMaxStages], q_last[kMaxStages];     // phase parity of the copy in flight, or -1
         for (int k = 0; k < kMaxStages; ++k)
             s_last[k] = q_last[k] = -1;
         uint32_t idle = 0;
         while (q_next < G) {
             bool progress = false;
             if (s_next < G && s_next < q_next + D) {
-                const int st = (int)(s_next % LS);
-                if (s_next < LS || mbar_try_wait(sfreed + st, (uint32_t)(((s_next / LS) - 1) & 1))) {
+                if (s_next < LS || mbar_test_wait(sfreed + s_st, s_par ^ 1u)) {
                     fence_proxy_async_smem();
-                    mbar_arrive_expect_tx(sfull + st, bytes);
-                    bulk_g2s(sbuf + st * stage_bytes, a.x + (group_of(s_next) * a.nb + my_lo) * 16, bytes, sfull + st);
-                    s_last[st] = s_next;
+                    mbar_arrive_expect_tx(sfull + s_st, bytes);
+                    bulk_g2s(sbuf + s_st * stage_bytes, a.x + (group_of(s_next) * a.nb + my_lo) * 16, bytes,
+                             sfull + s_st);
+                    s_last[s_st] = (int)s_par;
                     ++s_next;
+                    if (++s_st == LS) {
+                        s_st = 0;
+                        s_par ^= 1u;
+                    }
                     progress = true;
                 }
             }
             if (q_next < *scouted) {
-                const int st = (int)(q_next % LQ);
-                if (q_next < LQ || mbar_try_wait(qfreed + st, (uint32_t)(((q_next / LQ) - 1) & 1))) {
+                if (q_next < LQ || mbar_test_wait(qfreed + q_st, q_par ^ 1u)) {
                     fence_proxy_async_smem();
-                    mbar_arrive_expect_tx(qfull + st, bytes);
-                    bulk_g2s(qbuf + st * stage_bytes, a.x + (group_of(q_next) * a.nb + my_lo) * 16, bytes, qfull + st);
-                    q_last[st] = q_next;
+                    mbar_arrive_expect_tx(qfull + q_st, bytes);
+                    bulk_g2s(qbuf + q_st * stage_bytes, a.x + (group_of(q_next) * a.nb + my_lo) * 16, bytes,
+                             qfull + q_st);
+                    q_last[q_st] = (int)q_par;
                     ++q_next;
+                    if (++q_st == LQ) {
+                        q_st = 0;
+                        q_par ^= 1u;
+                    }
                     progress = true;
                 }
             }
@@ -525,11 +578,11 @@ nvfp4_fused_kernel(const FusedArgs a)
             for (int k = 0; k < kMaxStages; ++k) {
                 if (s_last[k] >= 0)
                     for (uint32_t n = 0; n < kSpinLimit; ++n)
-                        if (mbar_try_wait(sfull + k, (uint32_t)((s_last[k] / LS) & 1)))
+                        if (mbar_try_wait(sfull + k, (uint32_t)s_last[k]))
                             break;
                 if (q_last[k] >= 0)
                     for (uint32_t n = 0; n < kSpinLimit; ++n)
-                        if (mbar_try_wait(qfull + k, (uint32_t)((q_last[k] / LQ) & 1)))
+                        if (mbar_try_wait(qfull + k, (uint32_t)q_last[k]))
                             break;
             }
         }
@@ -541,15 +594,17 @@ nvfp4_fused_kernel(const FusedArgs a)
         // decision to stop is taken from a flag snapshot written before the
         // first meeting, so both warps always make the same choice.
         const int sw = warp - 2;
-        for (int64_t g = 0; g < G; ++g) {
-            const int st = (int)(g % LS);
+        const int nvec = (int)(my_n * 2);               // 16-byte vectors of the slice
+        int st = 0;
+        uint32_t par = 0;
+        for (int g = 0; g < G; ++g) {
             bool ok = true;
             if (bytes)
-                ok = __all_sync(0xFFFFFFFFu, wait_phase(sfull + st, (uint32_t)((g / LS) & 1), abort_flag, 4000u));
+                ok = __all_sync(0xFFFFFFFFu, wait_phase(sfull + st, par, abort_flag, 500u));
             uint32_t m = 0;
             if (ok && bytes) {
                 const uint4 *v = reinterpret_cast<const uint4 *>(sbuf + st * stage_bytes);
-                for (int64_t u = lane + 32 * sw; u < my_n * 2; u += 64) {
+                for (int u = lane + 32 * sw; u < nvec; u += 64) {
                     const uint4 q = v[u];
                     m = absmax_bf16x2(m, q.x);
                     m = absmax_bf16x2(m, q.y);
@@ -574,6 +629,7 @@ nvfp4_fused_kernel(const FusedArgs a)
                 const int64_t gg = group_of(g);
                 st_relaxed_u64(a.slots + gg * kMaxFusedCtas + rank,
                                ((unsigned long long)(gg + 1) << 32) | mx);
+                red_relaxed_add_u32(a.arrived + gg, 1u);
                 *scouted = (int)(g + 1);
             }
             named_barrier_sync(1, 64);                  // parts and snapshot may be rewritten
@@ -581,6 +637,10 @@ nvfp4_fused_kernel(const FusedArgs a)
                 break;
             if (lane == 0 && bytes)
                 mbar_arrive(sfreed + st);
+            if (++st == LS) {
+                st = 0;
+                par ^= 1u;
+            }
         }
         return;
     }
@@ -589,12 +649,12 @@ nvfp4_fused_kernel(const FusedArgs a)
     if (bytes == 0)
         return;
     const int cw = warp - 4;
-    const int64_t n32 = my_n / 32;
-    for (int64_t j = 0; j < G; ++j) {
-        const int st = (int)(j % LQ);
-        const int rs = (int)(j % kReadyRing);
-        bool ok = wait_phase(ready + rs, (uint32_t)((j / kReadyRing) & 1), abort_flag, 500u);
-        ok = ok && wait_phase(qfull + st, (uint32_t)((j / LQ) & 1), abort_flag, 500u);
+    const int n32 = (int)(my_n / 32);
+    int st = 0, rs = 0;                                 // quantize stage and ready slot of group j
+    uint32_t qpar = 0, rpar = 0;                        // their phase parities
+    for (int j = 0; j < G; ++j) {
+        bool ok = wait_phase(ready + rs, rpar, abort_flag, 200u);
+        ok = ok && wait_phase(qfull + st, qpar, abort_flag, 200u);
         if (!__all_sync(0xFFFFFFFFu, ok))
             break;
         const GroupConst gc = s_gc[rs];
@@ -605,7 +665,7 @@ nvfp4_fused_kernel(const FusedArgs a)
         uint8_t *scales = a.scales + gb0;
         uint32_t *mbits = a.mbits ? a.mbits + (gb0 >> 5) : nullptr;
         uint32_t cnt = 0;
-        for (int k32 = cw; k32 < (int)n32; k32 += kFusedComputeWarps) {
+        for (int k32 = cw; k32 < n32; k32 += kFusedComputeWarps) {
             const int k = k32 * 32 + lane;
             const BlockOut o = quantize_block<FOUR_SIX>(v[2 * k], v[2 * k + 1], gc);
             codes[k] = o.codes;
@@ -622,6 +682,14 @@ nvfp4_fused_kernel(const FusedArgs a)
             if (a.m4_count && cnt)
                 atomicAdd(a.m4_count + gj, cnt);
             mbar_arrive(qfreed + st);
+        }
+        if (++st == LQ) {
+            st = 0;
+            qpar ^= 1u;
+        }
+        if (++rs == kReadyRing) {
+            rs = 0;
+            rpar ^= 1u;
         }
     }
 }
@@ -653,11 +721,11 @@ static int sm_count()
 // device does not suit the single-pass schedule; the caller then takes the
 // two-pass path.
 cudaError_t launch_nvfp4_fused(const uint16_t *x, int64_t n_groups, int64_t nb, int four_six,
-                               unsigned long long *slots, uint8_t *codes, uint8_t *scales,
+                               unsigned long long *slots, uint32_t *arrived, uint8_t *codes, uint8_t *scales,
                                float *s2, uint32_t *mbits, uint32_t *m4_count, uint32_t *status,
                                cudaStream_t s)
 {
-    if (n_groups <= 0 || nb <= 0 || nb % 32 != 0)
+    if (n_groups <= 0 || n_groups > 0x7FFFFFFF || nb <= 0 || nb % 32 != 0)
         return cudaErrorNotSupported;
     int dev = 0, coop = 0, max_optin = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -665,7 +733,7 @@ cudaError_t launch_nvfp4_fused(const uint16_t *x, int64_t n_groups, int64_t nb, 
         cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
         return cudaErrorNotSupported;
     const int sms = sm_count();
-    if (!coop || sms <= 0 || !slots)
+    if (!coop || sms <= 0 || !slots || !arrived)
         return cudaErrorNotSupported;
     // Teams: the largest number of teams whose slices (one per CTA of a
     // team) still fit four stage buffers; small groups then get larger
@@ -723,6 +791,7 @@ cudaError_t launch_nvfp4_fused(const uint16_t *x, int64_t n_groups, int64_t nb, 
     args.qstages = LQ;
     args.distance = D;
     args.slots = slots;
+    args.arrived = arrived;
     args.status = status;
     args.codes = reinterpret_cast<uint2 *>(codes);
     args.scales = scales;
