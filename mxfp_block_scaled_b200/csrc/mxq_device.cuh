@@ -16,18 +16,20 @@ namespace mxq {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// Running max of |x| over bf16x2 words, as bf16x2 bits (both halves >= 0).
-// NaN propagates, so a non-finite element leaves bits >= 0x7F80 (Inf or NaN)
-// in its half.
+// Running max of |x| over bf16x2 words, per half, in one instruction
+// (max.NaN.xorsign.abs): the magnitude bits hold max(|acc|, |w|), the sign
+// bit is garbage (the xor of the operands' signs) and is dropped by
+// fold_halves.  NaN propagates as the canonical NaN, so a non-finite element
+// leaves magnitude bits >= 0x7F80 (Inf or NaN) in its half.
 __device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t acc, uint32_t w)
 {
-    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162 *>(&acc);
-    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162 *>(&w);
-    const __nv_bfloat162 r = __hmax2_nan(a, __habs2(b));
-    return *reinterpret_cast<const uint32_t *>(&r);
+    uint32_t r;
+    asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(acc), "r"(w));
+    return r;
 }
-// Larger half of non-negative bf16x2 bits (bit patterns order like values).
-__device__ __forceinline__ uint32_t fold_halves(uint32_t m) { return max(m & 0xFFFFu, m >> 16); }
+// Larger magnitude of the two halves of an absmax_bf16x2 result, as bf16
+// bits (bit patterns of non-negative bf16 values order like the values).
+__device__ __forceinline__ uint32_t fold_halves(uint32_t m) { return max(m & 0x7FFFu, (m >> 16) & 0x7FFFu); }
 
 // ---- packed conversions (PTX ISA: cvt with .e2m1x2 / .e4m3x2) ------------
 // Two fp32 values -> one byte of two E2M1 codes (lo in the low nibble),

@@ -15,10 +15,11 @@ constexpr int kNvThreads = 256;
 constexpr int kNvTileBlocks = 512;
 
 // Single-pass NVFP4 schedule: one cooperative CTA per SM.
-// 21 compute warps (2 and 1 full rounds over the gate_up / down slices of
-// the full-size layer), a publisher warp, a loader warp and two scout warps.
+// 21 compute warps (two full rounds over a 1344-block slice), a publisher
+// warp, a loader warp and four scout warps (one per SM sub-partition).
 constexpr int kFusedComputeWarps = 21;
-constexpr int kFusedThreads = 32 * (kFusedComputeWarps + 4);
+constexpr int kFusedScoutWarps = 4;
+constexpr int kFusedThreads = 32 * (kFusedComputeWarps + 2 + kFusedScoutWarps);
 
 // Verifier: one CTA reduces one chunk of a tensor.
 constexpr int kVerifyThreads = 256;

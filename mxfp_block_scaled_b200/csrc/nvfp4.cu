@@ -417,7 +417,7 @@ nvfp4_fused_kernel(const FusedArgs a)
     uint64_t *ready = qfreed + kMaxStages;              // kReadyRing barriers
     uint8_t *buf = smem + 512;
     __shared__ GroupConst s_gc[kReadyRing];             // group constants, set before ready
-    __shared__ uint32_t s_scout_part[2];
+    __shared__ uint32_t s_scout_part[kFusedScoutWarps];
     __shared__ int s_scout_stop;
     __shared__ int s_scouted;                           // groups whose slot this CTA published
     __shared__ int s_abort;
@@ -445,7 +445,7 @@ nvfp4_fused_kernel(const FusedArgs a)
     if (threadIdx.x == 0) {
         for (int k = 0; k < kMaxStages; ++k) {
             mbar_init(sfull + k, 1);
-            mbar_init(sfreed + k, 2);                   // both scout warps
+            mbar_init(sfreed + k, kFusedScoutWarps);    // every scout warp
             mbar_init(qfull + k, 1);
             mbar_init(qfreed + k, kFusedComputeWarps);
         }
@@ -588,11 +588,11 @@ nvfp4_fused_kernel(const FusedArgs a)
         }
         return;
     }
-    if (warp < 4) {
+    if (warp < 2 + kFusedScoutWarps) {
         // ----------------------------------------------------------- scouts
-        // The two scout warps meet at a named barrier twice per group; the
+        // The scout warps meet at a named barrier twice per group; the
         // decision to stop is taken from a flag snapshot written before the
-        // first meeting, so both warps always make the same choice.
+        // first meeting, so every scout warp makes the same choice.
         const int sw = warp - 2;
         const int nvec = (int)(my_n * 2);               // 16-byte vectors of the slice
         int st = 0;
@@ -604,7 +604,8 @@ nvfp4_fused_kernel(const FusedArgs a)
             uint32_t m = 0;
             if (ok && bytes) {
                 const uint4 *v = reinterpret_cast<const uint4 *>(sbuf + st * stage_bytes);
-                for (int u = lane + 32 * sw; u < nvec; u += 64) {
+#pragma unroll 2
+                for (int u = lane + 32 * sw; u < nvec; u += 32 * kFusedScoutWarps) {
                     const uint4 q = v[u];
                     m = absmax_bf16x2(m, q.x);
                     m = absmax_bf16x2(m, q.y);
@@ -620,10 +621,12 @@ nvfp4_fused_kernel(const FusedArgs a)
             }
             if (sw == 0 && lane == 0)
                 s_scout_stop = *abort_flag;
-            named_barrier_sync(1, 64);                  // both parts written, stop decided
+            named_barrier_sync(1, 32 * kFusedScoutWarps);   // parts written, stop decided
             const int stop = s_scout_stop;
             if (!stop && sw == 0 && lane == 0) {
-                const uint32_t mx = max(s_scout_part[0], s_scout_part[1]);
+                uint32_t mx = 0;
+                for (int k = 0; k < kFusedScoutWarps; ++k)
+                    mx = max(mx, s_scout_part[k]);
                 if (mx >= 0x7F80u)
                     atomicOr(a.status, MXQ_DEV_NONFINITE_INPUT);
                 const int64_t gg = group_of(g);
@@ -632,7 +635,7 @@ nvfp4_fused_kernel(const FusedArgs a)
                 red_relaxed_add_u32(a.arrived + gg, 1u);
                 *scouted = (int)(g + 1);
             }
-            named_barrier_sync(1, 64);                  // parts and snapshot may be rewritten
+            named_barrier_sync(1, 32 * kFusedScoutWarps);   // parts and snapshot may be rewritten
             if (stop)
                 break;
             if (lane == 0 && bytes)
@@ -648,7 +651,7 @@ nvfp4_fused_kernel(const FusedArgs a)
     // -------------------------------------------------------- compute warps
     if (bytes == 0)
         return;
-    const int cw = warp - 4;
+    const int cw = warp - 2 - kFusedScoutWarps;
     const int n32 = (int)(my_n / 32);
     int st = 0, rs = 0;                                 // quantize stage and ready slot of group j
     uint32_t qpar = 0, rpar = 0;                        // their phase parities
