@@ -191,12 +191,12 @@ class Layer:
 
     def quantize(self, name):
         o = self.out[name]
-        self.mxq.mxq_quantize_nvfp4(o["x"], o["G"], o["R"], o["C"], "four_six", o["codes"], o["scales"],
-                                    o["s2"], o["mbits"], o["m4"], o["status"], o["wsq"])
+        self.mxq.mxq_quantize_nvfp4(o["x"], o["G"], o["R"], o["C"], "four_six", "linear", o["codes"],
+                                    o["scales"], o["s2"], o["mbits"], o["m4"], o["status"], o["wsq"])
 
     def verify(self, name):
         o = self.out[name]
-        self.mxq.mxq_dequant_relerr(o["x"], o["codes"], o["scales"], o["s2"], "nvfp4", o["nt"],
+        self.mxq.mxq_dequant_relerr(o["x"], o["codes"], o["scales"], o["s2"], "nvfp4", "linear", o["nt"],
                                     o["rows"], o["cols"], o["tps"], o["err"], o["ref"], o["rel"],
                                     o["wsv"])
 

@@ -50,8 +50,19 @@
  *     (16 for NVFP4, 32 for MX), otherwise MXQ_ERR_SHAPE.
  *   - Value codes: two 4-bit codes per byte, element 2j in the low nibble
  *     and element 2j+1 in the high nibble (NVFP4, MXFP4); one byte per
- *     element for MXFP8.  Scales: one byte per block, row-major
- *     [rows, cols / block] per group (the linear checkpoint layout).
+ *     element for MXFP8.  Scales: one byte per block, in one of two layouts
+ *     (mxq_layout): MXQ_LAYOUT_LINEAR, row-major [rows, cols / block] per
+ *     scale matrix (the checkpoint layout), or MXQ_LAYOUT_SWIZZLED_128X4,
+ *     the tiled layout block-scaled tensor-core GEMMs read: the matrix is
+ *     padded to a multiple of 128 rows and 4 columns and cut into tiles of
+ *     128 x 4 scales (512 bytes) stored row-tile-major; inside a tile the
+ *     scale of (row r, column c) sits at byte
+ *     (r % 32) * 16 + ((r / 32) % 4) * 4 + (c % 4).  Padding bytes are 0.
+ *     The pages only say that a loader may repack or interleave quantized
+ *     weights for the kernel (josch15366/Qwen3.8-Flash-Next-NVFP4-
+ *     LocalHessian-Experts, "Verifying the merge"); the tile layout is the
+ *     public block-scaling convention of the tensor-core GEMMs, not
+ *     something the pages define.
  */
 #ifndef MXQ_H
 #define MXQ_H
@@ -95,6 +106,11 @@ typedef enum mxq_scale_mode {
     MXQ_SCALE_FOUR_SIX = 1   /* 4/6-optimal block scales */
 } mxq_scale_mode;
 
+typedef enum mxq_layout {
+    MXQ_LAYOUT_LINEAR = 0,          /* row-major [rows, cols / block] */
+    MXQ_LAYOUT_SWIZZLED_128X4 = 1   /* 128 x 4 tiles, see the conventions */
+} mxq_layout;
+
 typedef enum mxq_op {
     MXQ_OP_QUANTIZE_NVFP4 = 0,
     MXQ_OP_QUANTIZE_ACT = 1,
@@ -106,6 +122,13 @@ MXQ_API int mxq_version(void);
 
 /* Human-readable name of a status code (static string, never NULL). */
 MXQ_API const char *mxq_status_string(mxq_status s);
+
+/* Bytes of the scale output of `n_matrices` scale matrices, each holding the
+ * block scales of a [rows, cols] tensor (block 16 for NVFP4, 32 for MX), in
+ * `layout`: n * rows * (cols / block) when linear, n * pad128(rows) *
+ * pad4(cols / block) when swizzled.  Returns 0 for invalid arguments. */
+MXQ_API size_t mxq_scale_bytes(mxq_fmt fmt, mxq_layout layout, int64_t n_matrices, int64_t rows,
+                               int64_t cols);
 
 /* Bytes of device workspace an entry point needs (0 if none).
  *   MXQ_OP_QUANTIZE_NVFP4: n = n_groups, rows, cols as passed to it;
@@ -123,8 +146,11 @@ MXQ_API size_t mxq_workspace_bytes(mxq_op op, int64_t n, int64_t rows, int64_t c
  *            gate and up share weight_scale_2; down slabs [H, I] form their
  *            own groups.  cols % 16 == 0.
  *   mode     MXQ_SCALE_RTN or MXQ_SCALE_FOUR_SIX.
+ *   layout   scale layout; each group is one scale matrix [rows, cols/16].
  *   codes    out, uint8 [n_groups, rows, cols/2] E2M1 nibbles.
- *   scales   out, uint8 [n_groups, rows, cols/16] E4M3 block scales.
+ *   scales   out, E4M3 block scales, mxq_scale_bytes(MXQ_FMT_NVFP4, layout,
+ *            n_groups, rows, cols) bytes: [n_groups, rows, cols/16] when
+ *            linear.
  *   s2       out, fp32 [n_groups]: s2 = RN32(amax_g / 2688).
  *   mbits    out, nullable, uint32 [ceil(n_groups*rows*cols/16 / 32)]:
  *            bit (b % 32) of word (b / 32) is 1 when block b (row-major
@@ -142,7 +168,7 @@ MXQ_API size_t mxq_workspace_bytes(mxq_op op, int64_t n, int64_t rows, int64_t c
  * the M=4 plan is kept only when its exact squared error
  * sum (x_i - q_i*D*s2)^2 is strictly lower than the M=6 plan's. */
 MXQ_API mxq_status mxq_quantize_nvfp4(const uint16_t *x, int64_t n_groups, int64_t rows,
-                              int64_t cols, mxq_scale_mode mode, uint8_t *codes,
+                              int64_t cols, mxq_scale_mode mode, mxq_layout layout, uint8_t *codes,
                               uint8_t *scales, float *s2, uint32_t *mbits,
                               uint32_t *m4_count, uint32_t *status, void *workspace,
                               size_t workspace_bytes, cudaStream_t stream);
@@ -154,29 +180,38 @@ MXQ_API mxq_status mxq_quantize_nvfp4(const uint16_t *x, int64_t n_groups, int64
  *           rows = product of the leading dimensions).
  *   fmt     MXQ_FMT_MXFP4 (E2M1, qmax 6) or MXQ_FMT_MXFP8 (E4M3, qmax 448).
  *   block   must be 32 (MXQ_ERR_UNSUPPORTED otherwise).
+ *   layout  scale layout; the whole [rows, cols/32] is one scale matrix
+ *           (stack tensors whose row count is a multiple of 128, or call
+ *           once per tensor, to get one tiled matrix per tensor).
  *   codes   out, uint8 [rows, cols/2] (MXFP4) or [rows, cols] (MXFP8).
- *   scales  out, uint8 [rows, cols/32], byte = e + 127 with e the smallest
+ *   scales  out, mxq_scale_bytes(fmt, layout, 1, rows, cols) bytes
+ *           ([rows, cols/32] when linear), byte = e + 127 with e the smallest
  *           integer such that amax <= qmax * 2^e (= ceil(log2(amax/qmax))),
  *           clamped to [-127, 127]; an all-zero block gives byte 0.
  *   status  nullable.
  * code_i = FMT(x_i * 2^-e), round to nearest even, sign kept. */
 MXQ_API mxq_status mxq_quantize_mx(const uint16_t *x, int64_t rows, int64_t cols, mxq_fmt fmt,
-                           int block, uint8_t *codes, uint8_t *scales, uint32_t *status,
-                           cudaStream_t stream);
+                           int block, mxq_layout layout, uint8_t *codes, uint8_t *scales,
+                           uint32_t *status, cudaStream_t stream);
 
 /* Dynamic activation quantization of a token tile [T, hidden].
  * Source: josch15366/Qwen3.8-Flash-Next-NVFP4-LocalHessian-Experts,
  * introduction (input_scale = amax/2688); MJPansa/Qwen3.8-Flash-Next-MXFP4-FP8-R12,
  * "Quantization format" (activations dynamically quantized to MXFP8).
  *   fmt = MXQ_FMT_NVFP4: the whole tile is one group, input_scale =
- *         RN32(amax / 2688) written to *input_scale (device fp32), block
- *         scales plain amax/6 (RTN); codes [T, hidden/2], scales
- *         [T, hidden/16]; workspace required.
+ *         RN32(amax / 2688) written to *input_scale (device fp32); block
+ *         scales by `mode`: MXQ_SCALE_RTN (plain amax/6, the pages'
+ *         activation recipe) or MXQ_SCALE_FOUR_SIX (the weights' 4/6-optimal
+ *         rule applied to the tile); codes [T, hidden/2], scales as
+ *         mxq_quantize_nvfp4 with one group; workspace required.
  *   fmt = MXQ_FMT_MXFP8 or MXQ_FMT_MXFP4: as mxq_quantize_mx with block 32;
+ *         mode must be MXQ_SCALE_RTN (MXQ_ERR_UNSUPPORTED otherwise);
  *         input_scale, workspace may be NULL.
+ *   layout scale layout, as for the quantizers above.
  *   status required. */
 MXQ_API mxq_status mxq_quantize_act(const uint16_t *tokens, int64_t T, int64_t hidden,
-                            mxq_fmt fmt, uint8_t *codes, uint8_t *scales,
+                            mxq_fmt fmt, mxq_scale_mode mode, mxq_layout layout,
+                            uint8_t *codes, uint8_t *scales,
                             float *input_scale, uint32_t *status, void *workspace,
                             size_t workspace_bytes, cudaStream_t stream);
 
@@ -191,6 +226,10 @@ MXQ_API mxq_status mxq_quantize_act(const uint16_t *tokens, int64_t T, int64_t h
  *   s2       NVFP4 only: fp32 [n_tensors / tensors_per_scale]; tensor t
  *            reads s2[t / tensors_per_scale] (2 for fused gate_up, so that
  *            gate_e and up_e read the shared weight_scale_2).  NULL for MX.
+ *   layout   layout of `scales`.  For the tiled layout, tensors_per_scale
+ *            consecutive tensors form one scale matrix (one NVFP4 group;
+ *            for MX pass n_tensors when the stack was quantized as one
+ *            matrix, 1 when each tensor was).
  *   sum_sq_err, sum_sq_ref   out, fp64 [n_tensors]: sum (x - deq)^2 and
  *            sum x^2 with deq = RN32((q * D) * s2) (NVFP4) or q * 2^e (MX).
  *   relerr   out, nullable, fp64 [n_tensors]: sqrt(err) / sqrt(ref)
@@ -200,7 +239,7 @@ MXQ_API mxq_status mxq_quantize_act(const uint16_t *tokens, int64_t T, int64_t h
  * so repeated calls give bit-identical results. */
 MXQ_API mxq_status mxq_dequant_relerr(const uint16_t *x, const uint8_t *codes,
                               const uint8_t *scales, const float *s2, mxq_fmt fmt,
-                              int64_t n_tensors, int64_t rows, int64_t cols,
+                              mxq_layout layout, int64_t n_tensors, int64_t rows, int64_t cols,
                               int64_t tensors_per_scale, double *sum_sq_err,
                               double *sum_sq_ref, double *relerr, void *workspace,
                               size_t workspace_bytes, cudaStream_t stream);
@@ -212,7 +251,7 @@ MXQ_API mxq_status mxq_dequant_relerr(const uint16_t *x, const uint8_t *codes,
  * can cause.  It takes no workspace: the per-chunk partial sums live in a
  * fixed 2 MiB array inside the library's device image, which every GPU that
  * loads the library holds until the process exits.  Arguments, outputs and
- * results are those of mxq_dequant_relerr.
+ * results are those of mxq_dequant_relerr with linear scales.
  *   Limit: n_tensors * ceil(rows * cols / 16384) <= 131072 chunks (for
  *   example 1024 tensors of 768 x 2048, or 512 of 2048 x 768); larger
  *   requests return MXQ_ERR_WORKSPACE before anything is enqueued.

@@ -30,6 +30,19 @@ static size_t verify_workspace_bytes(int64_t n_tensors, int64_t rows, int64_t co
 
 static bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
+static bool layout_ok(mxq_layout l) { return l == MXQ_LAYOUT_LINEAR || l == MXQ_LAYOUT_SWIZZLED_128X4; }
+
+// Tiled scales of `n` matrices of rows x cb scales: zero the whole buffer
+// first when a matrix has padding (rows % 128 or cb % 4), so that the
+// padding bytes are 0; the kernels write every real scale.
+static cudaError_t zero_tiled_padding(uint8_t *scales, int64_t n, int64_t rows, int64_t cb,
+                                      cudaStream_t stream)
+{
+    if (rows % 128 == 0 && cb % 4 == 0)
+        return cudaSuccess;
+    return cudaMemsetAsync(scales, 0, (size_t)n * swz128x4_bytes((uint64_t)rows, (uint64_t)cb), stream);
+}
+
 // rows * cols * n without overflow, all non-negative.
 static bool mul_ok(int64_t a, int64_t b, int64_t *out)
 {
@@ -47,7 +60,7 @@ using namespace mxq;
 
 extern "C" {
 
-int mxq_version(void) { return 10000; }
+int mxq_version(void) { return 10100; }
 
 const char *mxq_status_string(mxq_status s)
 {
@@ -61,6 +74,21 @@ const char *mxq_status_string(mxq_status s)
     case MXQ_ERR_UNSUPPORTED: return "unsupported request";
     }
     return "unknown status";
+}
+
+size_t mxq_scale_bytes(mxq_fmt fmt, mxq_layout layout, int64_t n_matrices, int64_t rows,
+                       int64_t cols)
+{
+    int64_t tmp;
+    if (n_matrices < 0 || rows < 0 || cols < 0 || !layout_ok(layout))
+        return 0;
+    const int64_t blk = fmt == MXQ_FMT_NVFP4 ? 16 : (fmt == MXQ_FMT_MXFP4 || fmt == MXQ_FMT_MXFP8 ? 32 : 0);
+    if (blk == 0 || cols % blk != 0 || !mul_ok(rows, cols, &tmp) || !mul_ok(tmp, n_matrices, &tmp))
+        return 0;
+    const int64_t cb = cols / blk;
+    if (layout == MXQ_LAYOUT_LINEAR)
+        return (size_t)(n_matrices * rows * cb);
+    return (size_t)n_matrices * (size_t)swz128x4_bytes((uint64_t)rows, (uint64_t)cb);
 }
 
 size_t mxq_workspace_bytes(mxq_op op, int64_t n, int64_t rows, int64_t cols)
@@ -86,7 +114,8 @@ size_t mxq_workspace_bytes(mxq_op op, int64_t n, int64_t rows, int64_t cols)
 }
 
 mxq_status mxq_quantize_nvfp4(const uint16_t *x, int64_t n_groups, int64_t rows, int64_t cols,
-                              mxq_scale_mode mode, uint8_t *codes, uint8_t *scales, float *s2,
+                              mxq_scale_mode mode, mxq_layout layout, uint8_t *codes,
+                              uint8_t *scales, float *s2,
                               uint32_t *mbits, uint32_t *m4_count, uint32_t *status,
                               void *workspace, size_t workspace_bytes, cudaStream_t stream)
 {
@@ -94,11 +123,16 @@ mxq_status mxq_quantize_nvfp4(const uint16_t *x, int64_t n_groups, int64_t rows,
         return MXQ_ERR_INVALID_ARG;
     if (mode != MXQ_SCALE_RTN && mode != MXQ_SCALE_FOUR_SIX)
         return MXQ_ERR_INVALID_ARG;
+    if (!layout_ok(layout))
+        return MXQ_ERR_INVALID_ARG;
     if (cols % 16 != 0)
         return MXQ_ERR_SHAPE;
     int64_t gsize, total;
     if (!mul_ok(rows, cols, &gsize) || !mul_ok(gsize, n_groups, &total) || total > (INT64_MAX / 4))
         return MXQ_ERR_SHAPE;
+    const bool swz = layout == MXQ_LAYOUT_SWIZZLED_128X4;
+    if (swz && gsize / 16 > 0x7FFFFFFF)
+        return MXQ_ERR_SHAPE;   // tiled offsets index the blocks of a group in 32 bits
     if (n_groups == 0)
         return MXQ_OK;
     if (!x || !codes || !scales || !s2 || !status)
@@ -113,18 +147,21 @@ mxq_status mxq_quantize_nvfp4(const uint16_t *x, int64_t n_groups, int64_t rows,
         return MXQ_ERR_ALIGN;
     const int64_t nb = gsize / 16;
     const int64_t total_blocks = total / 16;
+    const ScaleLayout sl = make_scale_layout(swz ? 1 : 0, rows, cols / 16);
     uint32_t *amax_bits = static_cast<uint32_t *>(workspace);
     unsigned long long *slots = reinterpret_cast<unsigned long long *>(
         static_cast<uint8_t *>(workspace) + nvfp4_slots_offset(n_groups));
     // amax bits / arrival counts and amax slots start at zero (a slot's tag
     // is its group + 1)
     cudaError_t e = cudaMemsetAsync(workspace, 0, need, stream);
+    if (e == cudaSuccess && swz)
+        e = zero_tiled_padding(scales, n_groups, rows, cols / 16, stream);
     if (e == cudaSuccess && m4_count)
         e = cudaMemsetAsync(m4_count, 0, (size_t)n_groups * sizeof(uint32_t), stream);
     if (e != cudaSuccess)
         return MXQ_ERR_CUDA;
     // single pass (one HBM read of x) when the shape allows it
-    e = launch_nvfp4_fused(x, n_groups, nb, mode == MXQ_SCALE_FOUR_SIX, slots, amax_bits, codes, scales, s2,
+    e = launch_nvfp4_fused(x, n_groups, nb, mode == MXQ_SCALE_FOUR_SIX, slots, amax_bits, codes, scales, sl, s2,
                            mbits, m4_count, status, stream);
     if (e == cudaSuccess)
         return MXQ_OK;
@@ -141,17 +178,20 @@ mxq_status mxq_quantize_nvfp4(const uint16_t *x, int64_t n_groups, int64_t rows,
         e = launch_group_amax(x, n_groups, nb, amax_bits, status, stream);
     if (e == cudaSuccess)
         e = launch_nvfp4_quant(x, n_groups, nb, mode == MXQ_SCALE_FOUR_SIX, amax_bits, codes, scales,
-                               s2, mbits, mbits_atomic, mode == MXQ_SCALE_FOUR_SIX ? m4_count : nullptr,
+                               sl, s2, mbits, mbits_atomic, mode == MXQ_SCALE_FOUR_SIX ? m4_count : nullptr,
                                stream);
     return e == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
 }
 
 mxq_status mxq_quantize_mx(const uint16_t *x, int64_t rows, int64_t cols, mxq_fmt fmt, int block,
-                           uint8_t *codes, uint8_t *scales, uint32_t *status, cudaStream_t stream)
+                           mxq_layout layout, uint8_t *codes, uint8_t *scales, uint32_t *status,
+                           cudaStream_t stream)
 {
     if (rows < 0 || cols < 0)
         return MXQ_ERR_INVALID_ARG;
     if (fmt != MXQ_FMT_MXFP4 && fmt != MXQ_FMT_MXFP8)
+        return MXQ_ERR_INVALID_ARG;
+    if (!layout_ok(layout))
         return MXQ_ERR_INVALID_ARG;
     if (block != 32)
         return MXQ_ERR_UNSUPPORTED;
@@ -166,15 +206,26 @@ mxq_status mxq_quantize_mx(const uint16_t *x, int64_t rows, int64_t cols, mxq_fm
         return MXQ_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(scales, 16) || (status && !aligned(status, 4)))
         return MXQ_ERR_ALIGN;
-    cudaError_t e = launch_mx_quant(x, total / 32, (int)fmt, codes, scales, status, stream);
+    const bool swz = layout == MXQ_LAYOUT_SWIZZLED_128X4;
+    if (swz && total / 32 > 0x7FFFFFFF)
+        return MXQ_ERR_SHAPE;   // tiled offsets index the blocks in 32 bits
+    const ScaleLayout sl = make_scale_layout(swz ? 1 : 0, rows, cols / 32);
+    cudaError_t e = swz ? zero_tiled_padding(scales, 1, rows, cols / 32, stream) : cudaSuccess;
+    if (e == cudaSuccess)
+        e = launch_mx_quant(x, total / 32, (int)fmt, codes, scales, sl, status, stream);
     return e == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
 }
 
 mxq_status mxq_quantize_act(const uint16_t *tokens, int64_t T, int64_t hidden, mxq_fmt fmt,
-                            uint8_t *codes, uint8_t *scales, float *input_scale, uint32_t *status,
+                            mxq_scale_mode mode, mxq_layout layout, uint8_t *codes,
+                            uint8_t *scales, float *input_scale, uint32_t *status,
                             void *workspace, size_t workspace_bytes, cudaStream_t stream)
 {
     if (T < 0 || hidden < 0)
+        return MXQ_ERR_INVALID_ARG;
+    if (mode != MXQ_SCALE_RTN && mode != MXQ_SCALE_FOUR_SIX)
+        return MXQ_ERR_INVALID_ARG;
+    if (!layout_ok(layout))
         return MXQ_ERR_INVALID_ARG;
     if (!status)
         return MXQ_ERR_INVALID_ARG;
@@ -187,16 +238,20 @@ mxq_status mxq_quantize_act(const uint16_t *tokens, int64_t T, int64_t hidden, m
             return cudaMemsetAsync(input_scale, 0, sizeof(float), stream) == cudaSuccess ? MXQ_OK
                                                                                           : MXQ_ERR_CUDA;
         }
-        return mxq_quantize_nvfp4(tokens, 1, T, hidden, MXQ_SCALE_RTN, codes, scales, input_scale,
+        return mxq_quantize_nvfp4(tokens, 1, T, hidden, mode, layout, codes, scales, input_scale,
                                   nullptr, nullptr, status, workspace, workspace_bytes, stream);
     }
-    if (fmt == MXQ_FMT_MXFP4 || fmt == MXQ_FMT_MXFP8)
-        return mxq_quantize_mx(tokens, T, hidden, fmt, 32, codes, scales, status, stream);
+    if (fmt == MXQ_FMT_MXFP4 || fmt == MXQ_FMT_MXFP8) {
+        if (mode != MXQ_SCALE_RTN)
+            return MXQ_ERR_UNSUPPORTED;
+        return mxq_quantize_mx(tokens, T, hidden, fmt, 32, layout, codes, scales, status, stream);
+    }
     return MXQ_ERR_INVALID_ARG;
 }
 
 mxq_status mxq_dequant_relerr(const uint16_t *x, const uint8_t *codes, const uint8_t *scales,
-                              const float *s2, mxq_fmt fmt, int64_t n_tensors, int64_t rows,
+                              const float *s2, mxq_fmt fmt, mxq_layout layout, int64_t n_tensors,
+                              int64_t rows,
                               int64_t cols, int64_t tensors_per_scale, double *sum_sq_err,
                               double *sum_sq_ref, double *relerr, void *workspace,
                               size_t workspace_bytes, cudaStream_t stream)
@@ -205,7 +260,10 @@ mxq_status mxq_dequant_relerr(const uint16_t *x, const uint8_t *codes, const uin
         return MXQ_ERR_INVALID_ARG;
     if (fmt != MXQ_FMT_NVFP4 && fmt != MXQ_FMT_MXFP4 && fmt != MXQ_FMT_MXFP8)
         return MXQ_ERR_INVALID_ARG;
-    if (fmt == MXQ_FMT_NVFP4 && tensors_per_scale < 1)
+    if (!layout_ok(layout))
+        return MXQ_ERR_INVALID_ARG;
+    const bool swz = layout == MXQ_LAYOUT_SWIZZLED_128X4;
+    if ((fmt == MXQ_FMT_NVFP4 || swz) && tensors_per_scale < 1)
         return MXQ_ERR_INVALID_ARG;
     const int blk = (fmt == MXQ_FMT_NVFP4) ? 16 : 32;
     if (cols % blk != 0)
@@ -213,6 +271,9 @@ mxq_status mxq_dequant_relerr(const uint16_t *x, const uint8_t *codes, const uin
     int64_t tsize, total;
     if (!mul_ok(rows, cols, &tsize) || !mul_ok(tsize, n_tensors, &total) || total > (INT64_MAX / 4))
         return MXQ_ERR_SHAPE;
+    int64_t msize = 0;
+    if (swz && (!mul_ok(tsize, tensors_per_scale, &msize) || msize / blk > 0x7FFFFFFF))
+        return MXQ_ERR_SHAPE;   // tiled offsets index the blocks of a matrix in 32 bits
     if (n_tensors == 0)
         return MXQ_OK;
     if (!sum_sq_err || !sum_sq_ref)
@@ -227,7 +288,9 @@ mxq_status mxq_dequant_relerr(const uint16_t *x, const uint8_t *codes, const uin
         return MXQ_ERR_WORKSPACE;
     if (!aligned(workspace, 256))
         return MXQ_ERR_ALIGN;
-    cudaError_t e = launch_verify(x, codes, scales, s2, (int)fmt, n_tensors, tsize, tensors_per_scale,
+    const ScaleLayout sl = make_scale_layout(swz ? 1 : 0, rows * (swz ? tensors_per_scale : 1), cols / blk);
+    cudaError_t e = launch_verify(x, codes, scales, s2, (int)fmt, sl, n_tensors, rows, tsize,
+                                  tensors_per_scale < 1 ? 1 : tensors_per_scale,
                                   static_cast<double *>(workspace), sum_sq_err, sum_sq_ref, relerr, stream);
     return e == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
 }

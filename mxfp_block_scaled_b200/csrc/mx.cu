@@ -34,7 +34,7 @@ __device__ __forceinline__ int mx_exponent(uint32_t amax_bits)
 template <int FMT>
 __global__ void __launch_bounds__(256)
 mx_quant_kernel(const uint4 *__restrict__ x, int64_t nblk, uint8_t *__restrict__ codes,
-                uint8_t *__restrict__ scales, uint32_t *__restrict__ status)
+                uint8_t *__restrict__ scales, const ScaleLayout sl, uint32_t *__restrict__ status)
 {
     for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk;
          b += (int64_t)gridDim.x * blockDim.x) {
@@ -58,7 +58,7 @@ mx_quant_kernel(const uint4 *__restrict__ x, int64_t nblk, uint8_t *__restrict__
 #pragma unroll
         for (int j = 0; j < 16; ++j)
             y[j] = __fmul2_rn(make_float2(bf16_lo(w[j]), bf16_hi(w[j])), sc2);
-        scales[b] = (uint8_t)(e + 127);
+        scales[sl.swz ? tiled_scale_offset(sl, 0, (uint32_t)b) : (uint64_t)b] = (uint8_t)(e + 127);
         if (FMT == MXQ_FMT_MXFP8) {
             uint32_t o[8];
 #pragma unroll
@@ -79,7 +79,7 @@ mx_quant_kernel(const uint4 *__restrict__ x, int64_t nblk, uint8_t *__restrict__
 }
 
 cudaError_t launch_mx_quant(const uint16_t *x, int64_t nblk32, int fmt, uint8_t *codes,
-                            uint8_t *scales, uint32_t *status, cudaStream_t s)
+                            uint8_t *scales, const ScaleLayout &sl, uint32_t *status, cudaStream_t s)
 {
     if (nblk32 == 0)
         return cudaSuccess;
@@ -88,9 +88,9 @@ cudaError_t launch_mx_quant(const uint16_t *x, int64_t nblk32, int fmt, uint8_t 
         ctas = 0x7FFFFFFF;
     const uint4 *xv = reinterpret_cast<const uint4 *>(x);
     if (fmt == MXQ_FMT_MXFP8)
-        mx_quant_kernel<MXQ_FMT_MXFP8><<<(unsigned)ctas, 256, 0, s>>>(xv, nblk32, codes, scales, status);
+        mx_quant_kernel<MXQ_FMT_MXFP8><<<(unsigned)ctas, 256, 0, s>>>(xv, nblk32, codes, scales, sl, status);
     else
-        mx_quant_kernel<MXQ_FMT_MXFP4><<<(unsigned)ctas, 256, 0, s>>>(xv, nblk32, codes, scales, status);
+        mx_quant_kernel<MXQ_FMT_MXFP4><<<(unsigned)ctas, 256, 0, s>>>(xv, nblk32, codes, scales, sl, status);
     return cudaGetLastError();
 }
 

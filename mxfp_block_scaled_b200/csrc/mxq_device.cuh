@@ -175,6 +175,58 @@ __device__ __forceinline__ float2 div2_bf16(float2 x, float2 d, float2 nr)
     return __ffma2_rn(e, nr, q0);                                       // q0 - e * r
 }
 
+// ---- division by a run-time invariant divisor ---------------------------
+// q = n / d for unsigned 32-bit n and 1 <= d < 2^31 with one high multiply
+// (Granlund and Montgomery, "Division by invariant integers using
+// multiplication", PLDI 1994, section 4): with l = ceil(log2 d) and
+// m = floor(2^32 (2^l - d) / d) + 1, q = (t + ((n - t) >> 1)) >> (l - 1)
+// where t = mulhi(m, n); d = 1 uses shift 0 and m = 0 (then q = n).
+struct FastDiv {
+    uint32_t d, m, s1, s2;
+};
+
+__host__ __device__ inline FastDiv make_fastdiv(uint32_t d)
+{
+    FastDiv f;
+    f.d = d;
+    uint32_t l = 0;
+    while (l < 32 && (1ull << l) < d)
+        ++l;
+    f.m = (uint32_t)((((1ull << l) - d) << 32) / d + 1);
+    f.s1 = l ? 1u : 0u;
+    f.s2 = l ? l - 1 : 0u;
+    if (d == 1)
+        f.m = 0;
+    return f;
+}
+
+__device__ __forceinline__ uint32_t fastdiv(uint32_t n, const FastDiv &f)
+{
+    const uint32_t t = __umulhi(f.m, n);
+    return (t + ((n - t) >> f.s1)) >> f.s2;
+}
+
+// ---- 128x4 tiled scale layout ---------------------------------------------
+// Byte offset of the scale of (row r, column c) of one scale matrix whose
+// column count rounds up to `ntc` groups of 4: the matrix is cut into tiles
+// of 128 rows x 4 columns (512 bytes each), stored row-tile-major
+// (tile (r / 128, c / 4) at ((r / 128) * ntc + c / 4) * 512); inside a tile
+// the byte of (r, c) sits at (r % 32) * 16 + ((r / 32) % 4) * 4 + c % 4.
+// This is the scale-factor layout that block-scaled tensor-core GEMMs read
+// (four 32-row slabs interleaved so that one 16-byte row holds the scales of
+// rows r, r + 32, r + 64, r + 96 for four consecutive blocks).
+__host__ __device__ __forceinline__ uint32_t swz128x4(uint32_t r, uint32_t c, uint32_t ntc)
+{
+    return (((r >> 7) * ntc + (c >> 2)) << 9) + ((r & 31u) << 4) + (((r >> 5) & 3u) << 2) + (c & 3u);
+}
+
+// Bytes of one scale matrix of `rows` x `cols` scales in the tiled layout
+// (rows padded to 128, columns to 4).
+__host__ __device__ __forceinline__ uint64_t swz128x4_bytes(uint64_t rows, uint64_t cols)
+{
+    return ((rows + 127) / 128) * 128 * (((cols + 3) / 4) * 4);
+}
+
 // Barrier `id` (1..15) among `count` threads (a multiple of 32).
 __device__ __forceinline__ void named_barrier_sync(int id, int count)
 {

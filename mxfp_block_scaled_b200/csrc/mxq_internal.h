@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "mxq_device.cuh"
+
 namespace mxq {
 
 constexpr float kGlobalDivisor = 2688.0f;  // 6 * 448: weight_scale_2 / input_scale
@@ -27,6 +29,36 @@ constexpr int64_t kVerifyChunk = 16384;  // elements per chunk (multiple of 32)
 
 size_t align_up(size_t v, size_t a);
 
+// Where block scales go (mxq_layout).  Linear: the scale of block b of a
+// matrix is byte b of it.  Tiled: byte swz128x4(b / cb, b % cb, ntc) of the
+// matrix, each matrix msz bytes.
+struct ScaleLayout {
+    int swz;          // 0 linear, 1 tiled 128 x 4
+    uint32_t cb;      // blocks per row (cols / block size)
+    uint32_t ntc;     // column tiles per matrix, ceil(cb / 4)
+    uint64_t msz;     // bytes of one tiled matrix
+    FastDiv cbdiv;    // division by cb
+};
+
+inline ScaleLayout make_scale_layout(int swz, int64_t rows_per_matrix, int64_t cb)
+{
+    ScaleLayout l;
+    l.swz = swz;
+    l.cb = (uint32_t)cb;
+    l.ntc = (uint32_t)((cb + 3) / 4);
+    l.msz = swz128x4_bytes((uint64_t)rows_per_matrix, (uint64_t)cb);
+    l.cbdiv = make_fastdiv(cb > 0 ? (uint32_t)cb : 1u);
+    return l;
+}
+
+// Byte offset of the scale of block bg (row-major block index inside its
+// matrix) of matrix m.
+__device__ __forceinline__ uint64_t tiled_scale_offset(const ScaleLayout &l, uint64_t m, uint32_t bg)
+{
+    const uint32_t r = fastdiv(bg, l.cbdiv), c = bg - r * l.cb;
+    return m * l.msz + swz128x4(r, c, l.ntc);
+}
+
 // Largest grid of the single-pass NVFP4 schedule (one CTA per SM).
 constexpr int kMaxFusedCtas = 256;
 
@@ -41,17 +73,19 @@ cudaError_t launch_group_amax(const uint16_t *x, int64_t n_groups, int64_t nb,
                               uint32_t *amax_bits, uint32_t *status, cudaStream_t s);
 cudaError_t launch_nvfp4_quant(const uint16_t *x, int64_t n_groups, int64_t nb, int four_six,
                                const uint32_t *amax_bits, uint8_t *codes, uint8_t *scales,
+                               const ScaleLayout &sl,
                                float *s2, uint32_t *mbits, int mbits_atomic,
                                uint32_t *m4_count, cudaStream_t s);
 cudaError_t launch_nvfp4_fused(const uint16_t *x, int64_t n_groups, int64_t nb, int four_six,
                                unsigned long long *slots, uint32_t *arrived, uint8_t *codes, uint8_t *scales,
+                               const ScaleLayout &sl,
                                float *s2, uint32_t *mbits, uint32_t *m4_count, uint32_t *status,
                                cudaStream_t s);
 cudaError_t launch_mx_quant(const uint16_t *x, int64_t nblk32, int fmt, uint8_t *codes,
-                            uint8_t *scales, uint32_t *status, cudaStream_t s);
+                            uint8_t *scales, const ScaleLayout &sl, uint32_t *status, cudaStream_t s);
 cudaError_t launch_verify(const uint16_t *x, const uint8_t *codes, const uint8_t *scales,
-                          const float *s2, int fmt, int64_t n_tensors, int64_t tsize,
-                          int64_t tensors_per_scale, double *partials, double *sum_sq_err,
+                          const float *s2, int fmt, const ScaleLayout &sl, int64_t n_tensors,
+                          int64_t rows, int64_t tsize, int64_t tensors_per_scale, double *partials, double *sum_sq_err,
                           double *sum_sq_ref, double *relerr, cudaStream_t s);
 
 } // namespace mxq

@@ -65,6 +65,7 @@ extern "C" mxq_status mxq_dequant_relerr_noalloc(const uint16_t *x, const uint8_
     const mxq_status st = scratch_for_current_device(&scratch);
     if (st != MXQ_OK)
         return st;
-    return mxq_dequant_relerr(x, codes, scales, s2, fmt, n_tensors, rows, cols, tensors_per_scale,
+    return mxq_dequant_relerr(x, codes, scales, s2, fmt, MXQ_LAYOUT_LINEAR, n_tensors, rows, cols,
+                              tensors_per_scale,
                               sum_sq_err, sum_sq_ref, relerr, scratch, kScratchBytes, stream);
 }

@@ -273,7 +273,7 @@ template <bool FOUR_SIX>
 __global__ void __launch_bounds__(kNvThreads)
 nvfp4_quant_kernel(const uint4 *__restrict__ x, int64_t n_groups, int64_t nb,
                    const uint32_t *__restrict__ amax_bits, uint2 *__restrict__ codes,
-                   uint8_t *__restrict__ scales, float *__restrict__ s2_out,
+                   uint8_t *__restrict__ scales, const ScaleLayout sl, float *__restrict__ s2_out,
                    uint32_t *__restrict__ mbits, int mbits_atomic, uint32_t *__restrict__ m4_count)
 {
     __shared__ GroupConst s_gc;
@@ -311,7 +311,8 @@ nvfp4_quant_kernel(const uint4 *__restrict__ x, int64_t n_groups, int64_t nb,
                     o = quantize_block<FOUR_SIX>(v[k][0], v[k][1], gc);
                     const int64_t gb = g * nb + b;
                     codes[gb] = o.codes;
-                    scales[gb] = (uint8_t)o.scale;
+                    scales[sl.swz ? tiled_scale_offset(sl, (uint64_t)g, (uint32_t)b) : (uint64_t)gb] =
+                        (uint8_t)o.scale;
                 }
                 if (mbits) {
                     const uint32_t word = __ballot_sync(0xFFFFFFFFu, o.m4);
@@ -376,6 +377,7 @@ struct FusedArgs {
     uint32_t *arrived;             // [n_groups] slots stored so far (starts at 0)
     uint2 *codes;
     uint8_t *scales;
+    ScaleLayout sl;
     float *s2_out;
     uint32_t *mbits, *m4_count;
 };
@@ -405,7 +407,7 @@ __device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity, volat
     return false;
 }
 
-template <bool FOUR_SIX>
+template <bool FOUR_SIX, bool SWZ>
 __global__ void __launch_bounds__(kFusedThreads, 1)
 nvfp4_fused_kernel(const FusedArgs a)
 {
@@ -672,7 +674,10 @@ nvfp4_fused_kernel(const FusedArgs a)
             const int k = k32 * 32 + lane;
             const BlockOut o = quantize_block<FOUR_SIX>(v[2 * k], v[2 * k + 1], gc);
             codes[k] = o.codes;
-            scales[k] = (uint8_t)o.scale;
+            if (SWZ)
+                a.scales[tiled_scale_offset(a.sl, (uint64_t)gj, (uint32_t)(my_lo + k))] = (uint8_t)o.scale;
+            else
+                scales[k] = (uint8_t)o.scale;
             const uint32_t word = __ballot_sync(0xFFFFFFFFu, o.m4);
             if (lane == 0) {
                 if (mbits)
@@ -725,8 +730,8 @@ static int sm_count()
 // two-pass path.
 cudaError_t launch_nvfp4_fused(const uint16_t *x, int64_t n_groups, int64_t nb, int four_six,
                                unsigned long long *slots, uint32_t *arrived, uint8_t *codes, uint8_t *scales,
-                               float *s2, uint32_t *mbits, uint32_t *m4_count, uint32_t *status,
-                               cudaStream_t s)
+                               const ScaleLayout &sl, float *s2, uint32_t *mbits, uint32_t *m4_count,
+                               uint32_t *status, cudaStream_t s)
 {
     if (n_groups <= 0 || n_groups > 0x7FFFFFFF || nb <= 0 || nb % 32 != 0)
         return cudaErrorNotSupported;
@@ -773,7 +778,10 @@ cudaError_t launch_nvfp4_fused(const uint16_t *x, int64_t n_groups, int64_t nb, 
         LQ = kMaxStages;
     const int D = LQ + 2 <= kReadyRing - 1 - LQ ? LQ + 2 : kReadyRing - 1 - LQ;
     const size_t dyn = 512 + (size_t)(LS + LQ) * (size_t)slice_bytes;
-    const void *fn = four_six ? (const void *)nvfp4_fused_kernel<true> : (const void *)nvfp4_fused_kernel<false>;
+    const void *fn = four_six ? (sl.swz ? (const void *)nvfp4_fused_kernel<true, true>
+                                        : (const void *)nvfp4_fused_kernel<true, false>)
+                              : (sl.swz ? (const void *)nvfp4_fused_kernel<false, true>
+                                        : (const void *)nvfp4_fused_kernel<false, false>);
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
     if (e != cudaSuccess)
         return e;
@@ -798,6 +806,7 @@ cudaError_t launch_nvfp4_fused(const uint16_t *x, int64_t n_groups, int64_t nb, 
     args.status = status;
     args.codes = reinterpret_cast<uint2 *>(codes);
     args.scales = scales;
+    args.sl = sl;
     args.s2_out = s2;
     args.mbits = mbits;
     args.m4_count = four_six ? m4_count : nullptr;
@@ -807,7 +816,7 @@ cudaError_t launch_nvfp4_fused(const uint16_t *x, int64_t n_groups, int64_t nb, 
 
 cudaError_t launch_nvfp4_quant(const uint16_t *x, int64_t n_groups, int64_t nb, int four_six,
                                const uint32_t *amax_bits, uint8_t *codes, uint8_t *scales,
-                               float *s2, uint32_t *mbits, int mbits_atomic,
+                               const ScaleLayout &sl, float *s2, uint32_t *mbits, int mbits_atomic,
                                uint32_t *m4_count, cudaStream_t s)
 {
     if (n_groups == 0)
@@ -819,10 +828,10 @@ cudaError_t launch_nvfp4_quant(const uint16_t *x, int64_t n_groups, int64_t nb, 
     uint2 *cv = reinterpret_cast<uint2 *>(codes);
     if (four_six)
         nvfp4_quant_kernel<true><<<grid, kNvThreads, 0, s>>>(xv, n_groups, nb, amax_bits, cv, scales,
-                                                             s2, mbits, mbits_atomic, m4_count);
+                                                             sl, s2, mbits, mbits_atomic, m4_count);
     else
         nvfp4_quant_kernel<false><<<grid, kNvThreads, 0, s>>>(xv, n_groups, nb, amax_bits, cv, scales,
-                                                              s2, mbits, mbits_atomic, m4_count);
+                                                              sl, s2, mbits, mbits_atomic, m4_count);
     return cudaGetLastError();
 }
 

@@ -104,12 +104,13 @@ __device__ __forceinline__ void cta_reduce_store(double err, double ref, double 
     __syncthreads();
 }
 
-template <int FMT>
+template <int FMT, bool SWZ>
 __global__ void __launch_bounds__(kVerifyThreads)
 verify_chunk_kernel(const uint16_t *__restrict__ x, const uint8_t *__restrict__ codes,
                     const uint8_t *__restrict__ scales, const float *__restrict__ s2,
-                    int64_t n_tensors, int64_t tsize, int64_t chunks_per_tensor,
-                    int64_t tensors_per_scale, double *__restrict__ partials)
+                    const ScaleLayout sl, int64_t n_tensors, int64_t rows, int64_t tsize,
+                    int64_t chunks_per_tensor, int64_t tensors_per_scale,
+                    double *__restrict__ partials)
 {
     constexpr int BLK = (FMT == MXQ_FMT_NVFP4) ? 16 : 32;
     // blocks per thread per chunk; all of a thread's loads are issued before
@@ -126,6 +127,9 @@ verify_chunk_kernel(const uint16_t *__restrict__ x, const uint8_t *__restrict__ 
         const int64_t nblk = (hi - lo) / BLK;
         const int64_t first = (t * tsize + lo) / BLK;   // global block index
         const float sv = (FMT == MXQ_FMT_NVFP4) ? __ldg(s2 + t / tensors_per_scale) : 0.0f;
+        // tiled scales: tensor t is rows [(t % tps) * rows, ...) of matrix t / tps
+        const uint64_t smat = SWZ ? (uint64_t)(t / tensors_per_scale) : 0;
+        const uint32_t sb0 = SWZ ? (uint32_t)((t % tensors_per_scale) * rows) * sl.cb + (uint32_t)(lo / BLK) : 0;
         uint4 xv[PER][XV];
         uint4 cv[PER][CV];
         uint2 c2[PER];
@@ -146,7 +150,7 @@ verify_chunk_kernel(const uint16_t *__restrict__ x, const uint8_t *__restrict__ 
                     for (int q = 0; q < CV; ++q)
                         cv[u][q] = __ldg(reinterpret_cast<const uint4 *>(codes) + gb * CV + q);
                 }
-                sb[u] = __ldg(scales + gb);
+                sb[u] = __ldg(scales + (SWZ ? tiled_scale_offset(sl, smat, sb0 + (uint32_t)i) : (uint64_t)gb));
             }
         }
         double err = 0.0, ref = 0.0;
@@ -194,24 +198,27 @@ __global__ void verify_finalize_kernel(const double *__restrict__ partials, int6
 }
 
 cudaError_t launch_verify(const uint16_t *x, const uint8_t *codes, const uint8_t *scales,
-                          const float *s2, int fmt, int64_t n_tensors, int64_t tsize,
-                          int64_t tensors_per_scale, double *partials, double *sum_sq_err,
-                          double *sum_sq_ref, double *relerr, cudaStream_t s)
+                          const float *s2, int fmt, const ScaleLayout &sl, int64_t n_tensors,
+                          int64_t rows, int64_t tsize, int64_t tensors_per_scale, double *partials,
+                          double *sum_sq_err, double *sum_sq_ref, double *relerr, cudaStream_t s)
 {
     if (n_tensors == 0)
         return cudaSuccess;
     const int64_t cpt = tsize > 0 ? (tsize + kVerifyChunk - 1) / kVerifyChunk : 1;
     int64_t n_chunks = n_tensors * cpt;
     const unsigned grid = (unsigned)(n_chunks < 0x7FFFFFFF ? n_chunks : 0x7FFFFFFF);
-    if (fmt == MXQ_FMT_NVFP4)
-        verify_chunk_kernel<MXQ_FMT_NVFP4><<<grid, kVerifyThreads, 0, s>>>(
-            x, codes, scales, s2, n_tensors, tsize, cpt, tensors_per_scale, partials);
-    else if (fmt == MXQ_FMT_MXFP8)
-        verify_chunk_kernel<MXQ_FMT_MXFP8><<<grid, kVerifyThreads, 0, s>>>(
-            x, codes, scales, s2, n_tensors, tsize, cpt, tensors_per_scale, partials);
-    else
-        verify_chunk_kernel<MXQ_FMT_MXFP4><<<grid, kVerifyThreads, 0, s>>>(
-            x, codes, scales, s2, n_tensors, tsize, cpt, tensors_per_scale, partials);
+#define MXQ_VERIFY(F, W)                                                                      \
+    verify_chunk_kernel<F, W><<<grid, kVerifyThreads, 0, s>>>(x, codes, scales, s2, sl, n_tensors, \
+                                                              rows, tsize, cpt, tensors_per_scale, \
+                                                              partials)
+    if (fmt == MXQ_FMT_NVFP4) {
+        if (sl.swz) MXQ_VERIFY(MXQ_FMT_NVFP4, true); else MXQ_VERIFY(MXQ_FMT_NVFP4, false);
+    } else if (fmt == MXQ_FMT_MXFP8) {
+        if (sl.swz) MXQ_VERIFY(MXQ_FMT_MXFP8, true); else MXQ_VERIFY(MXQ_FMT_MXFP8, false);
+    } else {
+        if (sl.swz) MXQ_VERIFY(MXQ_FMT_MXFP4, true); else MXQ_VERIFY(MXQ_FMT_MXFP4, false);
+    }
+#undef MXQ_VERIFY
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;

@@ -26,9 +26,11 @@ DEV_WAIT_TIMEOUT = 0x2
 
 FMT = {"nvfp4": 0, "mxfp4": 1, "mxfp8": 2}
 SCALE_MODE = {"rtn": 0, "four_six": 1}
+LAYOUT = {"linear": 0, "swizzled_128x4": 1}
 OP = {"quantize_nvfp4": 0, "quantize_act": 1, "dequant_relerr": 2}
 
-EXPORTED = ("mxq_version", "mxq_status_string", "mxq_workspace_bytes", "mxq_quantize_nvfp4",
+EXPORTED = ("mxq_version", "mxq_status_string", "mxq_scale_bytes", "mxq_workspace_bytes",
+            "mxq_quantize_nvfp4",
             "mxq_quantize_mx", "mxq_quantize_act", "mxq_dequant_relerr",
             "mxq_dequant_relerr_noalloc")
 
@@ -56,16 +58,19 @@ def load(path=LIB_PATH):
     L.mxq_version.argtypes = []
     L.mxq_status_string.restype = ctypes.c_char_p
     L.mxq_status_string.argtypes = [i32]
+    L.mxq_scale_bytes.restype = sz
+    L.mxq_scale_bytes.argtypes = [i32, i32, i64, i64, i64]
     L.mxq_workspace_bytes.restype = sz
     L.mxq_workspace_bytes.argtypes = [i32, i64, i64, i64]
     L.mxq_quantize_nvfp4.restype = i32
-    L.mxq_quantize_nvfp4.argtypes = [vp, i64, i64, i64, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.mxq_quantize_nvfp4.argtypes = [vp, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     L.mxq_quantize_mx.restype = i32
-    L.mxq_quantize_mx.argtypes = [vp, i64, i64, i32, i32, vp, vp, vp, vp]
+    L.mxq_quantize_mx.argtypes = [vp, i64, i64, i32, i32, i32, vp, vp, vp, vp]
     L.mxq_quantize_act.restype = i32
-    L.mxq_quantize_act.argtypes = [vp, i64, i64, i32, vp, vp, vp, vp, vp, sz, vp]
+    L.mxq_quantize_act.argtypes = [vp, i64, i64, i32, i32, i32, vp, vp, vp, vp, vp, sz, vp]
     L.mxq_dequant_relerr.restype = i32
-    L.mxq_dequant_relerr.argtypes = [vp, vp, vp, vp, i32, i64, i64, i64, i64, vp, vp, vp, vp, sz, vp]
+    L.mxq_dequant_relerr.argtypes = [vp, vp, vp, vp, i32, i32, i64, i64, i64, i64, vp, vp, vp, vp, sz,
+                                     vp]
     L.mxq_dequant_relerr_noalloc.restype = i32
     L.mxq_dequant_relerr_noalloc.argtypes = [vp, vp, vp, vp, i32, i64, i64, i64, i64, vp, vp, vp, vp]
     if path == LIB_PATH:
@@ -91,6 +96,10 @@ def _check(fn, rc):
         raise MxqError(fn, rc)
 
 
+def scale_bytes(fmt, layout, n_matrices, rows, cols):
+    return load().mxq_scale_bytes(FMT[fmt], LAYOUT[layout], n_matrices, rows, cols)
+
+
 def workspace_bytes(op, n, rows, cols):
     return load().mxq_workspace_bytes(OP[op], n, rows, cols)
 
@@ -101,33 +110,35 @@ def _workspace(op, n, rows, cols, device):
 
 
 # ---------------------------------------------------------------- C names --
-def mxq_quantize_nvfp4(x, n_groups, rows, cols, mode, codes, scales, s2, mbits, m4_count,
+def mxq_quantize_nvfp4(x, n_groups, rows, cols, mode, layout, codes, scales, s2, mbits, m4_count,
                        status, workspace, stream=None):
-    rc = load().mxq_quantize_nvfp4(_p(x), n_groups, rows, cols, SCALE_MODE[mode], _p(codes),
+    rc = load().mxq_quantize_nvfp4(_p(x), n_groups, rows, cols, SCALE_MODE[mode], LAYOUT[layout],
+                                   _p(codes),
                                    _p(scales), _p(s2), _p(mbits), _p(m4_count), _p(status),
                                    _p(workspace), workspace.numel() if workspace is not None else 0,
                                    _stream(stream))
     _check("mxq_quantize_nvfp4", rc)
 
 
-def mxq_quantize_mx(x, rows, cols, fmt, block, codes, scales, status, stream=None):
-    rc = load().mxq_quantize_mx(_p(x), rows, cols, FMT[fmt], block, _p(codes), _p(scales),
-                                _p(status), _stream(stream))
+def mxq_quantize_mx(x, rows, cols, fmt, block, layout, codes, scales, status, stream=None):
+    rc = load().mxq_quantize_mx(_p(x), rows, cols, FMT[fmt], block, LAYOUT[layout], _p(codes),
+                                _p(scales), _p(status), _stream(stream))
     _check("mxq_quantize_mx", rc)
 
 
-def mxq_quantize_act(tokens, T, hidden, fmt, codes, scales, input_scale, status, workspace,
-                     stream=None):
-    rc = load().mxq_quantize_act(_p(tokens), T, hidden, FMT[fmt], _p(codes), _p(scales),
+def mxq_quantize_act(tokens, T, hidden, fmt, mode, layout, codes, scales, input_scale, status,
+                     workspace, stream=None):
+    rc = load().mxq_quantize_act(_p(tokens), T, hidden, FMT[fmt], SCALE_MODE[mode], LAYOUT[layout],
+                                 _p(codes), _p(scales),
                                  _p(input_scale), _p(status), _p(workspace),
                                  workspace.numel() if workspace is not None else 0, _stream(stream))
     _check("mxq_quantize_act", rc)
 
 
-def mxq_dequant_relerr(x, codes, scales, s2, fmt, n_tensors, rows, cols, tensors_per_scale,
-                       sum_sq_err, sum_sq_ref, relerr, workspace, stream=None):
-    rc = load().mxq_dequant_relerr(_p(x), _p(codes), _p(scales), _p(s2), FMT[fmt], n_tensors, rows,
-                                   cols, tensors_per_scale, _p(sum_sq_err), _p(sum_sq_ref),
+def mxq_dequant_relerr(x, codes, scales, s2, fmt, layout, n_tensors, rows, cols,
+                       tensors_per_scale, sum_sq_err, sum_sq_ref, relerr, workspace, stream=None):
+    rc = load().mxq_dequant_relerr(_p(x), _p(codes), _p(scales), _p(s2), FMT[fmt], LAYOUT[layout],
+                                   n_tensors, rows, cols, tensors_per_scale, _p(sum_sq_err), _p(sum_sq_ref),
                                    _p(relerr), _p(workspace),
                                    workspace.numel() if workspace is not None else 0,
                                    _stream(stream))
@@ -154,16 +165,18 @@ def _bf16(x):
     return x
 
 
-def quantize_nvfp4(x, mode="four_six", with_mbits=True, stream=None):
+def quantize_nvfp4(x, mode="four_six", with_mbits=True, stream=None, layout="linear"):
     """x: bf16 [G, R, C] on the device.  Returns a dict of device tensors:
-    codes [G,R,C/2] u8, scales [G,R,C/16] u8, s2 [G] f32, mbits u32 words,
-    m4_count [G] i32-view of u32, status [1]."""
+    codes [G,R,C/2] u8, scales ([G,R,C/16] u8 when linear, the flat tiled
+    bytes of G matrices when layout="swizzled_128x4"), s2 [G] f32, mbits u32
+    words, m4_count [G] i32-view of u32, status [1]."""
     _bf16(x)
     G, R, C = x.shape
     dev = x.device
     out = {
         "codes": torch.empty((G, R, C // 2), dtype=torch.uint8, device=dev),
-        "scales": torch.empty((G, R, C // 16), dtype=torch.uint8, device=dev),
+        "scales": torch.empty((G, R, C // 16), dtype=torch.uint8, device=dev) if layout == "linear"
+        else torch.empty(max(scale_bytes("nvfp4", layout, G, R, C), 1), dtype=torch.uint8, device=dev),
         "s2": torch.empty(G, dtype=torch.float32, device=dev),
         "mbits": torch.empty(((G * R * C // 16) + 31) // 32 or 1, dtype=torch.int32, device=dev)
         if with_mbits else None,
@@ -171,13 +184,15 @@ def quantize_nvfp4(x, mode="four_six", with_mbits=True, stream=None):
         "status": torch.zeros(1, dtype=torch.int32, device=dev),
     }
     ws, _ = _workspace("quantize_nvfp4", G, R, C, dev)
-    mxq_quantize_nvfp4(x, G, R, C, mode, out["codes"], out["scales"], out["s2"], out["mbits"],
-                       out["m4_count"], out["status"], ws, stream)
+    mxq_quantize_nvfp4(x, G, R, C, mode, layout, out["codes"], out["scales"], out["s2"],
+                       out["mbits"], out["m4_count"], out["status"], ws, stream)
     return out
 
 
-def quantize_mx(x, fmt, stream=None):
-    """x: bf16 [..., C].  Returns dict codes, scales, status."""
+def quantize_mx(x, fmt, stream=None, layout="linear"):
+    """x: bf16 [..., C], quantized as one [rows, C] matrix.  Returns dict
+    codes, scales (tiled bytes of that one matrix when layout is
+    "swizzled_128x4"), status."""
     _bf16(x)
     C = x.shape[-1]
     R = x.numel() // C if C else 0
@@ -185,39 +200,43 @@ def quantize_mx(x, fmt, stream=None):
     out = {
         "codes": torch.empty(x.shape[:-1] + ((C // 2) if fmt == "mxfp4" else C,), dtype=torch.uint8,
                              device=dev),
-        "scales": torch.empty(x.shape[:-1] + (C // 32,), dtype=torch.uint8, device=dev),
+        "scales": torch.empty(x.shape[:-1] + (C // 32,), dtype=torch.uint8, device=dev)
+        if layout == "linear"
+        else torch.empty(max(scale_bytes(fmt, layout, 1, R, C), 1), dtype=torch.uint8, device=dev),
         "status": torch.zeros(1, dtype=torch.int32, device=dev),
     }
-    mxq_quantize_mx(x, R, C, fmt, 32, out["codes"], out["scales"], out["status"], stream)
+    mxq_quantize_mx(x, R, C, fmt, 32, layout, out["codes"], out["scales"], out["status"], stream)
     return out
 
 
-def quantize_act(tokens, fmt, stream=None):
-    """tokens: bf16 [T, hidden].  NVFP4 returns input_scale too."""
+def quantize_act(tokens, fmt, stream=None, mode="rtn", layout="linear"):
+    """tokens: bf16 [T, hidden].  NVFP4 returns input_scale too; mode
+    "four_six" applies the 4/6-optimal block scales to the tile."""
     _bf16(tokens)
     T, H = tokens.shape
     dev = tokens.device
     blk = 16 if fmt == "nvfp4" else 32
     out = {
         "codes": torch.empty((T, H if fmt == "mxfp8" else H // 2), dtype=torch.uint8, device=dev),
-        "scales": torch.empty((T, H // blk), dtype=torch.uint8, device=dev),
+        "scales": torch.empty((T, H // blk), dtype=torch.uint8, device=dev) if layout == "linear"
+        else torch.empty(max(scale_bytes(fmt, layout, 1, T, H), 1), dtype=torch.uint8, device=dev),
         "input_scale": torch.empty(1, dtype=torch.float32, device=dev),
         "status": torch.zeros(1, dtype=torch.int32, device=dev),
     }
     ws, _ = _workspace("quantize_act", T, H, 0, dev)
-    mxq_quantize_act(tokens, T, H, fmt, out["codes"], out["scales"], out["input_scale"],
-                     out["status"], ws, stream)
+    mxq_quantize_act(tokens, T, H, fmt, mode, layout, out["codes"], out["scales"],
+                     out["input_scale"], out["status"], ws, stream)
     return out
 
 
 def dequant_relerr(x, codes, scales, s2, fmt, n_tensors, rows, cols, tensors_per_scale=1,
-                   stream=None):
+                   stream=None, layout="linear"):
     """Per-tensor fp64 (sum_sq_err, sum_sq_ref, relerr) on the device."""
     dev = x.device
     err = torch.empty(max(n_tensors, 1), dtype=torch.float64, device=dev)
     ref = torch.empty_like(err)
     rel = torch.empty_like(err)
     ws, _ = _workspace("dequant_relerr", n_tensors, rows, cols, dev)
-    mxq_dequant_relerr(x, codes, scales, s2, fmt, n_tensors, rows, cols, tensors_per_scale, err,
-                       ref, rel, ws, stream)
+    mxq_dequant_relerr(x, codes, scales, s2, fmt, layout, n_tensors, rows, cols, tensors_per_scale,
+                       err, ref, rel, ws, stream)
     return err[:n_tensors], ref[:n_tensors], rel[:n_tensors]

@@ -1,8 +1,8 @@
 """CPU oracle of the block-scaled microscaling quantizer.
 
-TEST INFRASTRUCTURE ONLY.  The C oracle (``mxq_oracle.c``) and the exact
-rational micro-oracle (``micro.py``) are the checkers the CUDA library is
-compared against.  Only the test suite, ``__graft_entry__.smoke()`` and the
+TEST INFRASTRUCTURE ONLY.  The C oracle (``mxq_oracle.c``), the exact
+rational micro-oracle (``micro.py``) and the scale-layout permutation
+(``layout.py``) are the checkers the CUDA library is compared against.  Only the test suite, ``__graft_entry__.smoke()`` and the
 benchmark's CPU-baseline leg may import this package; the product library
 neither imports nor links it, and the two share no code.
 """

@@ -62,44 +62,68 @@ def test_host_argument_errors_return_before_any_launch(lib):
     vp = ctypes.c_void_p
     fake = vp(0x1000)           # never dereferenced: every call below fails its checks first
     # NVFP4: cols not a multiple of 16
-    assert lib.mxq_quantize_nvfp4(fake, 1, 4, 24, 1, fake, fake, fake, None, None, fake, fake,
+    assert lib.mxq_quantize_nvfp4(fake, 1, 4, 24, 1, 0, fake, fake, fake, None, None, fake, fake,
                                   4096, None) == 2
     # negative sizes, bad mode
-    assert lib.mxq_quantize_nvfp4(fake, -1, 4, 16, 1, fake, fake, fake, None, None, fake, fake,
+    assert lib.mxq_quantize_nvfp4(fake, -1, 4, 16, 1, 0, fake, fake, fake, None, None, fake, fake,
                                   4096, None) == 1
-    assert lib.mxq_quantize_nvfp4(fake, 1, 4, 16, 7, fake, fake, fake, None, None, fake, fake,
+    assert lib.mxq_quantize_nvfp4(fake, 1, 4, 16, 7, 0, fake, fake, fake, None, None, fake, fake,
                                   4096, None) == 1
     # null output / status
-    assert lib.mxq_quantize_nvfp4(fake, 1, 4, 16, 1, None, fake, fake, None, None, fake, fake,
+    assert lib.mxq_quantize_nvfp4(fake, 1, 4, 16, 1, 0, None, fake, fake, None, None, fake, fake,
                                   4096, None) == 1
-    assert lib.mxq_quantize_nvfp4(fake, 1, 4, 16, 1, fake, fake, fake, None, None, None, fake,
+    assert lib.mxq_quantize_nvfp4(fake, 1, 4, 16, 1, 0, fake, fake, fake, None, None, None, fake,
                                   4096, None) == 1
     # misaligned input
-    assert lib.mxq_quantize_nvfp4(vp(0x1002), 1, 4, 16, 1, fake, fake, fake, None, None, fake,
+    assert lib.mxq_quantize_nvfp4(vp(0x1002), 1, 4, 16, 1, 0, fake, fake, fake, None, None, fake,
                                   fake, 4096, None) == 3
     # workspace too small
-    assert lib.mxq_quantize_nvfp4(fake, 1, 4, 16, 1, fake, fake, fake, None, None, fake, fake,
+    assert lib.mxq_quantize_nvfp4(fake, 1, 4, 16, 1, 0, fake, fake, fake, None, None, fake, fake,
                                   8, None) == 4
     # MX: block size other than 32, bad format, bad shape
-    assert lib.mxq_quantize_mx(fake, 4, 64, 2, 16, fake, fake, None, None) == 6
-    assert lib.mxq_quantize_mx(fake, 4, 64, 0, 32, fake, fake, None, None) == 1
-    assert lib.mxq_quantize_mx(fake, 4, 48, 2, 32, fake, fake, None, None) == 2
+    assert lib.mxq_quantize_mx(fake, 4, 64, 2, 16, 0, fake, fake, None, None) == 6
+    assert lib.mxq_quantize_mx(fake, 4, 64, 0, 32, 0, fake, fake, None, None) == 1
+    assert lib.mxq_quantize_mx(fake, 4, 48, 2, 32, 0, fake, fake, None, None) == 2
     # verifier: missing s2 for NVFP4, tensors_per_scale < 1
-    assert lib.mxq_dequant_relerr(fake, fake, fake, None, 0, 2, 4, 16, 1, fake, fake, None, fake,
+    assert lib.mxq_dequant_relerr(fake, fake, fake, None, 0, 0, 2, 4, 16, 1, fake, fake, None, fake,
                                   4096, None) == 1
-    assert lib.mxq_dequant_relerr(fake, fake, fake, fake, 0, 2, 4, 16, 0, fake, fake, None, fake,
+    assert lib.mxq_dequant_relerr(fake, fake, fake, fake, 0, 0, 2, 4, 16, 0, fake, fake, None, fake,
+                                  4096, None) == 1
+    # unknown layout / mode values
+    assert lib.mxq_quantize_nvfp4(fake, 1, 4, 16, 1, 5, fake, fake, fake, None, None, fake, fake,
+                                  4096, None) == 1
+    assert lib.mxq_quantize_mx(fake, 4, 64, 2, 32, 9, fake, fake, None, None) == 1
+    assert lib.mxq_dequant_relerr(fake, fake, fake, None, 2, 3, 2, 4, 64, 1, fake, fake, None, fake,
+                                  4096, None) == 1
+    assert lib.mxq_quantize_act(fake, 4, 64, 0, 2, 0, fake, fake, fake, fake, fake, 4096, None) == 1
+    # MX activations have no 4/6 mode
+    assert lib.mxq_quantize_act(fake, 4, 64, 2, 1, 0, fake, fake, None, fake, None, 0, None) == 6
+    # tiled layout: a scale matrix needs at least one tensor
+    assert lib.mxq_dequant_relerr(fake, fake, fake, None, 2, 1, 2, 4, 64, 0, fake, fake, None, fake,
                                   4096, None) == 1
     # activation: status required; NVFP4 needs input_scale
-    assert lib.mxq_quantize_act(fake, 4, 64, 0, fake, fake, fake, None, fake, 4096, None) == 1
-    assert lib.mxq_quantize_act(fake, 4, 64, 0, fake, fake, None, fake, fake, 4096, None) == 1
+    assert lib.mxq_quantize_act(fake, 4, 64, 0, 0, 0, fake, fake, fake, None, fake, 4096, None) == 1
+    assert lib.mxq_quantize_act(fake, 4, 64, 0, 0, 0, fake, fake, None, fake, fake, 4096, None) == 1
+
+
+def test_scale_bytes(lib):
+    # linear: one byte per block; tiled: rows padded to 128, blocks per row to 4
+    assert lib.mxq_scale_bytes(0, 0, 512, 1536, 2048) == 512 * 1536 * 128
+    assert lib.mxq_scale_bytes(0, 1, 512, 1536, 2048) == 512 * 1536 * 128
+    assert lib.mxq_scale_bytes(0, 1, 2, 130, 80) == 2 * 256 * 8        # 5 blocks -> 8
+    assert lib.mxq_scale_bytes(2, 1, 1, 1, 32) == 128 * 4
+    assert lib.mxq_scale_bytes(1, 0, 3, 7, 64) == 3 * 7 * 2
+    assert lib.mxq_scale_bytes(0, 0, 1, 4, 24) == 0                      # cols % 16
+    assert lib.mxq_scale_bytes(0, 2, 1, 4, 16) == 0                      # unknown layout
+    assert lib.mxq_scale_bytes(7, 0, 1, 4, 32) == 0                      # unknown format
 
 
 def test_empty_inputs_are_no_ops(lib):
     # zero groups / zero rows: nothing to do, success without touching memory
-    assert lib.mxq_quantize_nvfp4(None, 0, 4, 16, 1, None, None, None, None, None, None, None, 0,
+    assert lib.mxq_quantize_nvfp4(None, 0, 4, 16, 1, 0, None, None, None, None, None, None, None, 0,
                                   None) == 0
-    assert lib.mxq_quantize_mx(None, 0, 64, 2, 32, None, None, None, None) == 0
-    assert lib.mxq_dequant_relerr(None, None, None, None, 2, 0, 4, 64, 1, None, None, None, None, 0,
+    assert lib.mxq_quantize_mx(None, 0, 64, 2, 32, 0, None, None, None, None) == 0
+    assert lib.mxq_dequant_relerr(None, None, None, None, 2, 0, 0, 4, 64, 1, None, None, None, None, 0,
                                   None) == 0
 
 

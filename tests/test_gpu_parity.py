@@ -149,7 +149,7 @@ def test_deterministic_and_canaries():
     ws, _ = mxq._workspace("quantize_nvfp4", G, R, C, "cuda")
     results = []
     for _ in range(2):
-        mxq.mxq_quantize_nvfp4(gu, G, R, C, "four_six", codes[pad:pad + n // 2],
+        mxq.mxq_quantize_nvfp4(gu, G, R, C, "four_six", "linear", codes[pad:pad + n // 2],
                                scales[pad:pad + n // 16], s2[:G], mb[:(n // 16) // 32], m4[:G], st, ws)
         torch.cuda.synchronize()
         results.append((codes.clone(), scales.clone(), s2.clone(), mb.clone()))
