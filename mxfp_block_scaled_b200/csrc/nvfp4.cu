@@ -653,8 +653,15 @@ nvfp4_fused_kernel(const FusedArgs a)
     // -------------------------------------------------------- compute warps
     if (bytes == 0)
         return;
+    // Chunks of 32 blocks are dealt round-robin over the compute warps along
+    // the whole sequence of this CTA's groups (chunk n32 * j + k of group j
+    // goes to warp (n32 * j + k) % kFusedComputeWarps), so the work stays
+    // balanced when a slice's chunk count is not a multiple of the warp
+    // count; a warp with no chunk in a group still frees the group's buffer.
     const int cw = warp - 2 - kFusedScoutWarps;
     const int n32 = (int)(my_n / 32);
+    const int step = n32 % kFusedComputeWarps;          // chunk offset gained per group
+    int first = cw;                                     // this warp's first chunk in group j
     int st = 0, rs = 0;                                 // quantize stage and ready slot of group j
     uint32_t qpar = 0, rpar = 0;                        // their phase parities
     for (int j = 0; j < G; ++j) {
@@ -670,7 +677,7 @@ nvfp4_fused_kernel(const FusedArgs a)
         uint8_t *scales = a.scales + gb0;
         uint32_t *mbits = a.mbits ? a.mbits + (gb0 >> 5) : nullptr;
         uint32_t cnt = 0;
-        for (int k32 = cw; k32 < n32; k32 += kFusedComputeWarps) {
+        for (int k32 = first; k32 < n32; k32 += kFusedComputeWarps) {
             const int k = k32 * 32 + lane;
             const BlockOut o = quantize_block<FOUR_SIX>(v[2 * k], v[2 * k + 1], gc);
             codes[k] = o.codes;
@@ -699,6 +706,9 @@ nvfp4_fused_kernel(const FusedArgs a)
             rs = 0;
             rpar ^= 1u;
         }
+        first -= step;                                  // (cw - n32 * (j + 1)) mod warps
+        if (first < 0)
+            first += kFusedComputeWarps;
     }
 }
 

@@ -176,3 +176,32 @@ def test_tiled_mxfp8_scales_drive_a_block_scaled_gemm():
                              la["scales"].reshape(-1).view(torch.float8_e8m0fnu),
                              lb["scales"].reshape(-1).view(torch.float8_e8m0fnu), out_dtype=torch.bfloat16)
     assert (bad.double() - ref).abs().max().item() > 10 * max(err, 1e-3)
+
+
+def test_tiled_nvfp4_scales_drive_a_block_scaled_gemm():
+    """NVFP4 operands (E2M1 pairs, E4M3 scale per 16 in the tiled layout) in a
+    block-scaled FP4 GEMM; the global scales are applied outside it."""
+    if not hasattr(torch, "float4_e2m1fn_x2"):
+        pytest.skip("this torch has no packed FP4 dtype")
+    M, N, K = 256, 256, 512
+    a = _rand_bf16((1, M, K), seed=21, std=1.0)
+    b = _rand_bf16((1, N, K), seed=22, std=1.0)
+    qa, qb = mxq.quantize_nvfp4(a, layout=SWZ), mxq.quantize_nvfp4(b, layout=SWZ)
+    la, lb = mxq.quantize_nvfp4(a), mxq.quantize_nvfp4(b)
+    torch.cuda.synchronize()
+    e2m1 = torch.tensor([0, .5, 1, 1.5, 2, 3, 4, 6, -0., -.5, -1, -1.5, -2, -3, -4, -6],
+                        dtype=torch.float64, device="cuda")
+
+    def qd(q, rows):     # q * D (the global scale left out), [rows, K]
+        c = q["codes"].reshape(rows, K // 2).long()
+        v = torch.stack([e2m1[c & 15], e2m1[c >> 4]], dim=-1).reshape(rows, K)
+        d = q["scales"].reshape(rows, K // 16).view(torch.float8_e4m3fn).double()
+        return v * d.repeat_interleave(16, dim=1)
+
+    ref = qd(la, M) @ qd(lb, N).t()
+    fp4 = torch.float4_e2m1fn_x2
+    out = _scaled_mm_or_skip(qa["codes"].reshape(M, K // 2).view(fp4), qb["codes"].reshape(N, K // 2).view(fp4).t(),
+                             qa["scales"].view(torch.float8_e4m3fn), qb["scales"].view(torch.float8_e4m3fn),
+                             out_dtype=torch.bfloat16)
+    err = (out.double() - ref).abs().max().item()
+    assert err <= 0.02 * ref.abs().max().item(), err
