@@ -10,6 +10,7 @@ unstacked tensor (1024 gate/up tensors [768, 2048] and 512 down tensors
 larger than L2, so no flush is needed between steps.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mine|reference]
+    python bench.py --workload fp8_requant     # FP8 -> MXFP4 requantization of the same layer
 
 Prints one JSON line on rank 0.  Under torchrun every rank converts its own
 layer (independent units, no data-path collective: weak scaling); the step
@@ -329,6 +330,81 @@ def run_reference(args, rank, world):
 
 
 # ------------------------------------------------------------------ main --
+REQ_BYTES = 1.0 + 0.5 + 1.0 / 32    # read E4M3, write E2M1 codes + UE8M0 scales (block scales ~0)
+
+
+def run_requant(args, device):
+    """FP8 -> MXFP4 requantization of one full-size routed-expert layer held
+    as block-FP8 (E4M3 codes + one fp32 scale per 128 x 128 block):
+    gate_up [512 * 1536, 2048] and down [512 * 2048, 768]."""
+    from mxfp_block_scaled_b200 import mxq, workloads
+    E = args.experts
+    srcs = []
+    for name, rows, cols in (("gate_up", E * 2 * INTER, HIDDEN), ("down", E * HIDDEN, INTER)):
+        codes = torch.empty((rows, cols), dtype=torch.uint8, device=device)
+        bs = torch.empty((rows // 128, -(-cols // 128)), dtype=torch.float32, device=device)
+        step = 128 * 256
+        for i, r0 in enumerate(range(0, rows, step)):
+            c, b = workloads.block_fp8_source(min(step, rows - r0), cols, seed=1000 + i, device=device)
+            codes[r0:r0 + c.shape[0]] = c
+            bs[r0 // 128:r0 // 128 + b.shape[0]] = b
+        out = {"codes": torch.empty((rows, cols // 2), dtype=torch.uint8, device=device),
+               "scales": torch.empty((rows, cols // 32), dtype=torch.uint8, device=device),
+               "status": torch.zeros(1, dtype=torch.int32, device=device)}
+        srcs.append((name, rows, cols, codes, bs, out))
+    torch.cuda.synchronize()
+
+    def step(ev=None):
+        for i, (name, rows, cols, codes, bs, out) in enumerate(srcs):
+            if ev is not None:
+                ev[i][0].record()
+            mxq.mxq_requant_fp8_mx(codes, bs, rows, cols, 128, 128, "mxfp4", "linear", out["codes"],
+                                   out["scales"], out["status"])
+            if ev is not None:
+                ev[i][1].record()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    for s_ in srcs:
+        if int(s_[5]["status"].item()) != 0:
+            raise RuntimeError("device status on " + s_[0])
+    events = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+               for _ in srcs] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device_uuid()) as clk:
+        torch.cuda.synchronize()
+        t0.record()
+        for k in range(args.steps):
+            step(events[k])
+        t1.record()
+        torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / args.steps
+    call_ms = [statistics.mean(events[k][i][0].elapsed_time(events[k][i][1]) for k in range(args.steps))
+               for i in range(len(srcs))]
+    n = sum(r * c for _, r, c, _, _, _ in srcs)
+    peak, peak_kind = measured_peak()
+    value = n * REQ_BYTES / (ms * 1e-3) / 1e9
+    gu_n = srcs[0][1] * srcs[0][2]
+    achieved = gu_n * REQ_BYTES / (call_ms[0] * 1e-3) / 1e9
+    return {
+        "metric": "FP8 -> MXFP4 requantization HBM GB/s (1 GPU)", "value": value, "unit": "GB/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": "one full-size routed-expert layer as block FP8 (E4M3 + fp32 scale per "
+                               "128x128) -> MXFP4: gate_up [512*1536, 2048] + down [512*2048, 768]",
+                   "elements_per_gpu": n, "algorithmic_bytes_per_element": REQ_BYTES,
+                   "l2": "inputs 2.4 GB, larger than L2; no flush",
+                   "call_ms": dict(zip(["requant_gate_up", "requant_down"], call_ms))},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "kernel": "requant_fp8_mx_kernel<MXFP4> (gate_up)", "peak_kind": peak_kind},
+        "gpu_launches": args.steps * len(srcs),
+        "clocks": clk.summary(),
+    }
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -339,6 +415,9 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the e2e and CPU-baseline legs (profiling runs)")
+    ap.add_argument("--workload", default="nvfp4_layer", choices=["nvfp4_layer", "fp8_requant"],
+                    help="nvfp4_layer: the headline quantize + verify step; fp8_requant: block-FP8 "
+                         "-> MXFP4 requantization of the same layer")
     ap.add_argument("--experts", type=int, default=EXPERTS,
                     help="experts in the layer; fewer than 512 only for small profiling captures")
     args = ap.parse_args()
@@ -361,6 +440,11 @@ def main():
     from mxfp_block_scaled_b200 import build, mxq
     build.build()
     mxq.load()
+    if args.workload == "fp8_requant":
+        if world > 1:
+            raise SystemExit("--workload fp8_requant runs on one GPU")
+        print(json.dumps(run_requant(args, device)), flush=True)
+        return 0
 
     layer = Layer(seed=rank, device=device, experts=args.experts)
     torch.cuda.synchronize()

@@ -194,6 +194,31 @@ MXQ_API mxq_status mxq_quantize_mx(const uint16_t *x, int64_t rows, int64_t cols
                            int block, mxq_layout layout, uint8_t *codes, uint8_t *scales,
                            uint32_t *status, cudaStream_t stream);
 
+/* FP8 -> MX requantization of a block-FP8 source tensor.
+ * Source: MJPansa/Qwen3.8-Flash-Next-MXFP4-FP8-R12, "Quantization and layer
+ * selection" (the conversion started from the released FP8 weights, without
+ * a BF16 copy) and "Quantization format" (converted routed experts are MXFP4
+ * E2M1 with UE8M0 scales; retained layers keep the source block-FP8 format).
+ * The pages do not give the source block shape or the arithmetic of the
+ * conversion; the readings are stated here.
+ *   fp8     E4M3 codes [rows, cols], one byte per value, 16-byte aligned.
+ *   bscale  fp32 [ceil(rows / brows), ceil(cols / bcols)]: value (r, c) of
+ *           the source is E4M3(code) * bscale[r / brows][c / bcols].
+ *   brows, bcols  source block shape (128 x 128 in the usual block-FP8
+ *           checkpoints); bcols must be a multiple of 32 (MXQ_ERR_SHAPE).
+ *   fmt, layout, codes, scales, status  as mxq_quantize_mx (block 32; the
+ *           whole [rows, cols/32] is one scale matrix); rows * cols / 32 must
+ *           stay below 2^32 (MXQ_ERR_SHAPE).
+ * Each value is dequantized once to fp32, w = RN32(E4M3(code) * scale), and
+ * every run of 32 w is MX-quantized as mxq_quantize_mx does with bf16 input:
+ * e = smallest integer with amax <= qmax * 2^e (clamped to [-127, 127]),
+ * code = FMT(w * 2^-e).  A NaN source code (S.1111.111) or a non-finite
+ * scale sets MXQ_DEV_NONFINITE_INPUT. */
+MXQ_API mxq_status mxq_requant_fp8_mx(const uint8_t *fp8, const float *bscale, int64_t rows,
+                                      int64_t cols, int64_t brows, int64_t bcols, mxq_fmt fmt,
+                                      mxq_layout layout, uint8_t *codes, uint8_t *scales,
+                                      uint32_t *status, cudaStream_t stream);
+
 /* Dynamic activation quantization of a token tile [T, hidden].
  * Source: josch15366/Qwen3.8-Flash-Next-NVFP4-LocalHessian-Experts,
  * introduction (input_scale = amax/2688); MJPansa/Qwen3.8-Flash-Next-MXFP4-FP8-R12,

@@ -216,6 +216,37 @@ mxq_status mxq_quantize_mx(const uint16_t *x, int64_t rows, int64_t cols, mxq_fm
     return e == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
 }
 
+mxq_status mxq_requant_fp8_mx(const uint8_t *fp8, const float *bscale, int64_t rows, int64_t cols,
+                              int64_t brows, int64_t bcols, mxq_fmt fmt, mxq_layout layout,
+                              uint8_t *codes, uint8_t *scales, uint32_t *status, cudaStream_t stream)
+{
+    if (rows < 0 || cols < 0 || brows < 1 || bcols < 1)
+        return MXQ_ERR_INVALID_ARG;
+    if (fmt != MXQ_FMT_MXFP4 && fmt != MXQ_FMT_MXFP8)
+        return MXQ_ERR_INVALID_ARG;
+    if (!layout_ok(layout))
+        return MXQ_ERR_INVALID_ARG;
+    if (cols % 32 != 0 || bcols % 32 != 0 || brows > 0x7FFFFFFF || bcols > 0x7FFFFFFF)
+        return MXQ_ERR_SHAPE;
+    int64_t total;
+    if (!mul_ok(rows, cols, &total) || total / 32 > 0xFFFFFFFFll)
+        return MXQ_ERR_SHAPE;
+    if (total == 0)
+        return MXQ_OK;
+    if (!fp8 || !bscale || !codes || !scales)
+        return MXQ_ERR_INVALID_ARG;
+    if (!aligned(fp8, 16) || !aligned(bscale, 4) || !aligned(codes, 16) || !aligned(scales, 16) ||
+        (status && !aligned(status, 4)))
+        return MXQ_ERR_ALIGN;
+    const bool swz = layout == MXQ_LAYOUT_SWIZZLED_128X4;
+    const ScaleLayout sl = make_scale_layout(swz ? 1 : 0, rows, cols / 32);
+    cudaError_t e = swz ? zero_tiled_padding(scales, 1, rows, cols / 32, stream) : cudaSuccess;
+    if (e == cudaSuccess)
+        e = launch_requant_fp8_mx(fp8, bscale, rows, cols, brows, bcols, (int)fmt, codes, scales, sl,
+                                  status, stream);
+    return e == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
+}
+
 mxq_status mxq_quantize_act(const uint16_t *tokens, int64_t T, int64_t hidden, mxq_fmt fmt,
                             mxq_scale_mode mode, mxq_layout layout, uint8_t *codes,
                             uint8_t *scales, float *input_scale, uint32_t *status,

@@ -78,6 +78,119 @@ mx_quant_kernel(const uint4 *__restrict__ x, int64_t nblk, uint8_t *__restrict__
     }
 }
 
+// ---------------------------------------------------------------------------
+// FP8 -> MX requantization of a block-FP8 source
+// (MJPansa/Qwen3.8-Flash-Next-MXFP4-FP8-R12, "Quantization and layer
+// selection": the conversion starts from the released FP8 weights;
+// "Quantization format": retained layers stay in the source block-FP8
+// format).  Each value is dequantized once to fp32, w = RN32(E4M3 * scale)
+// with the fp32 scale of its brows x bcols source block, and each run of 32
+// w is MX-quantized as above, the exponent read off the fp32 amax bits:
+// amax = m * 2^E, qmax = c * 2^k  =>  e = E - k + (m > c), clamped.
+// ---------------------------------------------------------------------------
+template <int FMT>
+__device__ __forceinline__ int mx_exponent_f32(uint32_t amax_bits)
+{
+    constexpr int k = (FMT == MXQ_FMT_MXFP8) ? 8 : 2;
+    constexpr uint32_t c_mant = (FMT == MXQ_FMT_MXFP8) ? 0x600000u : 0x400000u;  // .75 / .5
+    const uint32_t E = amax_bits >> 23;
+    if (E == 0)
+        return -127;
+    int e = (int)E - 127 - k + ((amax_bits & 0x7FFFFFu) > c_mant ? 1 : 0);
+    return e < -127 ? -127 : (e > 127 ? 127 : e);
+}
+
+struct RequantArgs {
+    const uint4 *fp8;        // 32 E4M3 bytes per MX block (2 x uint4)
+    const float *bscale;     // [ceil(rows / brows), nbc]
+    int64_t nblk;            // MX blocks (rows * cols / 32), < 2^32
+    uint32_t cb, nbc;        // MX blocks per row; source blocks per row
+    FastDiv cbdiv, browsdiv, bcdiv;   // / cb, / brows, / (bcols / 32)
+    uint8_t *codes, *scales;
+    ScaleLayout sl;
+    uint32_t *status;
+};
+
+template <int FMT>
+__global__ void __launch_bounds__(256) requant_fp8_mx_kernel(const RequantArgs a)
+{
+    for (int64_t bb = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; bb < a.nblk;
+         bb += (int64_t)gridDim.x * blockDim.x) {
+        const uint32_t b = (uint32_t)bb;
+        const uint4 v0 = __ldg(a.fp8 + 2 * bb), v1 = __ldg(a.fp8 + 2 * bb + 1);
+        const uint32_t r = fastdiv(b, a.cbdiv), j = b - r * a.cb;
+        const float sc = __ldg(a.bscale + (uint64_t)fastdiv(r, a.browsdiv) * a.nbc + fastdiv(j, a.bcdiv));
+        const float2 sc2 = make_float2(sc, sc);
+        const uint32_t w8[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        float2 w[16];
+        uint32_t m = 0;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            // 4 E4M3 bytes -> two f16x2 pairs (exact) -> fp32, times the scale (one rounding)
+            w[2 * t] = __fmul2_rn(f16x2_to_float2(e4m3x2_to_f16x2(w8[t])), sc2);
+            w[2 * t + 1] = __fmul2_rn(f16x2_to_float2(e4m3x2_to_f16x2(w8[t] >> 16)), sc2);
+            m = max(m, max(__float_as_uint(w[2 * t].x) & 0x7FFFFFFFu, __float_as_uint(w[2 * t].y) & 0x7FFFFFFFu));
+            m = max(m, max(__float_as_uint(w[2 * t + 1].x) & 0x7FFFFFFFu,
+                           __float_as_uint(w[2 * t + 1].y) & 0x7FFFFFFFu));
+        }
+        if (m >= 0x7F800000u && a.status)
+            atomicOr(a.status, MXQ_DEV_NONFINITE_INPUT);
+        const int e = mx_exponent_f32<FMT>(m);
+        const float s = e == 127 ? 0x1p-127f : __uint_as_float((uint32_t)(127 - e) << 23);   // 2^-e
+        const float2 s2 = make_float2(s, s);
+#pragma unroll
+        for (int t = 0; t < 16; ++t)
+            w[t] = __fmul2_rn(w[t], s2);                // exact (a power of two)
+        a.scales[a.sl.swz ? tiled_scale_offset(a.sl, 0, b) : (uint64_t)b] = (uint8_t)(e + 127);
+        if (FMT == MXQ_FMT_MXFP8) {
+            uint32_t o[8];
+#pragma unroll
+            for (int t = 0; t < 8; ++t)
+                o[t] = e4m3x2(w[2 * t].x, w[2 * t].y) | (e4m3x2(w[2 * t + 1].x, w[2 * t + 1].y) << 16);
+            uint4 *dst = reinterpret_cast<uint4 *>(a.codes) + 2 * bb;
+            dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+            dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+        } else {
+            uint4 o;
+            o.x = e2m1x8(w[0], w[1], w[2], w[3]);
+            o.y = e2m1x8(w[4], w[5], w[6], w[7]);
+            o.z = e2m1x8(w[8], w[9], w[10], w[11]);
+            o.w = e2m1x8(w[12], w[13], w[14], w[15]);
+            reinterpret_cast<uint4 *>(a.codes)[bb] = o;
+        }
+    }
+}
+
+cudaError_t launch_requant_fp8_mx(const uint8_t *fp8, const float *bscale, int64_t rows, int64_t cols,
+                                  int64_t brows, int64_t bcols, int fmt, uint8_t *codes,
+                                  uint8_t *scales, const ScaleLayout &sl, uint32_t *status,
+                                  cudaStream_t s)
+{
+    RequantArgs a;
+    a.fp8 = reinterpret_cast<const uint4 *>(fp8);
+    a.bscale = bscale;
+    a.nblk = rows * cols / 32;
+    a.cb = (uint32_t)(cols / 32);
+    a.nbc = (uint32_t)((cols + bcols - 1) / bcols);
+    a.cbdiv = make_fastdiv(a.cb);
+    a.browsdiv = make_fastdiv((uint32_t)brows);
+    a.bcdiv = make_fastdiv((uint32_t)(bcols / 32));
+    a.codes = codes;
+    a.scales = scales;
+    a.sl = sl;
+    a.status = status;
+    if (a.nblk == 0)
+        return cudaSuccess;
+    int64_t ctas = (a.nblk + 255) / 256;
+    if (ctas > 148 * 64)
+        ctas = 148 * 64;
+    if (fmt == MXQ_FMT_MXFP8)
+        requant_fp8_mx_kernel<MXQ_FMT_MXFP8><<<(unsigned)ctas, 256, 0, s>>>(a);
+    else
+        requant_fp8_mx_kernel<MXQ_FMT_MXFP4><<<(unsigned)ctas, 256, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_mx_quant(const uint16_t *x, int64_t nblk32, int fmt, uint8_t *codes,
                             uint8_t *scales, const ScaleLayout &sl, uint32_t *status, cudaStream_t s)
 {

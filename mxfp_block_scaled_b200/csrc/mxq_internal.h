@@ -83,6 +83,10 @@ cudaError_t launch_nvfp4_fused(const uint16_t *x, int64_t n_groups, int64_t nb, 
                                cudaStream_t s);
 cudaError_t launch_mx_quant(const uint16_t *x, int64_t nblk32, int fmt, uint8_t *codes,
                             uint8_t *scales, const ScaleLayout &sl, uint32_t *status, cudaStream_t s);
+cudaError_t launch_requant_fp8_mx(const uint8_t *fp8, const float *bscale, int64_t rows, int64_t cols,
+                                  int64_t brows, int64_t bcols, int fmt, uint8_t *codes,
+                                  uint8_t *scales, const ScaleLayout &sl, uint32_t *status,
+                                  cudaStream_t s);
 cudaError_t launch_verify(const uint16_t *x, const uint8_t *codes, const uint8_t *scales,
                           const float *s2, int fmt, const ScaleLayout &sl, int64_t n_tensors,
                           int64_t rows, int64_t tsize, int64_t tensors_per_scale, double *partials, double *sum_sq_err,

@@ -31,7 +31,7 @@ OP = {"quantize_nvfp4": 0, "quantize_act": 1, "dequant_relerr": 2}
 
 EXPORTED = ("mxq_version", "mxq_status_string", "mxq_scale_bytes", "mxq_workspace_bytes",
             "mxq_quantize_nvfp4",
-            "mxq_quantize_mx", "mxq_quantize_act", "mxq_dequant_relerr",
+            "mxq_quantize_mx", "mxq_requant_fp8_mx", "mxq_quantize_act", "mxq_dequant_relerr",
             "mxq_dequant_relerr_noalloc")
 
 
@@ -66,6 +66,8 @@ def load(path=LIB_PATH):
     L.mxq_quantize_nvfp4.argtypes = [vp, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     L.mxq_quantize_mx.restype = i32
     L.mxq_quantize_mx.argtypes = [vp, i64, i64, i32, i32, i32, vp, vp, vp, vp]
+    L.mxq_requant_fp8_mx.restype = i32
+    L.mxq_requant_fp8_mx.argtypes = [vp, vp, i64, i64, i64, i64, i32, i32, vp, vp, vp, vp]
     L.mxq_quantize_act.restype = i32
     L.mxq_quantize_act.argtypes = [vp, i64, i64, i32, i32, i32, vp, vp, vp, vp, vp, sz, vp]
     L.mxq_dequant_relerr.restype = i32
@@ -124,6 +126,13 @@ def mxq_quantize_mx(x, rows, cols, fmt, block, layout, codes, scales, status, st
     rc = load().mxq_quantize_mx(_p(x), rows, cols, FMT[fmt], block, LAYOUT[layout], _p(codes),
                                 _p(scales), _p(status), _stream(stream))
     _check("mxq_quantize_mx", rc)
+
+
+def mxq_requant_fp8_mx(fp8, bscale, rows, cols, brows, bcols, fmt, layout, codes, scales, status,
+                       stream=None):
+    rc = load().mxq_requant_fp8_mx(_p(fp8), _p(bscale), rows, cols, brows, bcols, FMT[fmt],
+                                   LAYOUT[layout], _p(codes), _p(scales), _p(status), _stream(stream))
+    _check("mxq_requant_fp8_mx", rc)
 
 
 def mxq_quantize_act(tokens, T, hidden, fmt, mode, layout, codes, scales, input_scale, status,
@@ -206,6 +215,26 @@ def quantize_mx(x, fmt, stream=None, layout="linear"):
         "status": torch.zeros(1, dtype=torch.int32, device=dev),
     }
     mxq_quantize_mx(x, R, C, fmt, 32, layout, out["codes"], out["scales"], out["status"], stream)
+    return out
+
+
+def requant_fp8_mx(fp8, bscale, brows, bcols, fmt, stream=None, layout="linear"):
+    """fp8: uint8 E4M3 codes [R, C] on the device; bscale: fp32
+    [ceil(R/brows), ceil(C/bcols)].  Returns dict codes, scales, status."""
+    if fp8.dtype != torch.uint8 or not fp8.is_contiguous() or fp8.dim() != 2:
+        raise ValueError("expected a contiguous uint8 [rows, cols] tensor of E4M3 codes")
+    if bscale.dtype != torch.float32 or not bscale.is_contiguous():
+        raise ValueError("expected contiguous fp32 block scales")
+    R, C = fp8.shape
+    dev = fp8.device
+    out = {
+        "codes": torch.empty((R, (C // 2) if fmt == "mxfp4" else C), dtype=torch.uint8, device=dev),
+        "scales": torch.empty((R, C // 32), dtype=torch.uint8, device=dev) if layout == "linear"
+        else torch.empty(max(scale_bytes(fmt, layout, 1, R, C), 1), dtype=torch.uint8, device=dev),
+        "status": torch.zeros(1, dtype=torch.int32, device=dev),
+    }
+    mxq_requant_fp8_mx(fp8, bscale, R, C, brows, bcols, fmt, layout, out["codes"], out["scales"],
+                       out["status"], stream)
     return out
 
 

@@ -129,6 +129,31 @@ def activation_tile(T, seed=0, device="cpu", hidden=2048):
     return a.to(torch.bfloat16)
 
 
+def block_fp8_source(rows, cols, seed=0, device="cpu", brows=128, bcols=128):
+    """A block-FP8 source tensor as stored by FP8 checkpoints: E4M3 codes
+    [rows, cols] (uint8) and one fp32 scale per brows x bcols block
+    (MJPansa/Qwen3.8-Flash-Next-MXFP4-FP8-R12, "Quantization format": the
+    retained layers keep the source block-FP8 format; the block shape is a
+    reading, 128 x 128).  Codes are drawn directly, not encoded from values:
+    random sign, exponent field 1..15 drawn with weight 2^field (large
+    magnitudes most frequent, as in a tensor scaled to use the FP8 range),
+    uniform mantissa, the NaN pattern S.1111.111 replaced by S.1111.110, and
+    1 % of codes zero.  Scales are log-uniform in [2^-16, 2^-6]."""
+    g = _gen(seed, device)
+    w = torch.pow(2.0, torch.arange(1, 16, dtype=torch.float32, device=device))
+    expo = torch.multinomial(w / w.sum(), rows * cols, replacement=True, generator=g) + 1
+    mant = torch.randint(0, 8, (rows * cols,), generator=g, device=device)
+    sign = torch.randint(0, 2, (rows * cols,), generator=g, device=device)
+    mag = expo * 8 + mant
+    mag = torch.where(mag == 0x7F, torch.full_like(mag, 0x7E), mag)
+    zero = torch.rand(rows * cols, generator=g, device=device) < 0.01
+    mag = torch.where(zero, torch.zeros_like(mag), mag)
+    codes = (sign * 128 + mag).to(torch.uint8).reshape(rows, cols)
+    nbr, nbc = -(-rows // brows), -(-cols // bcols)
+    scales = torch.pow(2.0, torch.empty((nbr, nbc), device=device).uniform_(-16.0, -6.0, generator=g))
+    return codes, scales.to(torch.float32)
+
+
 def bf16_bits(t):
     """bf16 tensor -> numpy uint16 array of its bit patterns (host copy)."""
     return t.detach().contiguous().view(torch.int16).cpu().numpy().view("uint16")

@@ -17,6 +17,7 @@ from .capi import (  # noqa: F401
     mx_exponent,
     quantize_nvfp4,
     quantize_mx,
+    requant_fp8_mx,
     dequant_relerr,
     relerr_from_sums,
 )

@@ -58,6 +58,8 @@ def lib():
         L.oracle_quantize_nvfp4.argtypes = [vp, i64, i64, i64, i, d, vp, vp, vp, vp]
         L.oracle_quantize_mx.restype = i
         L.oracle_quantize_mx.argtypes = [vp, i64, i64, i, vp, vp]
+        L.oracle_requant_fp8_mx.restype = i
+        L.oracle_requant_fp8_mx.argtypes = [vp, vp, i64, i64, i64, i64, i, vp, vp]
         L.oracle_dequant_relerr.restype = i
         L.oracle_dequant_relerr.argtypes = [vp, vp, vp, vp, i, i64, i64, i64, i64, vp, vp]
         _lib = L
@@ -127,6 +129,22 @@ def quantize_mx(x_bits, fmt):
     rc = lib().oracle_quantize_mx(_ptr(x), R, C, f, _ptr(codes), _ptr(scales))
     if rc != 0:
         raise RuntimeError("oracle_quantize_mx failed: %d" % rc)
+    return codes, scales
+
+
+def requant_fp8_mx(fp8, bscale, brows, bcols, fmt):
+    """fp8: uint8 E4M3 codes [R, C]; bscale: float32 [ceil(R/brows), ceil(C/bcols)].
+    Returns MX codes and scales of the fp32-dequantized source."""
+    q = np.ascontiguousarray(fp8, np.uint8)
+    R, C = q.shape
+    sc = np.ascontiguousarray(bscale, np.float32)
+    f = {"mxfp4": 1, "mxfp8": 2}[fmt]
+    codes = np.zeros((R, (C // 2) if f == 1 else C), np.uint8)
+    scales = np.zeros((R, C // 32), np.uint8)
+    rc = lib().oracle_requant_fp8_mx(_ptr(q), _ptr(sc), R, C, brows, bcols, f, _ptr(codes),
+                                     _ptr(scales))
+    if rc != 0:
+        raise RuntimeError("oracle_requant_fp8_mx failed: %d" % rc)
     return codes, scales
 
 

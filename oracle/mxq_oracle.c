@@ -346,6 +346,64 @@ int oracle_quantize_mx(const uint16_t *x, int64_t rows, int64_t cols, int fmt,
  *   MXFP4 / MXFP8: deq = q * 2^(b - 127).
  * sum_sq_err[t] = sum (x - deq)^2, sum_sq_ref[t] = sum x^2, both as
  * binary64 sums in element order.  Returns 0 or -1. */
+/* FP8 -> MX requantization [P4 "Quantization and layer selection": the
+ * conversion started from the released FP8 weights, without a BF16 copy;
+ * "Quantization format": the retained layers stay in the source block-FP8
+ * format, the converted ones are MXFP4 E2M1 with UE8M0 scales].
+ * Readings (the pages give neither): the source stores one E4M3 byte per
+ * value and one fp32 scale per brows x bcols block, value = E4M3 * scale;
+ * the conversion dequantizes each value to fp32 with one rounding,
+ * w = RN32(E4M3(code) * scale), then quantizes the fp32 w exactly as the
+ * bf16 MX path does (same exponent rule on the block amax, same encoding of
+ * w * 2^-e).  fp8 [rows, cols]; bscale [ceil(rows/brows), ceil(cols/bcols)].
+ * Returns -3 for a NaN source code or a non-finite scale. */
+int oracle_requant_fp8_mx(const uint8_t *fp8, const float *bscale, int64_t rows,
+                          int64_t cols, int64_t brows, int64_t bcols, int fmt,
+                          uint8_t *codes, uint8_t *scales)
+{
+    if (rows < 0 || cols < 0 || cols % 32 != 0 || brows < 1 || bcols < 1 ||
+        (fmt != 1 && fmt != 2))
+        return -1;
+    const double qmax = (fmt == 1) ? 6.0 : 448.0;
+    const int64_t nbc = (cols + bcols - 1) / bcols;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t j = 0; j < cols / 32; ++j) {
+            float w[32];
+            double amax = 0.0;
+            for (int i = 0; i < 32; ++i) {
+                const int64_t c = j * 32 + i;
+                const uint8_t q = fp8[r * cols + c];
+                const float sc = bscale[(r / brows) * nbc + c / bcols];
+                if ((q & 0x7F) == 0x7F || !isfinite(sc))
+                    return -3;
+                /* E4M3 value (4 significant bits) times the fp32 scale is
+                   exact in binary64; the cast rounds it once to binary32 */
+                w[i] = (float)(oracle_e4m3_value(q) * (double)sc);
+                if (!isfinite(w[i]))
+                    return -3;
+                if (fabs((double)w[i]) > amax)
+                    amax = fabs((double)w[i]);
+            }
+            const int e = oracle_mx_exponent(amax, qmax);
+            const int64_t b = r * (cols / 32) + j;
+            scales[b] = (uint8_t)(e + 127);
+            for (int i = 0; i < 32; ++i) {
+                const double y = ldexp((double)w[i], -e);      /* exact */
+                if (fmt == 1) {
+                    const unsigned cc = oracle_e2m1_encode(y) & 0xFu;
+                    if (i & 1)
+                        codes[b * 16 + i / 2] |= (uint8_t)(cc << 4);
+                    else
+                        codes[b * 16 + i / 2] = (uint8_t)cc;
+                } else {
+                    codes[b * 32 + i] = (uint8_t)oracle_e4m3_encode(y);
+                }
+            }
+        }
+    }
+    return 0;
+}
+
 int oracle_dequant_relerr(const uint16_t *x, const uint8_t *codes,
                           const uint8_t *scales, const float *s2, int fmt,
                           int64_t n_tensors, int64_t rows, int64_t cols,

@@ -101,6 +101,13 @@ def test_host_argument_errors_return_before_any_launch(lib):
     # tiled layout: a scale matrix needs at least one tensor
     assert lib.mxq_dequant_relerr(fake, fake, fake, None, 2, 1, 2, 4, 64, 0, fake, fake, None, fake,
                                   4096, None) == 1
+    # FP8 -> MX requantization: source block width not a multiple of 32, bad block, bad format
+    assert lib.mxq_requant_fp8_mx(fake, fake, 4, 64, 128, 48, 1, 0, fake, fake, None, None) == 2
+    assert lib.mxq_requant_fp8_mx(fake, fake, 4, 64, 0, 128, 1, 0, fake, fake, None, None) == 1
+    assert lib.mxq_requant_fp8_mx(fake, fake, 4, 64, 128, 128, 0, 0, fake, fake, None, None) == 1
+    assert lib.mxq_requant_fp8_mx(fake, fake, 4, 48, 128, 128, 1, 0, fake, fake, None, None) == 2
+    assert lib.mxq_requant_fp8_mx(None, fake, 4, 64, 128, 128, 1, 0, fake, fake, None, None) == 1
+    assert lib.mxq_requant_fp8_mx(None, None, 0, 64, 128, 128, 1, 0, None, None, None, None) == 0
     # activation: status required; NVFP4 needs input_scale
     assert lib.mxq_quantize_act(fake, 4, 64, 0, 0, 0, fake, fake, fake, None, fake, 4096, None) == 1
     assert lib.mxq_quantize_act(fake, 4, 64, 0, 0, 0, fake, fake, None, fake, fake, 4096, None) == 1

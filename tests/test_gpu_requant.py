@@ -1,0 +1,53 @@
+"""FP8 -> MX requantization on the GPU (mxq_requant_fp8_mx, through the C
+ABI) against the CPU oracle on the same seeded block-FP8 sources:
+bit-exact codes and scale bytes, linear and tiled scale layouts, source
+blocks that do and do not align with the tensor edges."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import layout
+from mxfp_block_scaled_b200 import mxq, workloads
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _setup():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from mxfp_block_scaled_b200 import build
+    build.build()
+    mxq.load()
+    oracle.build()
+
+
+@pytest.mark.parametrize("fmt", ["mxfp8", "mxfp4"])
+@pytest.mark.parametrize("rows,cols,brows,bcols", [(256, 512, 128, 128), (200, 384, 128, 128),
+                                                   (96, 256, 32, 64), (1, 32, 128, 128),
+                                                   (1536, 2048, 128, 128)])
+@pytest.mark.parametrize("lay", ["linear", "swizzled_128x4"])
+def test_requant_bit_exact(fmt, rows, cols, brows, bcols, lay):
+    codes, scales = workloads.block_fp8_source(rows, cols, seed=rows + cols, brows=brows, bcols=bcols)
+    out = mxq.requant_fp8_mx(codes.cuda(), scales.cuda(), brows, bcols, fmt, layout=lay)
+    torch.cuda.synchronize()
+    assert int(out["status"].item()) == 0
+    oc, os_ = oracle.requant_fp8_mx(codes.numpy(), scales.numpy(), brows, bcols, fmt)
+    assert np.array_equal(out["codes"].cpu().numpy(), oc)
+    got = out["scales"].cpu().numpy().reshape(-1)
+    want = os_.reshape(-1) if lay == "linear" else layout.to_tiled_128x4(os_)
+    assert np.array_equal(got, want)
+
+
+def test_requant_nonfinite_source_sets_status():
+    codes, scales = workloads.block_fp8_source(128, 256, seed=9)
+    codes[5, 77] = 0x7F                       # the E4M3 NaN pattern
+    out = mxq.requant_fp8_mx(codes.cuda(), scales.cuda(), 128, 128, "mxfp8")
+    torch.cuda.synchronize()
+    assert int(out["status"].item()) & mxq.DEV_NONFINITE_INPUT
+    codes, scales = workloads.block_fp8_source(128, 256, seed=9)
+    scales[0, 1] = float("inf")
+    out = mxq.requant_fp8_mx(codes.cuda(), scales.cuda(), 128, 128, "mxfp4")
+    torch.cuda.synchronize()
+    assert int(out["status"].item()) & mxq.DEV_NONFINITE_INPUT
