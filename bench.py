@@ -11,6 +11,7 @@ larger than L2, so no flush is needed between steps.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mine|reference]
     python bench.py --workload fp8_requant     # FP8 -> MXFP4 requantization of the same layer
+    python bench.py --workload nvfp4_weighted  # weighted-SSE scale search on the same layer
 
 Prints one JSON line on rank 0.  Under torchrun every rank converts its own
 layer (independent units, no data-path collective: weak scaling); the step
@@ -405,6 +406,78 @@ def run_requant(args, device):
     }
 
 
+def run_weighted(args, device):
+    """NVFP4 with the weighted-SSE scale search over one full-size layer:
+    gate_up [512, 1536, 2048] and down [512, 2048, 768], each with one shared
+    row of per-input-channel weights (the mean squared activation of a
+    synthetic 4096-token tile)."""
+    from mxfp_block_scaled_b200 import mxq, workloads
+    layer = Layer(seed=0, device=device, experts=args.experts)
+    calls = []
+    for name, x in (("gate_up", layer.gu), ("down", layer.dn)):
+        G, R, C = x.shape
+        a = workloads.activation_tile(4096, seed=7, device=device, hidden=C).float()
+        h = (a * a).mean(0).contiguous()
+        ws, _ = mxq._workspace("quantize_nvfp4", G, R, C, device)
+        out = {"codes": torch.empty((G, R, C // 2), dtype=torch.uint8, device=device),
+               "scales": torch.empty((G, R, C // 16), dtype=torch.uint8, device=device),
+               "s2": torch.empty(G, dtype=torch.float32, device=device),
+               "status": torch.zeros(1, dtype=torch.int32, device=device)}
+        calls.append((name, x, h, ws, out))
+    torch.cuda.synchronize()
+
+    def step(ev=None):
+        for i, (name, x, h, ws, out) in enumerate(calls):
+            G, R, C = x.shape
+            if ev is not None:
+                ev[i][0].record()
+            mxq.mxq_quantize_nvfp4_weighted(x, G, R, C, h, 1, "linear", out["codes"], out["scales"],
+                                            out["s2"], out["status"], ws)
+            if ev is not None:
+                ev[i][1].record()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    for c in calls:
+        if int(c[4]["status"].item()) != 0:
+            raise RuntimeError("device status on " + c[0])
+    events = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+               for _ in calls] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device_uuid()) as clk:
+        torch.cuda.synchronize()
+        t0.record()
+        for k in range(args.steps):
+            step(events[k])
+        t1.record()
+        torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / args.steps
+    call_ms = [statistics.mean(events[k][i][0].elapsed_time(events[k][i][1]) for k in range(args.steps))
+               for i in range(len(calls))]
+    n = layer.n_elems
+    peak, peak_kind = measured_peak()
+    gu_n = layer.gu.numel()
+    achieved = gu_n * Q_BYTES / (call_ms[0] * 1e-3) / 1e9
+    return {
+        "metric": "NVFP4 weighted-SSE scale search, quantize HBM GB/s (1 GPU)",
+        "value": n * Q_BYTES / (ms * 1e-3) / 1e9, "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "one full-size routed-expert layer, NVFP4 with the weighted-SSE scale "
+                               "search: gate_up bf16 [512,1536,2048] + down [512,2048,768]",
+                   "elements_per_gpu": n, "algorithmic_bytes_per_element": Q_BYTES,
+                   "passes": "two (group amax, then the search): W is read twice",
+                   "call_ms": dict(zip(["gate_up", "down"], call_ms))},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "kernel": "nvfp4_weighted_kernel (gate_up; limited by its binary64 "
+                               "arithmetic, not by HBM)", "peak_kind": peak_kind},
+        "gpu_launches": args.steps * len(calls) * 2,
+        "clocks": clk.summary(),
+    }
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -415,7 +488,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the e2e and CPU-baseline legs (profiling runs)")
-    ap.add_argument("--workload", default="nvfp4_layer", choices=["nvfp4_layer", "fp8_requant"],
+    ap.add_argument("--workload", default="nvfp4_layer",
+                    choices=["nvfp4_layer", "fp8_requant", "nvfp4_weighted"],
                     help="nvfp4_layer: the headline quantize + verify step; fp8_requant: block-FP8 "
                          "-> MXFP4 requantization of the same layer")
     ap.add_argument("--experts", type=int, default=EXPERTS,
@@ -444,6 +518,11 @@ def main():
         if world > 1:
             raise SystemExit("--workload fp8_requant runs on one GPU")
         print(json.dumps(run_requant(args, device)), flush=True)
+        return 0
+    if args.workload == "nvfp4_weighted":
+        if world > 1:
+            raise SystemExit("--workload nvfp4_weighted runs on one GPU")
+        print(json.dumps(run_weighted(args, device)), flush=True)
         return 0
 
     layer = Layer(seed=rank, device=device, experts=args.experts)

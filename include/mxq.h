@@ -173,6 +173,32 @@ MXQ_API mxq_status mxq_quantize_nvfp4(const uint16_t *x, int64_t n_groups, int64
                               uint32_t *m4_count, uint32_t *status, void *workspace,
                               size_t workspace_bytes, cudaStream_t stream);
 
+/* NVFP4 quantization with a weighted-SSE block-scale search.
+ * Source: josch15366/Qwen3.8-Flash-Next-NVFP4-LocalHessian-Experts, "What is
+ * different about it": the per-group weight scales are chosen by a
+ * Hessian-weighted search (ModelOpt local_hessian) instead of the plain
+ * amax / MSE sweep.  The pages give no formula; the readings are stated here.
+ *   x, n_groups, rows, cols, layout, codes, scales, s2, status, workspace:
+ *            as mxq_quantize_nvfp4 (same groups, same s2 = RN32(amax_g / 2688),
+ *            workspace of MXQ_OP_QUANTIZE_NVFP4).
+ *   h        fp32 weights >= 0 per input channel (a diagonal Hessian estimate,
+ *            e.g. the mean squared activation of that channel), 16-byte
+ *            aligned: [cols] shared by every group (h_groups == 1) or
+ *            [n_groups, cols] (h_groups == n_groups).
+ * Per block of 16: the candidates are every E4M3 scale code from the amax/6
+ * plan's code to the four-over-six plan's code (both plans as in
+ * mxq_quantize_nvfp4); each candidate's value codes follow as in that entry
+ * point, and its weighted error sum_i h_i (x_i - q_i D s2)^2 is formed in
+ * binary64 in element order (deq = (q D) s2, e = x - deq, acc += h (e e),
+ * each operation rounded to nearest).  The lowest error wins; ties go to the
+ * smaller code.  A negative or non-finite weight, like a non-finite input,
+ * sets MXQ_DEV_NONFINITE_INPUT. */
+MXQ_API mxq_status mxq_quantize_nvfp4_weighted(const uint16_t *x, int64_t n_groups, int64_t rows,
+                                               int64_t cols, const float *h, int64_t h_groups,
+                                               mxq_layout layout, uint8_t *codes, uint8_t *scales,
+                                               float *s2, uint32_t *status, void *workspace,
+                                               size_t workspace_bytes, cudaStream_t stream);
+
 /* MX quantization (MXFP4 or MXFP8), one UE8M0 scale per 32 values.
  * Source: azampatti/Qwen3.8-Flash-Next-FP4-Local-AZ, "The shared expert";
  * MJPansa/Qwen3.8-Flash-Next-MXFP4-FP8-R12, "Quantization format".

@@ -183,6 +183,50 @@ mxq_status mxq_quantize_nvfp4(const uint16_t *x, int64_t n_groups, int64_t rows,
     return e == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
 }
 
+mxq_status mxq_quantize_nvfp4_weighted(const uint16_t *x, int64_t n_groups, int64_t rows,
+                                       int64_t cols, const float *h, int64_t h_groups,
+                                       mxq_layout layout, uint8_t *codes, uint8_t *scales, float *s2,
+                                       uint32_t *status, void *workspace, size_t workspace_bytes,
+                                       cudaStream_t stream)
+{
+    if (n_groups < 0 || rows < 0 || cols < 0)
+        return MXQ_ERR_INVALID_ARG;
+    if (!layout_ok(layout) || (h_groups != 1 && h_groups != n_groups))
+        return MXQ_ERR_INVALID_ARG;
+    if (cols % 16 != 0)
+        return MXQ_ERR_SHAPE;
+    int64_t gsize, total;
+    if (!mul_ok(rows, cols, &gsize) || !mul_ok(gsize, n_groups, &total) || total > (INT64_MAX / 4))
+        return MXQ_ERR_SHAPE;
+    const bool swz = layout == MXQ_LAYOUT_SWIZZLED_128X4;
+    if (swz && gsize / 16 > 0x7FFFFFFF)
+        return MXQ_ERR_SHAPE;
+    if (n_groups == 0)
+        return MXQ_OK;
+    if (!x || !h || !codes || !scales || !s2 || !status)
+        return MXQ_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(h, 16) || !aligned(codes, 16) || !aligned(scales, 16) ||
+        !aligned(s2, 4) || !aligned(status, 4))
+        return MXQ_ERR_ALIGN;
+    const size_t need = nvfp4_workspace_bytes(n_groups);
+    if (!workspace || workspace_bytes < need)
+        return MXQ_ERR_WORKSPACE;
+    if (!aligned(workspace, 256))
+        return MXQ_ERR_ALIGN;
+    const int64_t nb = gsize / 16;
+    const ScaleLayout sl = make_scale_layout(swz ? 1 : 0, rows, cols / 16);
+    uint32_t *amax_bits = static_cast<uint32_t *>(workspace);
+    cudaError_t e = cudaMemsetAsync(amax_bits, 0, (size_t)n_groups * sizeof(uint32_t), stream);
+    if (e == cudaSuccess && swz)
+        e = zero_tiled_padding(scales, n_groups, rows, cols / 16, stream);
+    if (e == cudaSuccess)
+        e = launch_group_amax(x, n_groups, nb, amax_bits, status, stream);
+    if (e == cudaSuccess)
+        e = launch_nvfp4_weighted(x, n_groups, nb, cols, amax_bits, h, h_groups == 1 ? 0 : cols, codes,
+                                  scales, sl, s2, status, stream);
+    return e == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
+}
+
 mxq_status mxq_quantize_mx(const uint16_t *x, int64_t rows, int64_t cols, mxq_fmt fmt, int block,
                            mxq_layout layout, uint8_t *codes, uint8_t *scales, uint32_t *status,
                            cudaStream_t stream)

@@ -81,6 +81,10 @@ cudaError_t launch_nvfp4_fused(const uint16_t *x, int64_t n_groups, int64_t nb, 
                                const ScaleLayout &sl,
                                float *s2, uint32_t *mbits, uint32_t *m4_count, uint32_t *status,
                                cudaStream_t s);
+cudaError_t launch_nvfp4_weighted(const uint16_t *x, int64_t n_groups, int64_t nb, int64_t cols,
+                                  const uint32_t *amax_bits, const float *h, int64_t h_stride,
+                                  uint8_t *codes, uint8_t *scales, const ScaleLayout &sl, float *s2,
+                                  uint32_t *status, cudaStream_t s);
 cudaError_t launch_mx_quant(const uint16_t *x, int64_t nblk32, int fmt, uint8_t *codes,
                             uint8_t *scales, const ScaleLayout &sl, uint32_t *status, cudaStream_t s);
 cudaError_t launch_requant_fp8_mx(const uint8_t *fp8, const float *bscale, int64_t rows, int64_t cols,

@@ -30,7 +30,7 @@ LAYOUT = {"linear": 0, "swizzled_128x4": 1}
 OP = {"quantize_nvfp4": 0, "quantize_act": 1, "dequant_relerr": 2}
 
 EXPORTED = ("mxq_version", "mxq_status_string", "mxq_scale_bytes", "mxq_workspace_bytes",
-            "mxq_quantize_nvfp4",
+            "mxq_quantize_nvfp4", "mxq_quantize_nvfp4_weighted",
             "mxq_quantize_mx", "mxq_requant_fp8_mx", "mxq_quantize_act", "mxq_dequant_relerr",
             "mxq_dequant_relerr_noalloc")
 
@@ -64,6 +64,9 @@ def load(path=LIB_PATH):
     L.mxq_workspace_bytes.argtypes = [i32, i64, i64, i64]
     L.mxq_quantize_nvfp4.restype = i32
     L.mxq_quantize_nvfp4.argtypes = [vp, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.mxq_quantize_nvfp4_weighted.restype = i32
+    L.mxq_quantize_nvfp4_weighted.argtypes = [vp, i64, i64, i64, vp, i64, i32, vp, vp, vp, vp, vp, sz,
+                                              vp]
     L.mxq_quantize_mx.restype = i32
     L.mxq_quantize_mx.argtypes = [vp, i64, i64, i32, i32, i32, vp, vp, vp, vp]
     L.mxq_requant_fp8_mx.restype = i32
@@ -120,6 +123,16 @@ def mxq_quantize_nvfp4(x, n_groups, rows, cols, mode, layout, codes, scales, s2,
                                    _p(workspace), workspace.numel() if workspace is not None else 0,
                                    _stream(stream))
     _check("mxq_quantize_nvfp4", rc)
+
+
+def mxq_quantize_nvfp4_weighted(x, n_groups, rows, cols, h, h_groups, layout, codes, scales, s2,
+                                status, workspace, stream=None):
+    rc = load().mxq_quantize_nvfp4_weighted(_p(x), n_groups, rows, cols, _p(h), h_groups,
+                                            LAYOUT[layout], _p(codes), _p(scales), _p(s2), _p(status),
+                                            _p(workspace),
+                                            workspace.numel() if workspace is not None else 0,
+                                            _stream(stream))
+    _check("mxq_quantize_nvfp4_weighted", rc)
 
 
 def mxq_quantize_mx(x, rows, cols, fmt, block, layout, codes, scales, status, stream=None):
@@ -195,6 +208,28 @@ def quantize_nvfp4(x, mode="four_six", with_mbits=True, stream=None, layout="lin
     ws, _ = _workspace("quantize_nvfp4", G, R, C, dev)
     mxq_quantize_nvfp4(x, G, R, C, mode, layout, out["codes"], out["scales"], out["s2"],
                        out["mbits"], out["m4_count"], out["status"], ws, stream)
+    return out
+
+
+def quantize_nvfp4_weighted(x, h, stream=None, layout="linear"):
+    """x: bf16 [G, R, C]; h: fp32 weights per input channel, [C] (shared) or
+    [G, C].  Returns dict codes, scales, s2, status."""
+    _bf16(x)
+    G, R, C = x.shape
+    if h.dtype != torch.float32 or not h.is_contiguous() or h.shape[-1] != C:
+        raise ValueError("expected contiguous fp32 weights [C] or [G, C]")
+    hg = 1 if h.dim() == 1 else h.shape[0]
+    dev = x.device
+    out = {
+        "codes": torch.empty((G, R, C // 2), dtype=torch.uint8, device=dev),
+        "scales": torch.empty((G, R, C // 16), dtype=torch.uint8, device=dev) if layout == "linear"
+        else torch.empty(max(scale_bytes("nvfp4", layout, G, R, C), 1), dtype=torch.uint8, device=dev),
+        "s2": torch.empty(max(G, 1), dtype=torch.float32, device=dev),
+        "status": torch.zeros(1, dtype=torch.int32, device=dev),
+    }
+    ws, _ = _workspace("quantize_nvfp4", G, R, C, dev)
+    mxq_quantize_nvfp4_weighted(x, G, R, C, h, hg, layout, out["codes"], out["scales"], out["s2"],
+                                out["status"], ws, stream)
     return out
 
 

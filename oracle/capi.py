@@ -58,6 +58,8 @@ def lib():
         L.oracle_quantize_nvfp4.argtypes = [vp, i64, i64, i64, i, d, vp, vp, vp, vp]
         L.oracle_quantize_mx.restype = i
         L.oracle_quantize_mx.argtypes = [vp, i64, i64, i, vp, vp]
+        L.oracle_quantize_nvfp4_weighted.restype = i
+        L.oracle_quantize_nvfp4_weighted.argtypes = [vp, i64, i64, i64, vp, i64, vp, vp, vp]
         L.oracle_requant_fp8_mx.restype = i
         L.oracle_requant_fp8_mx.argtypes = [vp, vp, i64, i64, i64, i64, i, vp, vp]
         L.oracle_dequant_relerr.restype = i
@@ -130,6 +132,23 @@ def quantize_mx(x_bits, fmt):
     if rc != 0:
         raise RuntimeError("oracle_quantize_mx failed: %d" % rc)
     return codes, scales
+
+
+def quantize_nvfp4_weighted(x_bits, h):
+    """x_bits: uint16 [G, R, C]; h: float32 [C] (shared) or [G, C].
+    Returns codes [G,R,C/2], scales [G,R,C/16], s2 [G]."""
+    x = _as_bits(x_bits)
+    G, R, C = x.shape
+    hh = np.ascontiguousarray(h, np.float32)
+    hg = 1 if hh.ndim == 1 else hh.shape[0]
+    codes = np.zeros((G, R, C // 2), np.uint8)
+    scales = np.zeros((G, R, C // 16), np.uint8)
+    s2 = np.zeros(G, np.float32)
+    rc = lib().oracle_quantize_nvfp4_weighted(_ptr(x), G, R, C, _ptr(hh), hg, _ptr(codes),
+                                              _ptr(scales), _ptr(s2))
+    if rc != 0:
+        raise RuntimeError("oracle_quantize_nvfp4_weighted failed: %d" % rc)
+    return codes, scales, s2
 
 
 def requant_fp8_mx(fp8, bscale, brows, bcols, fmt):

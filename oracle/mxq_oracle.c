@@ -346,6 +346,111 @@ int oracle_quantize_mx(const uint16_t *x, int64_t rows, int64_t cols, int fmt,
  *   MXFP4 / MXFP8: deq = q * 2^(b - 127).
  * sum_sq_err[t] = sum (x - deq)^2, sum_sq_ref[t] = sum x^2, both as
  * binary64 sums in element order.  Returns 0 or -1. */
+/* Codes of one NVFP4 block for a given E4M3 scale code (the value half of
+ * nvfp4_plan): d = RN32(D * s2), code_i = E2M1(RN32(x_i / d)); all codes 0
+ * when D or d is 0. */
+static void nvfp4_codes_for_scale(const float x[16], float s2, unsigned sc, uint8_t codes[16])
+{
+    const double D = oracle_e4m3_value(sc);
+    const float d = (float)D * s2;
+    for (int i = 0; i < 16; ++i)
+        codes[i] = (D == 0.0 || d == 0.0f) ? 0 : (uint8_t)oracle_e2m1_encode((double)(x[i] / d));
+}
+
+/* Weighted squared error of one block in binary64, in this exact order
+ * (the GPU forms the same operations in the same order):
+ *   deq_i = (q_i * D) * s2            exact (2 + 4 + 24 significant bits)
+ *   e_i   = x_i - deq_i               rounded to nearest
+ *   acc  += h_i * (e_i * e_i)         two roundings, i = 0 .. 15 */
+static double nvfp4_wsse(const float x[16], const float h[16], float s2, unsigned sc,
+                         const uint8_t codes[16])
+{
+    const double D = oracle_e4m3_value(sc);
+    double acc = 0.0;
+    for (int i = 0; i < 16; ++i) {
+        const double deq = (oracle_e2m1_value(codes[i]) * D) * (double)s2;
+        const double e = (double)x[i] - deq;
+        acc = acc + (double)h[i] * (e * e);
+    }
+    return acc;
+}
+
+/* NVFP4 with a weighted-SSE scale search [P1 "What is different about it":
+ * per-group weight scales chosen by a Hessian-weighted search (ModelOpt
+ * local_hessian) instead of the plain amax / MSE sweep].  The pages give
+ * the idea, not the search; readings:
+ *   - weights h >= 0 per input channel (a diagonal Hessian estimate such
+ *     as the mean squared activation of that channel), one row of `cols`
+ *     per group (h_groups == n_groups) or one shared row (h_groups == 1);
+ *   - candidates: every E4M3 scale code from the amax/6 plan's code to the
+ *     four-over-six plan's code of the same block (the codes between the
+ *     two plans of the 4/6 rule, both included);
+ *   - objective: sum h_c (x - q D s2)^2 over the block, formed in binary64
+ *     as nvfp4_wsse states; the lowest value wins, ties to the smaller
+ *     code (the amax/6 side).
+ * s2, the plans' codes and the value codes follow oracle_quantize_nvfp4.
+ * Returns 0, -1 on bad arguments, -3 on non-finite input or weight. */
+int oracle_quantize_nvfp4_weighted(const uint16_t *x, int64_t n_groups, int64_t rows,
+                                   int64_t cols, const float *h, int64_t h_groups,
+                                   uint8_t *codes, uint8_t *scales, float *s2_out)
+{
+    if (n_groups < 0 || rows < 0 || cols < 0 || cols % 16 != 0 ||
+        (h_groups != 1 && h_groups != n_groups))
+        return -1;
+    const int64_t gsize = rows * cols;
+    const int64_t nblk = gsize / 16;
+    for (int64_t i = 0; i < h_groups * cols; ++i)
+        if (!isfinite(h[i]) || h[i] < 0.0f)
+            return -3;
+    for (int64_t g = 0; g < n_groups; ++g) {
+        const uint16_t *xg = x + g * gsize;
+        const float *hg = h + (h_groups == 1 ? 0 : g * cols);
+        float amax_g = 0.0f;
+        for (int64_t i = 0; i < gsize; ++i) {
+            float v = fabsf(bf16_to_float(xg[i]));
+            if (!isfinite(v))
+                return -3;
+            if (v > amax_g)
+                amax_g = v;
+        }
+        const float s2 = amax_g / 2688.0f;
+        s2_out[g] = s2;
+        for (int64_t b = 0; b < nblk; ++b) {
+            float xb[16];
+            float amax_b = 0.0f;
+            for (int i = 0; i < 16; ++i) {
+                xb[i] = bf16_to_float(xg[b * 16 + i]);
+                if (fabsf(xb[i]) > amax_b)
+                    amax_b = fabsf(xb[i]);
+            }
+            const float *hb = hg + (b * 16) % cols;
+            unsigned lo = 0, hi = 0;
+            if (s2 > 0.0f) {
+                lo = oracle_e4m3_encode((double)(amax_b / (6.0f * s2)));
+                hi = oracle_e4m3_encode((double)(amax_b / (4.0f * s2)));
+            }
+            unsigned best_sc = lo;
+            uint8_t best[16], c[16];
+            nvfp4_codes_for_scale(xb, s2, lo, best);
+            double best_w = nvfp4_wsse(xb, hb, s2, lo, best);
+            for (unsigned sc = lo + 1; sc <= hi; ++sc) {
+                nvfp4_codes_for_scale(xb, s2, sc, c);
+                const double w = nvfp4_wsse(xb, hb, s2, sc, c);
+                if (w < best_w) {
+                    best_w = w;
+                    best_sc = sc;
+                    memcpy(best, c, 16);
+                }
+            }
+            const int64_t gb = g * nblk + b;
+            for (int j = 0; j < 8; ++j)
+                codes[gb * 8 + j] = (uint8_t)((best[2 * j] & 0xF) | ((best[2 * j + 1] & 0xF) << 4));
+            scales[gb] = (uint8_t)best_sc;
+        }
+    }
+    return 0;
+}
+
 /* FP8 -> MX requantization [P4 "Quantization and layer selection": the
  * conversion started from the released FP8 weights, without a BF16 copy;
  * "Quantization format": the retained layers stay in the source block-FP8

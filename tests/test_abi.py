@@ -101,6 +101,15 @@ def test_host_argument_errors_return_before_any_launch(lib):
     # tiled layout: a scale matrix needs at least one tensor
     assert lib.mxq_dequant_relerr(fake, fake, fake, None, 2, 1, 2, 4, 64, 0, fake, fake, None, fake,
                                   4096, None) == 1
+    # weighted search: weight rows neither 1 nor n_groups, cols % 16, misaligned weights
+    assert lib.mxq_quantize_nvfp4_weighted(fake, 2, 4, 16, fake, 3, 0, fake, fake, fake, fake, fake,
+                                           4096, None) == 1
+    assert lib.mxq_quantize_nvfp4_weighted(fake, 2, 4, 24, fake, 1, 0, fake, fake, fake, fake, fake,
+                                           4096, None) == 2
+    assert lib.mxq_quantize_nvfp4_weighted(fake, 2, 4, 16, vp(0x1004), 1, 0, fake, fake, fake, fake,
+                                           fake, 4096, None) == 3
+    assert lib.mxq_quantize_nvfp4_weighted(None, 0, 4, 16, None, 1, 0, None, None, None, None, None,
+                                           0, None) == 0
     # FP8 -> MX requantization: source block width not a multiple of 32, bad block, bad format
     assert lib.mxq_requant_fp8_mx(fake, fake, 4, 64, 128, 48, 1, 0, fake, fake, None, None) == 2
     assert lib.mxq_requant_fp8_mx(fake, fake, 4, 64, 0, 128, 1, 0, fake, fake, None, None) == 1
