@@ -291,6 +291,18 @@ def run_e2e(layer, steps, device):
 
 
 # ------------------------------------------------------------- reference --
+def max_over_ranks(x, world, device):
+    """The largest per-rank value over all ranks (the step time of a weak-
+    scaling run is the slowest rank's).  One all-reduce of one number: the
+    data path itself exchanges nothing between ranks."""
+    if world <= 1:
+        return float(x)
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def run_reference(args, rank, world):
     """The oracle (CPU) as the reference arm: each step converts one expert
     (gate_up + down) of the same layer shape, quantize + verify."""
@@ -552,11 +564,7 @@ def main():
             layer.step(events[k])
         end.record()
         barrier()
-    ms = start.elapsed_time(end) / args.steps
-    if world > 1:
-        t = torch.tensor([ms], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(start.elapsed_time(end) / args.steps, world, device)
     call_ms = [statistics.mean(events[k][i][0].elapsed_time(events[k][i][1]) for k in range(args.steps))
                for i in range(len(Layer.CALLS))]
     total_elems = layer.n_elems * world
