@@ -117,14 +117,21 @@ __device__ __forceinline__ Plan plan_from_quotients(const float2 (&x)[8], const 
     uint32_t q[8];
     p.codes.x = e2m1x8_enc_dec(y[0], y[1], y[2], y[3], *reinterpret_cast<uint32_t(*)[4]>(&q[0]));
     p.codes.y = e2m1x8_enc_dec(y[4], y[5], y[6], y[7], *reinterpret_cast<uint32_t(*)[4]>(&q[4]));
-    float2 acc = make_float2(0.0f, 0.0f);
-    uint32_t bh = 0u;
+    // Two independent partial sums each (pairs 0-3 and 4-7): the sums are
+    // exact in any order, so splitting them only shortens the dependency
+    // chains.
+    float2 acc0 = make_float2(0.0f, 0.0f), acc1 = make_float2(0.0f, 0.0f);
+    uint32_t bh0 = 0u, bh1 = 0u;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        bh = hfma2_bits(q[j], q[j], bh);
-        acc = __ffma2_rn(x[j], f16x2_to_float2(q[j]), acc);
+    for (int j = 0; j < 4; ++j) {
+        bh0 = hfma2_bits(q[j], q[j], bh0);
+        bh1 = hfma2_bits(q[j + 4], q[j + 4], bh1);
+        acc0 = __ffma2_rn(x[j], f16x2_to_float2(q[j]), acc0);
+        acc1 = __ffma2_rn(x[j + 4], f16x2_to_float2(q[j + 4]), acc1);
     }
+    const float2 acc = __fadd2_rn(acc0, acc1);
     p.a = __fadd_rn(acc.x, acc.y);
+    const uint32_t bh = hadd2_bits(bh0, bh1);         // <= 288 per half: exact in f16
     const float2 bf = f16x2_to_float2(bh);
     p.b = __fadd_rn(bf.x, bf.y);
     return p;
@@ -235,10 +242,8 @@ template <bool FOUR_SIX>
 __device__ __forceinline__ BlockOut quantize_block(uint4 v0, uint4 v1, const GroupConst &gc)
 {
     const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    uint32_t m = 0;
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-        m = absmax_bf16x2(m, w[j]);
+    const uint32_t m = absmax_bf16x2(absmax_bf16x2(absmax_bf16x2(w[0], w[1]), absmax_bf16x2(w[2], w[3])),
+                                     absmax_bf16x2(absmax_bf16x2(w[4], w[5]), absmax_bf16x2(w[6], w[7])));
     const float amax_b = __uint_as_float(fold_halves(m) << 16);
     if (!gc.qfast)
         return quantize_block_general<FOUR_SIX>(v0, v1, amax_b, gc);

@@ -78,3 +78,115 @@ def relerr_census(results):
     expert census)."""
     rel = torch.cat([q[k]["relerr"] for q in results for k in ("gate_up", "down")])
     return float(rel.mean()), float(rel.max()), int(rel.numel())
+
+
+# ------------------------------------------------ host-resident layers --
+def host_outputs(h_gate_up, h_down):
+    """Pinned host buffers for convert_layer_from_host: per stack the codes,
+    scales, s2 and per-tensor relative errors (gate_up unstacked into 2E
+    tensors, down into E)."""
+    out = {}
+    for name, h in (("gate_up", h_gate_up), ("down", h_down)):
+        E, R, C = h.shape
+        nt = 2 * E if name == "gate_up" else E
+        out[name] = {
+            "codes": torch.empty((E, R, C // 2), dtype=torch.uint8, pin_memory=True),
+            "scales": torch.empty((E, R, C // 16), dtype=torch.uint8, pin_memory=True),
+            "s2": torch.empty(E, dtype=torch.float32, pin_memory=True),
+            "relerr": torch.empty(nt, dtype=torch.float64, pin_memory=True),
+        }
+    return out
+
+
+class _Slot:
+    """Device buffers of one chunk of `chunk` experts of one stack."""
+
+    def __init__(self, chunk, R, C, tps, device):
+        self.x = torch.empty((chunk, R, C), dtype=torch.bfloat16, device=device)
+        self.codes = torch.empty((chunk, R, C // 2), dtype=torch.uint8, device=device)
+        self.scales = torch.empty((chunk, R, C // 16), dtype=torch.uint8, device=device)
+        self.s2 = torch.empty(chunk, dtype=torch.float32, device=device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        nt = chunk * tps
+        self.err = torch.empty(nt, dtype=torch.float64, device=device)
+        self.ref = torch.empty(nt, dtype=torch.float64, device=device)
+        self.rel = torch.empty(nt, dtype=torch.float64, device=device)
+        self.wsq, _ = mxq._workspace("quantize_nvfp4", chunk, R, C, device)
+        self.wsv, _ = mxq._workspace("dequant_relerr", nt, R // tps, C, device)
+        self.ev_in = torch.cuda.Event()      # input copied in
+        self.ev_done = torch.cuda.Event()    # outputs written
+        self.ev_out = torch.cuda.Event()     # outputs copied out (slot free again)
+        self.used = False
+
+
+class HostLayerConverter:
+    """NVFP4 4/6 quantize + verify of routed-expert layers that live in pinned
+    host memory, in chunks of `chunk` experts.  Host -> device copies, the
+    kernels and device -> host copies of neighbouring chunks are queued on
+    three streams (event-ordered, `nbuf` device buffers per stack), so both
+    PCIe directions and the GPU work at the same time.  The results equal one
+    call per stack over the whole layer: every expert is its own NVFP4 group
+    (gate and up of an expert still share one weight_scale_2) and every
+    unstacked tensor is verified on its own.
+
+        conv = HostLayerConverter(h_gate_up.shape, h_down.shape)
+        out = host_outputs(h_gate_up, h_down)
+        conv.run(h_gate_up, h_down, out)    # enqueues; the current stream waits for it
+        torch.cuda.current_stream().synchronize()
+    """
+
+    def __init__(self, gate_up_shape, down_shape, chunk=64, mode="four_six", device="cuda", nbuf=2):
+        self.chunk, self.mode, self.device = int(chunk), mode, torch.device(device)
+        self.stacks = []
+        for name, shape, tps in (("gate_up", tuple(gate_up_shape), 2), ("down", tuple(down_shape), 1)):
+            E, R, C = shape
+            c = min(self.chunk, E)
+            self.stacks.append((name, shape, tps, [_Slot(c, R, C, tps, self.device) for _ in range(nbuf)]))
+        self.s_h2d = torch.cuda.Stream(device=self.device)
+        self.s_comp = torch.cuda.Stream(device=self.device)
+        self.s_d2h = torch.cuda.Stream(device=self.device)
+
+    def run(self, h_gate_up, h_down, out):
+        cur = torch.cuda.current_stream(self.device)
+        for s in (self.s_h2d, self.s_comp, self.s_d2h):
+            s.wait_stream(cur)
+        for (name, shape, tps, slots), h in zip(self.stacks, (h_gate_up, h_down)):
+            E, R, C = shape
+            o = out[name]
+            for k, e0 in enumerate(range(0, E, self.chunk)):
+                n = min(self.chunk, E - e0)
+                sl = slots[k % len(slots)]
+                with torch.cuda.stream(self.s_h2d):
+                    if sl.used:
+                        self.s_h2d.wait_event(sl.ev_done)       # the previous chunk has read x
+                    sl.x[:n].copy_(h[e0:e0 + n], non_blocking=True)
+                    sl.ev_in.record(self.s_h2d)
+                with torch.cuda.stream(self.s_comp):
+                    self.s_comp.wait_event(sl.ev_in)
+                    if sl.used:
+                        self.s_comp.wait_event(sl.ev_out)       # its outputs have been copied out
+                    mxq.mxq_quantize_nvfp4(sl.x[:n], n, R, C, self.mode, "linear", sl.codes[:n],
+                                           sl.scales[:n], sl.s2[:n], None, None, sl.status, sl.wsq,
+                                           stream=self.s_comp)
+                    mxq.mxq_dequant_relerr(sl.x[:n], sl.codes[:n], sl.scales[:n], sl.s2[:n], "nvfp4",
+                                           "linear", n * tps, R // tps, C, tps, sl.err[:n * tps],
+                                           sl.ref[:n * tps], sl.rel[:n * tps], sl.wsv,
+                                           stream=self.s_comp)
+                    sl.ev_done.record(self.s_comp)
+                with torch.cuda.stream(self.s_d2h):
+                    self.s_d2h.wait_event(sl.ev_done)
+                    o["codes"][e0:e0 + n].copy_(sl.codes[:n], non_blocking=True)
+                    o["scales"][e0:e0 + n].copy_(sl.scales[:n], non_blocking=True)
+                    o["s2"][e0:e0 + n].copy_(sl.s2[:n], non_blocking=True)
+                    o["relerr"][e0 * tps:(e0 + n) * tps].copy_(sl.rel[:n * tps], non_blocking=True)
+                    sl.ev_out.record(self.s_d2h)
+                sl.used = True
+        cur.wait_stream(self.s_d2h)
+
+    def status(self):
+        """OR of the device status words of every chunk (after a sync)."""
+        v = 0
+        for _, _, _, slots in self.stacks:
+            for sl in slots:
+                v |= int(sl.status.item())
+        return v
