@@ -359,7 +359,7 @@ nvfp4_quant_kernel(const uint4 *__restrict__ x, int64_t n_groups, int64_t nb,
 //   quantize copy  (ring of `qstages`), issued only after the scouts are
 //                  done with that group, `distance` groups behind them, so
 //                  it normally hits the L2 copy the scout read left behind:
-//                  21 compute warps quantize it once a publisher warp has
+//                  20 compute warps quantize it once a publisher warp has
 //                  seen every CTA's slot for the group.  The publisher polls
 //                  only the one arrival word of a group; it reads the slots
 //                  (and checks their tags) once the count is complete, so
