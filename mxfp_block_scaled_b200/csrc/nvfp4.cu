@@ -658,15 +658,25 @@ nvfp4_fused_kernel(const FusedArgs a)
     // -------------------------------------------------------- compute warps
     if (bytes == 0)
         return;
-    // Chunks of 32 blocks are dealt round-robin over the compute warps along
-    // the whole sequence of this CTA's groups (chunk n32 * j + k of group j
-    // goes to warp (n32 * j + k) % kFusedComputeWarps), so the work stays
-    // balanced when a slice's chunk count is not a multiple of the warp
-    // count; a warp with no chunk in a group still frees the group's buffer.
+    // Chunks of 32 blocks are dealt per SM sub-partition (warp index mod 4):
+    // the n32 chunks of a group are cut into four runs, the longer runs going
+    // to sub-partitions 0 and 1, which host the light publisher and loader
+    // warps, and the shorter ones to 2 and 3, which host the scout warps (with
+    // the 42 chunks of the full-size slices: 11, 11, 10, 10).  Inside a
+    // sub-partition the chunks go round-robin over its compute warps along
+    // the whole group sequence, so a run whose length is not a multiple of
+    // the warp count stays balanced; a warp with no chunk in a group still
+    // frees the group's buffer.
+    static_assert(kFusedComputeWarps % 4 == 0 && (2 + kFusedScoutWarps) % 4 == 0,
+                  "compute warps must fill the four sub-partitions evenly");
+    constexpr int kWarpsPerPart = kFusedComputeWarps / 4;
     const int cw = warp - 2 - kFusedScoutWarps;
+    const int part = warp & 3, li = cw >> 2;            // sub-partition, index inside it
     const int n32 = (int)(my_n / 32);
-    const int step = n32 % kFusedComputeWarps;          // chunk offset gained per group
-    int first = cw;                                     // this warp's first chunk in group j
+    const int run = (n32 >> 2) + (part < (n32 & 3) ? 1 : 0);
+    const int run0 = part * (n32 >> 2) + min(part, n32 & 3);
+    const int step = run % kWarpsPerPart;               // offset gained per group
+    int first = li;                                     // this warp's first chunk of the run
     int st = 0, rs = 0;                                 // quantize stage and ready slot of group j
     uint32_t qpar = 0, rpar = 0;                        // their phase parities
     for (int j = 0; j < G; ++j) {
@@ -682,7 +692,8 @@ nvfp4_fused_kernel(const FusedArgs a)
         uint8_t *scales = a.scales + gb0;
         uint32_t *mbits = a.mbits ? a.mbits + (gb0 >> 5) : nullptr;
         uint32_t cnt = 0;
-        for (int k32 = first; k32 < n32; k32 += kFusedComputeWarps) {
+        for (int c = first; c < run; c += kWarpsPerPart) {
+            const int k32 = run0 + c;
             const int k = k32 * 32 + lane;
             const BlockOut o = quantize_block<FOUR_SIX>(v[2 * k], v[2 * k + 1], gc);
             codes[k] = o.codes;
@@ -711,9 +722,9 @@ nvfp4_fused_kernel(const FusedArgs a)
             rs = 0;
             rpar ^= 1u;
         }
-        first -= step;                                  // (cw - n32 * (j + 1)) mod warps
+        first -= step;                                  // (li - run * (j + 1)) mod warps
         if (first < 0)
-            first += kFusedComputeWarps;
+            first += kWarpsPerPart;
     }
 }
 
