@@ -349,6 +349,9 @@ mxq_status mxq_dequant_relerr(const uint16_t *x, const uint8_t *codes, const uin
     int64_t msize = 0;
     if (swz && (!mul_ok(tsize, tensors_per_scale, &msize) || msize / blk > 0x7FFFFFFF))
         return MXQ_ERR_SHAPE;   // tiled offsets index the blocks of a matrix in 32 bits
+    const int64_t cpt = tsize > 0 ? (tsize + kVerifyChunk - 1) / kVerifyChunk : 1;
+    if (n_tensors > 0x7FFFFFFF / cpt || tensors_per_scale > 0x7FFFFFFF)
+        return MXQ_ERR_SHAPE;   // the verifier indexes its chunks in 32 bits
     if (n_tensors == 0)
         return MXQ_OK;
     if (!sum_sq_err || !sum_sq_ref)

@@ -109,8 +109,8 @@ __global__ void __launch_bounds__(kVerifyThreads)
 verify_chunk_kernel(const uint16_t *__restrict__ x, const uint8_t *__restrict__ codes,
                     const uint8_t *__restrict__ scales, const float *__restrict__ s2,
                     const ScaleLayout sl, int64_t n_tensors, int64_t rows, int64_t tsize,
-                    int64_t chunks_per_tensor, int64_t tensors_per_scale,
-                    double *__restrict__ partials)
+                    int64_t chunks_per_tensor, int64_t tensors_per_scale, const FastDiv cptdiv,
+                    const FastDiv tpsdiv, double *__restrict__ partials)
 {
     constexpr int BLK = (FMT == MXQ_FMT_NVFP4) ? 16 : 32;
     // blocks per thread per chunk; all of a thread's loads are issued before
@@ -120,16 +120,19 @@ verify_chunk_kernel(const uint16_t *__restrict__ x, const uint8_t *__restrict__ 
     constexpr int CV = (FMT == MXQ_FMT_MXFP8) ? 2 : 1;            // uint4 of codes (MX)
     const int64_t n_chunks = n_tensors * chunks_per_tensor;
     for (int64_t c = blockIdx.x; c < n_chunks; c += gridDim.x) {
-        const int64_t t = c / chunks_per_tensor;
+        // chunk -> (tensor, chunk of the tensor) with one multiply-shift
+        // division (chunk counts stay below 2^32: checked at launch)
+        const int64_t t = fastdiv((uint32_t)c, cptdiv);
         const int64_t k = c - t * chunks_per_tensor;
+        const int64_t ts = fastdiv((uint32_t)t, tpsdiv);      // scale matrix / s2 of tensor t
         const int64_t lo = k * kVerifyChunk;
         const int64_t hi = min(lo + kVerifyChunk, tsize);
         const int64_t nblk = (hi - lo) / BLK;
         const int64_t first = (t * tsize + lo) / BLK;   // global block index
-        const float sv = (FMT == MXQ_FMT_NVFP4) ? __ldg(s2 + t / tensors_per_scale) : 0.0f;
+        const float sv = (FMT == MXQ_FMT_NVFP4) ? __ldg(s2 + ts) : 0.0f;
         // tiled scales: tensor t is rows [(t % tps) * rows, ...) of matrix t / tps
-        const uint64_t smat = SWZ ? (uint64_t)(t / tensors_per_scale) : 0;
-        const uint32_t sb0 = SWZ ? (uint32_t)((t % tensors_per_scale) * rows) * sl.cb + (uint32_t)(lo / BLK) : 0;
+        const uint64_t smat = SWZ ? (uint64_t)ts : 0;
+        const uint32_t sb0 = SWZ ? (uint32_t)((t - ts * tensors_per_scale) * rows) * sl.cb + (uint32_t)(lo / BLK) : 0;
         uint4 xv[PER][XV];
         uint4 cv[PER][CV];
         uint2 c2[PER];
@@ -207,10 +210,14 @@ cudaError_t launch_verify(const uint16_t *x, const uint8_t *codes, const uint8_t
     const int64_t cpt = tsize > 0 ? (tsize + kVerifyChunk - 1) / kVerifyChunk : 1;
     int64_t n_chunks = n_tensors * cpt;
     const unsigned grid = (unsigned)(n_chunks < 0x7FFFFFFF ? n_chunks : 0x7FFFFFFF);
+    if (n_chunks > 0x7FFFFFFF || cpt > 0x7FFFFFFF || tensors_per_scale > 0x7FFFFFFF)
+        return cudaErrorInvalidValue;                         // indices below are 32-bit
+    const FastDiv cptdiv = make_fastdiv((uint32_t)cpt);
+    const FastDiv tpsdiv = make_fastdiv((uint32_t)tensors_per_scale);
 #define MXQ_VERIFY(F, W)                                                                      \
     verify_chunk_kernel<F, W><<<grid, kVerifyThreads, 0, s>>>(x, codes, scales, s2, sl, n_tensors, \
                                                               rows, tsize, cpt, tensors_per_scale, \
-                                                              partials)
+                                                              cptdiv, tpsdiv, partials)
     if (fmt == MXQ_FMT_NVFP4) {
         if (sl.swz) MXQ_VERIFY(MXQ_FMT_NVFP4, true); else MXQ_VERIFY(MXQ_FMT_NVFP4, false);
     } else if (fmt == MXQ_FMT_MXFP8) {
