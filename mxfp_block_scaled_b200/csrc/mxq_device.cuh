@@ -181,6 +181,24 @@ __device__ __forceinline__ float2 div2_bf16(float2 x, float2 d, float2 nr)
     return __ffma2_rn(e, nr, q0);                                       // q0 - e * r
 }
 
+// ---- correctly rounded reciprocal of a pair -----------------------------
+// RN32(1/d) for |d| in [2^-60, 2^60]: the hardware approximation
+// (rcp.approx.ftz.f32 of the PTX ISA) refined by one Newton-Raphson step
+// whose residual 1 - d*y0 is formed by an FMA (Markstein, IBM J. Res. Dev.
+// 34(1), 1990).  In that range no operand or result is subnormal, so the
+// result depends on the significand of d alone; it equals the correctly
+// rounded reciprocal for every significand at every exponent of the range
+// (exhaustive check on the device: tests/test_gpu_reciprocal.py).  Outside
+// the range callers use __frcp_rn.
+__device__ __forceinline__ float2 rcp2_rn_mid(float2 d)
+{
+    float2 y0;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y0.x) : "f"(d.x));
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y0.y) : "f"(d.y));
+    const float2 e = __ffma2_rn(make_float2(-d.x, -d.y), y0, make_float2(1.0f, 1.0f));
+    return __ffma2_rn(y0, e, y0);
+}
+
 // ---- division by a run-time invariant divisor ---------------------------
 // q = n / d for unsigned 32-bit n and 1 <= d < 2^31 with one high multiply
 // (Granlund and Montgomery, "Division by invariant integers using

@@ -81,7 +81,8 @@ struct GroupConst {
     float s2;        // global scale
     float2 den;      // (RN32(6 s2), 4 s2): the divisors of the two plans' block scales
     float2 nr;       // (-RN32(1 / den.x), -RN32(1 / den.y)) when `tfast`
-    double s2h;      // s2 / 2 (exact), for the decision
+    double s2h;      // s2 / 2 (exact), for the exact decision
+    float s2hf;      // s2 / 2 in fp32 (exact when `qfast`), for the filtered decision
     int tfast;       // den in the range where the reciprocal quotient is exact
     int qfast;       // s2 in [2^-50, 2^50]: every non-zero block scale gives a
                      // divisor d = RN32(D s2) in [2^-59, 2^59], where the
@@ -98,6 +99,7 @@ __device__ __forceinline__ GroupConst make_group_const(uint32_t amax_bits)
     c.qfast = (c.s2 >= 0x1p-50f && c.s2 <= 0x1p50f) ? 1 : 0;
     c.nr = c.tfast ? make_float2(-__frcp_rn(c.den.x), -__frcp_rn(c.den.y)) : make_float2(0.0f, 0.0f);
     c.s2h = 0.5 * (double)c.s2;
+    c.s2hf = 0.5f * c.s2;
     return c;
 }
 
@@ -179,6 +181,34 @@ __device__ __forceinline__ double plan_g(float D, double s2h, const Plan &p)
     return dD * fma(dD * s2h, (double)p.b, -(double)p.a);
 }
 
+// The same decision, settled in fp32 for all but near-ties (fast path only:
+// s2 in [2^-50, 2^50], both scale codes non-zero).  With D_M = m 2^e (m a
+// 4-bit integer) the two scales satisfy 1 <= D4 / D6 <= 2, so e4 - e6 is 0
+// or 1; B_M = k/4 with k <= 2304.  Hence D_M B_M (<= 16 bits) and D_M^2 B_M
+// (<= 20 bits) are exact, and P = D6^2 B6 - D4^2 B4 is an integer multiple of
+// 2^(2 e6 - 2) below 2^(2 e6 + 20): exact as well.  What remains rounds
+// three times (v4 = D4 A4, Q = D6 A6 - v4, dl = s2/2 P - Q, each RN32 of an
+// exact product or FMA), so dl differs from G6/2 - G4/2 by at most
+// 2^-24 (|v4| + |Q| + |dl|) (1 + 2^-23).  When |dl| > 2^-20 (|v4| + |Q|)
+// that error is below |dl| / 15: the sign of dl is the sign of the exact
+// difference and it is not zero.  Otherwise it is a tie or a near-tie: equal
+// scales (both saturated at 448, as in every block whose amax is within a
+// few percent of the group amax) make the two plans identical, a tie kept at
+// M=6; the rest goes to the fp64 decision above.
+__device__ __forceinline__ bool prefer_four(float2 D, const GroupConst &gc, const Plan &p6, const Plan &p4)
+{
+    const float2 u = __fmul2_rn(D, make_float2(p6.b, p4.b));              // D B, exact
+    const float P = __fmaf_rn(D.x, u.x, -__fmul_rn(D.y, u.y));            // exact
+    const float v4 = __fmul_rn(D.y, p4.a);
+    const float Q = __fmaf_rn(D.x, p6.a, -v4);
+    const float dl = __fmaf_rn(gc.s2hf, P, -Q);
+    if (fabsf(dl) > 0x1p-20f * (fabsf(v4) + fabsf(Q)))
+        return dl > 0.0f;
+    if (D.x == D.y)
+        return false;
+    return plan_g(D.y, gc.s2h, p4) < plan_g(D.x, gc.s2h, p6);
+}
+
 struct BlockOut {
     uint2 codes;
     uint32_t scale;
@@ -237,7 +267,9 @@ __device__ __noinline__ BlockOut quantize_block_general(uint4 v0, uint4 v1, floa
 // One block of 16.  With s2 in [2^-50, 2^50] (`qfast`, uniform over a group)
 // and both scale codes non-zero, every divisor lies in the exact range of
 // the reciprocal quotient, so the two plans run straight-line with no range
-// tests; the block amax quotients of both plans share packed operations.
+// tests; the block amax quotients of both plans share packed operations, the
+// two reciprocals come from one refined approximation pair (rcp2_rn_mid) and
+// the M choice is settled in fp32 except at near-ties (prefer_four).
 template <bool FOUR_SIX>
 __device__ __forceinline__ BlockOut quantize_block(uint4 v0, uint4 v1, const GroupConst &gc)
 {
@@ -256,15 +288,17 @@ __device__ __forceinline__ BlockOut quantize_block(uint4 v0, uint4 v1, const Gro
     float2 x[8];
     unpack_x(w, x);
     BlockOut o;
-    const Plan p6 = make_plan_fast(x, d.x, __frcp_rn(d.x));
     if (!FOUR_SIX) {
+        const Plan p6 = make_plan_fast(x, d.x, __frcp_rn(d.x));
         o.codes = p6.codes;
         o.scale = sb & 0xFFu;
         o.m4 = false;
         return o;
     }
-    const Plan p4 = make_plan_fast(x, d.y, __frcp_rn(d.y));
-    const bool use4 = plan_g(D.y, gc.s2h, p4) < plan_g(D.x, gc.s2h, p6);
+    const float2 r = rcp2_rn_mid(d);                    // d in [2^-59, 2^59]
+    const Plan p6 = make_plan_fast(x, d.x, r.x);
+    const Plan p4 = make_plan_fast(x, d.y, r.y);
+    const bool use4 = prefer_four(D, gc, p6, p4);
     o.codes = use4 ? p4.codes : p6.codes;
     o.scale = use4 ? (sb >> 8) : (sb & 0xFFu);
     o.m4 = use4;

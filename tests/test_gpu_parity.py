@@ -122,6 +122,48 @@ def test_degenerate_values():
     check_nvfp4(to_dev_bf16(xb), mode="rtn", label="degenerate rtn")
 
 
+def _tie_rich_blocks(seed, nblocks):
+    """Blocks on grids both plans represent exactly (so the exact 4/6
+    decision meets ties G4 == G6 with different scale codes), blocks that
+    add an element both plans round to zero (equal non-zero errors), blocks
+    exact in the M=4 plan only, and plain random blocks; the first element
+    sets the group amax to 2.625, so s2 = 2^-10 exactly."""
+    from oracle import micro
+    rng = np.random.default_rng(seed)
+    s2 = 2.0 ** -10
+    scales = [v for v in micro.E4M3_LIST[1:127] if 1.5 * v in micro.E4M3_LIST and 1.5 * v <= 448]
+    x = np.zeros((nblocks, 16), np.float32)
+    for b in range(nblocks):
+        base = np.float32(scales[rng.integers(len(scales))] * s2)
+        v = rng.choice([0.0, 1.5, 3.0, 6.0, -1.5, -3.0, -6.0], 16) * base
+        v[rng.integers(16)] = 6.0 * base * rng.choice([1, -1])
+        if b % 4 == 1:
+            v[rng.integers(16)] = base * 2.0 ** -6
+        elif b % 4 == 2:
+            v = rng.standard_normal(16) * 0.3
+        elif b % 4 == 3:
+            v[rng.integers(16)] = base * 0.75
+        x[b] = v
+    x[0] = 0.0
+    x[0, 0] = 2.625
+    return x
+
+
+@pytest.mark.parametrize("shape", [(2, 4, 256), (3, 1, 16 * 33)])
+def test_exact_decision_at_ties(shape):
+    """Ties and near-ties of the two plans' exact errors leave the fp32
+    filter undecided and must fall back to the exact decision (M=6 on a
+    tie), bit-exact with the oracle on both schedules (single pass: blocks
+    per group a multiple of 32; two-pass otherwise)."""
+    G, R, C = shape
+    nb = R * C // 16
+    x = np.stack([_tie_rich_blocks(100 + g, nb).reshape(R, C) for g in range(G)])
+    xt = torch.from_numpy(x).to(torch.bfloat16)
+    out, (_, _, s2, m4) = check_nvfp4(xt.cuda(), label="ties %s" % (shape,))
+    assert np.all(s2 == np.float32(2.0 ** -10))
+    assert 0 < m4.sum() < m4.size
+
+
 def test_nonfinite_input_sets_status():
     x = torch.randn((2, 4, 32)).to(torch.bfloat16).cuda()
     x[1, 2, 5] = float("inf")
