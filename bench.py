@@ -12,6 +12,9 @@ larger than L2, so no flush is needed between steps.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mine|reference]
     python bench.py --workload fp8_requant     # FP8 -> MXFP4 requantization of the same layer
     python bench.py --workload nvfp4_weighted  # weighted-SSE scale search on the same layer
+    python bench.py --workload mxfp8_shared    # MXFP8 rewrite of 48 shared experts (dense + padded)
+    python bench.py --workload mxfp4_layer     # MXFP4 quantize + verify of a full-size layer
+    python bench.py --workload act_sweep       # activation tiles [T, 2048], NVFP4 and MXFP8
 
 Prints one JSON line on rank 0.  Under torchrun every rank converts its own
 layer (independent units, no data-path collective: weak scaling); the step
@@ -471,6 +474,292 @@ def run_weighted(args, device):
     }
 
 
+def time_calls(calls, steps, warmup):
+    """CUDA-event timing of `steps` passes over `calls` (callables issuing
+    device work on the current stream) after `warmup` passes: mean step
+    time, each call's mean time (ms) and the clock samples of the timed
+    region."""
+    for _ in range(warmup):
+        for c in calls:
+            c()
+    torch.cuda.synchronize()
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in calls]
+          for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device_uuid()) as clk:
+        torch.cuda.synchronize()
+        t0.record()
+        for k in range(steps):
+            for i, c in enumerate(calls):
+                ev[k][i][0].record()
+                c()
+                ev[k][i][1].record()
+        t1.record()
+        torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / steps
+    call_ms = [statistics.mean(ev[k][i][0].elapsed_time(ev[k][i][1]) for k in range(steps))
+               for i in range(len(calls))]
+    return ms, call_ms, clk.summary()
+
+
+MX_BYTES = {"mxfp8": 2.0 + 1.0 + 1.0 / 32, "mxfp4": 2.0 + 0.5 + 1.0 / 32}   # per element, each pass
+
+
+class MXStack:
+    """One stack of equally shaped tensors, quantized to MX as a single
+    [rows, cols] matrix (MX scales are per 32 values: no per-tensor state)
+    and verified per tensor of `trows` rows."""
+
+    def __init__(self, mxq, x2d, fmt, trows, device):
+        self.mxq, self.x, self.fmt, self.trows = mxq, x2d, fmt, trows
+        self.R, self.C = x2d.shape
+        self.nt = self.R // trows
+        self.codes = torch.empty((self.R, self.C if fmt == "mxfp8" else self.C // 2), dtype=torch.uint8,
+                                 device=device)
+        self.scales = torch.empty((self.R, self.C // 32), dtype=torch.uint8, device=device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        ws = mxq.workspace_bytes("dequant_relerr", self.nt, trows, self.C)
+        self.wsv = torch.empty(max(ws, 256), dtype=torch.uint8, device=device)
+        self.err, self.ref, self.rel = (torch.empty(self.nt, dtype=torch.float64, device=device)
+                                        for _ in range(3))
+
+    def quantize(self):
+        self.mxq.mxq_quantize_mx(self.x, self.R, self.C, self.fmt, 32, "linear", self.codes, self.scales,
+                                 self.status)
+
+    def verify(self):
+        self.mxq.mxq_dequant_relerr(self.x, self.codes, self.scales, None, self.fmt, "linear", self.nt,
+                                    self.trows, self.C, 1, self.err, self.ref, self.rel, self.wsv)
+
+
+def mx_cpu_baseline(stacks, fmt, budget_s=15.0):
+    """The oracle as it stands (single-threaded C) on whole tensors of the
+    same stacks, quantize + verify, until about budget_s of CPU work."""
+    import oracle
+    from mxfp_block_scaled_b200 import workloads
+    oracle.build()
+    n_el, t_total, done = 0, 0.0, 0
+    for k in range(max(s.nt for s in stacks)):
+        for s in stacks:
+            if k >= s.nt or t_total >= budget_s:
+                continue
+            xb = workloads.bf16_bits(s.x[k * s.trows:(k + 1) * s.trows])
+            t0 = time.perf_counter()
+            c, sc = oracle.quantize_mx(xb, fmt)
+            oracle.dequant_relerr(xb, c, sc, None, fmt, 1, s.trows, s.C, 1)
+            t_total += time.perf_counter() - t0
+            n_el += xb.size
+            done += 1
+        if t_total >= budget_s:
+            break
+    return {"value": n_el * 2 * MX_BYTES[fmt] / t_total / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": "%d tensors (%.1fM elements), %s quantize + verify, %.1f s single-threaded C"
+                      % (done, n_el / 1e6, fmt, t_total), "elements_per_s": n_el / t_total}
+
+
+def run_mx(args, device):
+    """MX quantize + verify.  mxfp8_shared: the shared-expert MXFP8 rewrite,
+    48 layers x {dense, MTP-style padded} of gate/up [2560, 2048] and down
+    [2048, 1280]; mxfp4_layer: one full-size routed-expert layer
+    [512, 1536, 2048] + [512, 2048, 768] with the Student-t tail mix, as the
+    MXFP4 layers of the mixed-format conversion."""
+    from mxfp_block_scaled_b200 import mxq, workloads
+    if args.workload == "mxfp8_shared":
+        fmt, layers = "mxfp8", 48
+        gus, dns = [], []
+        for L in range(layers):
+            for padded in (False, True):
+                gu, dn = workloads.shared_expert_layer(seed=L, device=device, padded=padded)
+                gus.append(gu)
+                dns.append(dn)
+        GU, DN = torch.stack(gus), torch.stack(dns)
+        del gus, dns
+        stacks = [MXStack(mxq, GU.view(-1, GU.shape[-1]), fmt, GU.shape[1] // 2, device),
+                  MXStack(mxq, DN.view(-1, DN.shape[-1]), fmt, DN.shape[1], device)]
+        workload = ("shared-expert MXFP8 rewrite, quantize + verify: 48 layers x {dense, padded} of "
+                    "gate/up bf16 [2560,2048] + down [2048,1280] (gate and up verified separately)")
+        check_pad = True
+    else:
+        fmt = "mxfp4"
+        GU, DN = workloads.student_t_mix_layer(seed=0, device=device, experts=args.experts)
+        stacks = [MXStack(mxq, GU.view(-1, GU.shape[-1]), fmt, GU.shape[1] // 2, device),
+                  MXStack(mxq, DN.view(-1, DN.shape[-1]), fmt, DN.shape[1], device)]
+        workload = ("one full-size routed-expert layer (Student-t tail mix), MXFP4 quantize + verify: "
+                    "gate_up bf16 [%d,1536,2048] + down [%d,2048,768]" % (args.experts, args.experts))
+        check_pad = False
+    torch.cuda.synchronize()
+    calls = [s.quantize for s in stacks] + [s.verify for s in stacks]
+    ms, call_ms, clocks = time_calls(calls, args.steps, args.warmup)
+    for s in stacks:
+        if int(s.status.item()) != 0:
+            raise RuntimeError("device status %#x" % int(s.status.item()))
+    if check_pad:
+        # the padded copies (odd stack entries) must quantize to exact zeros, codes and scale
+        # bytes: gate rows [640, 1280) and up rows [1920, 2560) of gate/up, columns [640, 1280)
+        # of down
+        cg = stacks[0].codes.view(GU.shape[0], GU.shape[1], -1)[1::2]
+        sg = stacks[0].scales.view(GU.shape[0], GU.shape[1], -1)[1::2]
+        cd = stacks[1].codes.view(DN.shape[0], DN.shape[1], -1)[1::2]
+        sd = stacks[1].scales.view(DN.shape[0], DN.shape[1], -1)[1::2]
+        zero = [cg[:, 640:1280], cg[:, 1920:], sg[:, 640:1280], sg[:, 1920:], cd[:, :, 640:], sd[:, :, 20:]]
+        if any(int(z.count_nonzero()) for z in zero):
+            raise RuntimeError("padded regions did not quantize to zeros")
+    n = sum(s.R * s.C for s in stacks)
+    bpe = 2 * MX_BYTES[fmt]
+    peak, peak_kind = measured_peak()
+    value = n * bpe / (ms * 1e-3) / 1e9
+    gu_n = stacks[0].R * stacks[0].C
+    achieved = gu_n * MX_BYTES[fmt] / (call_ms[0] * 1e-3) / 1e9
+    rel = torch.cat([s.rel for s in stacks]).cpu().numpy()
+    names = ["quantize_gate_up", "quantize_down", "verify_gate_up", "verify_down"]
+    result = {
+        "metric": "%s quantize+verify HBM GB/s (1 GPU)" % fmt.upper(), "value": value, "unit": "GB/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": workload, "elements_per_gpu": n, "algorithmic_bytes_per_element": bpe,
+                   "l2": "inputs %.1f GB, larger than L2; no flush" % (n * 2 / 1e9),
+                   "fraction_of_peak": value / peak, "peak_gbs": peak, "peak_kind": peak_kind,
+                   "call_ms": dict(zip(names, call_ms)),
+                   "quality": {"relerr_mean": float(rel.mean()), "relerr_max": float(rel.max()),
+                               "tensors": int(rel.size)}},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "kernel": "mx_quant_kernel<%s> (gate_up stack)" % fmt.upper(),
+                     "algorithmic_bytes_per_launch": gu_n * MX_BYTES[fmt], "peak_kind": peak_kind},
+        "gpu_launches": args.steps * (2 + 2 * KERNELS_PER_VERIFY),
+        "clocks": clocks,
+    }
+    if not args.no_extras:
+        result["cpu_baseline"] = mx_cpu_baseline(stacks, fmt, args.cpu_budget)
+    return result
+
+
+def time_loop(call, reps, warmup):
+    """Mean time (us) of `reps` back-to-back calls on the current stream,
+    CUDA events around the whole loop, and the clock samples."""
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device_uuid()) as clk:
+        torch.cuda.synchronize()
+        t0.record()
+        for _ in range(reps):
+            call()
+        t1.record()
+        torch.cuda.synchronize()
+    return t0.elapsed_time(t1) * 1e3 / reps, clk.summary()
+
+
+def time_graph(call, reps):
+    """Mean device time (us) per call of `reps` calls captured in one CUDA
+    graph (no host launch cost), or None where the capture is refused."""
+    try:
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            call()
+        torch.cuda.current_stream().wait_stream(s)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(reps):
+                call()
+        g.replay()
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record()
+        g.replay()
+        t1.record()
+        torch.cuda.synchronize()
+        del g
+        return t0.elapsed_time(t1) * 1e3 / reps
+    except Exception as e:   # capture refused: report the stream timing only
+        log("graph capture:", e)
+        torch.cuda.synchronize()
+        return None
+
+
+ACT_T = (1, 16, 256, 4096, 65536)
+ACT_BYTES = {"nvfp4": 2.0 + 0.5 + 1.0 / 16, "mxfp8": 2.0 + 1.0 + 1.0 / 32}   # quantize only
+
+
+def run_act(args, device):
+    """Dynamic activation quantization of token tiles [T, 2048] (N(0, 1),
+    four outlier channels x 30): NVFP4 (input_scale = amax/2688, amax/6
+    block scales) and MXFP8, each T timed as back-to-back calls on one
+    stream (the latency of a call in a stream of calls)."""
+    from mxfp_block_scaled_b200 import mxq, workloads
+    H = HIDDEN
+    sweep, launches = {}, 0
+    clocks = None
+    for T in ACT_T:
+        x = workloads.activation_tile(T, seed=T, device=device)
+        for fmt in ("nvfp4", "mxfp8"):
+            blk = 16 if fmt == "nvfp4" else 32
+            codes = torch.empty((T, H if fmt == "mxfp8" else H // 2), dtype=torch.uint8, device=device)
+            scales = torch.empty((T, H // blk), dtype=torch.uint8, device=device)
+            isc = torch.empty(1, dtype=torch.float32, device=device)
+            st = torch.zeros(1, dtype=torch.int32, device=device)
+            ws, _ = mxq._workspace("quantize_act", T, H, 0, device)
+
+            def call(x=x, fmt=fmt, codes=codes, scales=scales, isc=isc, st=st, ws=ws, T=T):
+                mxq.mxq_quantize_act(x, T, H, fmt, "rtn", "linear", codes, scales, isc, st, ws)
+
+            reps = 2000 if T <= 256 else (400 if T <= 4096 else 50)
+            us, clk = time_loop(call, reps, max(args.warmup, 3))
+            us_graph = time_graph(call, reps)
+            if int(st.item()) != 0:
+                raise RuntimeError("device status %#x (T=%d, %s)" % (int(st.item()), T, fmt))
+            best = min(us, us_graph) if us_graph is not None else us
+            sweep["%s_T%d" % (fmt, T)] = {"us_per_call": us, "us_per_call_graph": us_graph,
+                                          "gbs": T * H * ACT_BYTES[fmt] / (best * 1e-6) / 1e9}
+            launches += reps
+            if T == ACT_T[-1] and fmt == "nvfp4":
+                clocks = clk
+        del x
+    peak, peak_kind = measured_peak()
+    top = sweep["nvfp4_T%d" % ACT_T[-1]]
+    n_top = ACT_T[-1] * H
+    result = {
+        "metric": "dynamic activation quantization GB/s, NVFP4 at T=65536 (1 GPU)",
+        "value": top["gbs"], "unit": "GB/s", "n_gpus": 1, "steps": 1, "warmup": max(args.warmup, 3),
+        "ms_per_step": n_top * ACT_BYTES["nvfp4"] / (top["gbs"] * 1e9) * 1e3, "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": "token tiles bf16 [T,2048], T in {1,16,256,4096,65536}, N(0,1) with "
+                               "channels 101/717/1333/1949 x30; NVFP4 (RTN block scales, "
+                               "input_scale = amax/2688) and MXFP8",
+                   "algorithmic_bytes_per_element": ACT_BYTES,
+                   "l2": "T=65536 tile 268 MB, larger than L2; smaller tiles are L2-resident by design",
+                   "sweep": sweep, "peak_gbs": peak, "peak_kind": peak_kind},
+        "roofline": {"bound": "hbm", "achieved": top["gbs"], "peak": peak, "unit": "GB/s",
+                     "frac": top["gbs"] / peak, "traffic": None,
+                     "kernel": "mxq_quantize_act NVFP4 at T=65536 (group_amax_kernel + nvfp4_quant_kernel: "
+                               "the tile is read twice, so the ceiling is 2.5625/4.5625 of the peak)",
+                     "algorithmic_bytes_per_launch": n_top * ACT_BYTES["nvfp4"], "peak_kind": peak_kind},
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    if not args.no_extras:
+        import oracle
+        oracle.build()
+        x = workloads.activation_tile(4096, seed=4096, device="cpu")
+        xb = workloads.bf16_bits(x).reshape(1, 4096, H)
+        n_el, t = 0, 0.0
+        while t < args.cpu_budget / 2:
+            t0 = time.perf_counter()
+            oracle.quantize_nvfp4(xb, mode=0)
+            t += time.perf_counter() - t0
+            n_el += xb.size
+        result["cpu_baseline"] = {"value": n_el * ACT_BYTES["nvfp4"] / t / 1e9, "unit": "GB/s", "cores": 1,
+                                  "kind": "oracle",
+                                  "sample": "the T=4096 tile, NVFP4 quantize repeated for %.1f s "
+                                            "single-threaded C" % t,
+                                  "elements_per_s": n_el / t}
+    return result
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -482,9 +771,12 @@ def main():
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the e2e and CPU-baseline legs (profiling runs)")
     ap.add_argument("--workload", default="nvfp4_layer",
-                    choices=["nvfp4_layer", "fp8_requant", "nvfp4_weighted"],
+                    choices=["nvfp4_layer", "fp8_requant", "nvfp4_weighted", "mxfp8_shared",
+                             "mxfp4_layer", "act_sweep"],
                     help="nvfp4_layer: the headline quantize + verify step; fp8_requant: block-FP8 "
-                         "-> MXFP4 requantization of the same layer")
+                         "-> MXFP4 requantization of the same layer; nvfp4_weighted: weighted-SSE "
+                         "scale search; mxfp8_shared / mxfp4_layer: MX quantize + verify; act_sweep: "
+                         "dynamic activation quantization over T")
     ap.add_argument("--experts", type=int, default=EXPERTS,
                     help="experts in the layer; fewer than 512 only for small profiling captures")
     args = ap.parse_args()
@@ -516,6 +808,12 @@ def main():
         if world > 1:
             raise SystemExit("--workload nvfp4_weighted runs on one GPU")
         print(json.dumps(run_weighted(args, device)), flush=True)
+        return 0
+    if args.workload in ("mxfp8_shared", "mxfp4_layer", "act_sweep"):
+        if world > 1:
+            raise SystemExit("--workload %s runs on one GPU" % args.workload)
+        run = run_act if args.workload == "act_sweep" else run_mx
+        print(json.dumps(run(args, device)), flush=True)
         return 0
 
     layer = Layer(seed=rank, device=device, experts=args.experts)

@@ -151,18 +151,41 @@ mxq_status mxq_quantize_nvfp4(const uint16_t *x, int64_t n_groups, int64_t rows,
     uint32_t *amax_bits = static_cast<uint32_t *>(workspace);
     unsigned long long *slots = reinterpret_cast<unsigned long long *>(
         static_cast<uint8_t *>(workspace) + nvfp4_slots_offset(n_groups));
+    cudaError_t e = cudaSuccess;
+    // one small group (an activation tile): one thread-block cluster, no
+    // workspace traffic
+    if (n_groups == 1 && nb <= kSmallMaxBlocks) {
+        if (swz)
+            e = zero_tiled_padding(scales, n_groups, rows, cols / 16, stream);
+        if (e == cudaSuccess && m4_count)
+            e = cudaMemsetAsync(m4_count, 0, sizeof(uint32_t), stream);
+        if (e != cudaSuccess)
+            return MXQ_ERR_CUDA;
+        e = launch_nvfp4_small(x, nb, mode == MXQ_SCALE_FOUR_SIX, codes, scales, sl, s2, mbits, m4_count,
+                               status, stream);
+        if (e == cudaSuccess)
+            return MXQ_OK;
+        if (e != cudaErrorNotSupported)
+            return MXQ_ERR_CUDA;
+        (void)cudaGetLastError();
+    }
     // amax bits / arrival counts and amax slots start at zero (a slot's tag
     // is its group + 1)
-    cudaError_t e = cudaMemsetAsync(workspace, 0, need, stream);
+    e = cudaMemsetAsync(workspace, 0, need, stream);
     if (e == cudaSuccess && swz)
         e = zero_tiled_padding(scales, n_groups, rows, cols / 16, stream);
     if (e == cudaSuccess && m4_count)
         e = cudaMemsetAsync(m4_count, 0, (size_t)n_groups * sizeof(uint32_t), stream);
     if (e != cudaSuccess)
         return MXQ_ERR_CUDA;
-    // single pass (one HBM read of x) when the shape allows it
-    e = launch_nvfp4_fused(x, n_groups, nb, mode == MXQ_SCALE_FOUR_SIX, slots, amax_bits, codes, scales, sl, s2,
-                           mbits, m4_count, status, stream);
+    // single pass (one HBM read of x) when the shape allows it and there
+    // are several groups: a lone group has nothing to overlap its grid-wide
+    // amax with, and two passes over a tile that stays in L2 are faster
+    if (n_groups > 1)
+        e = launch_nvfp4_fused(x, n_groups, nb, mode == MXQ_SCALE_FOUR_SIX, slots, amax_bits, codes, scales, sl,
+                               s2, mbits, m4_count, status, stream);
+    else
+        e = cudaErrorNotSupported;
     if (e == cudaSuccess)
         return MXQ_OK;
     if (e != cudaErrorNotSupported)

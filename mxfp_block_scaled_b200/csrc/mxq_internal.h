@@ -86,6 +86,12 @@ cudaError_t launch_nvfp4_fused(const uint16_t *x, int64_t n_groups, int64_t nb, 
                                const ScaleLayout &sl,
                                float *s2, uint32_t *mbits, uint32_t *m4_count, uint32_t *status,
                                cudaStream_t s);
+// One group of at most kSmallMaxBlocks blocks by one thread-block cluster
+// (cudaErrorNotSupported where the device or the size does not allow it).
+constexpr int64_t kSmallMaxBlocks = 96 * 1024;    // 3 MiB of bf16
+cudaError_t launch_nvfp4_small(const uint16_t *x, int64_t nb, int four_six, uint8_t *codes, uint8_t *scales,
+                               const ScaleLayout &sl, float *s2, uint32_t *mbits, uint32_t *m4_count,
+                               uint32_t *status, cudaStream_t s);
 cudaError_t launch_nvfp4_weighted(const uint16_t *x, int64_t n_groups, int64_t nb, int64_t cols,
                                   const uint32_t *amax_bits, const float *h, int64_t h_stride,
                                   uint8_t *codes, uint8_t *scales, const ScaleLayout &sl, float *s2,

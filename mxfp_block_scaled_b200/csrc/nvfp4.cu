@@ -24,6 +24,8 @@
 // bits) are exact in fp64.  So the decision has no rounding at all.
 //
 // Pipeline: group_amax_kernel (pass 1) -> nvfp4_quant_kernel (pass 2).
+#include <cooperative_groups.h>
+
 #include "mxq_device.cuh"
 #include "mxq_internal.h"
 #include "mxq.h"
@@ -1027,6 +1029,183 @@ cudaError_t launch_nvfp4_quant(const uint16_t *x, int64_t n_groups, int64_t nb, 
         nvfp4_quant_kernel<false><<<grid, kNvThreads, 0, s>>>(xv, n_groups, nb, amax_bits, cv, scales,
                                                               sl, s2, mbits, mbits_atomic, m4_count);
     return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// One small group (an activation tile of up to a few hundred tokens) by one
+// thread-block cluster of P CTAs: each CTA copies its share of the blocks
+// into shared memory while reducing its amax, the cluster combines the P
+// maxima through distributed shared memory, and each CTA quantizes its share
+// from shared memory.  One launch, no grid-wide hand-over and no workspace.
+// Shares are multiples of 32 blocks, so each warp's M bits fill one word.
+// ---------------------------------------------------------------------------
+constexpr int kSmallThreads = 512;
+constexpr int kSmallMaxCtas = 16;
+
+template <bool FOUR_SIX, bool SWZ>
+__global__ void __launch_bounds__(kSmallThreads)
+nvfp4_small_kernel(const uint4 *__restrict__ x, int64_t nb, int64_t share, uint2 *__restrict__ codes,
+                   uint8_t *__restrict__ scales, const ScaleLayout sl, float *__restrict__ s2_out,
+                   uint32_t *__restrict__ mbits, uint32_t *__restrict__ m4_count, uint32_t *__restrict__ status)
+{
+    namespace cg = cooperative_groups;
+    extern __shared__ uint4 tile[];                     // 2 vectors per block of this CTA's share
+    __shared__ uint32_t s_warp[kSmallThreads / 32];
+    __shared__ uint32_t s_amax;                         // this CTA's amax, read by the whole cluster
+    __shared__ GroupConst s_gc;
+    __shared__ uint32_t s_m4;
+    cg::cluster_group cluster = cg::this_cluster();
+    const unsigned rank = cluster.block_rank(), P = cluster.num_blocks();
+    const int64_t b0 = min(nb, (int64_t)rank * share);
+    const int n = (int)(min(nb, b0 + share) - b0);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+
+    // eight loads in flight per thread before any is used: a 64 KB share
+    // arrives in one memory round trip
+    uint32_t m = 0;
+    for (int base = 0; base < 2 * n; base += 8 * kSmallThreads) {
+        uint4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = base + u * kSmallThreads + threadIdx.x;
+            if (i < 2 * n)
+                v[u] = __ldg(x + 2 * b0 + i);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = base + u * kSmallThreads + threadIdx.x;
+            if (i < 2 * n) {
+                tile[i] = v[u];
+                m = absmax_bf16x2(absmax_bf16x2(m, v[u].x), absmax_bf16x2(v[u].y, v[u].z));
+                m = absmax_bf16x2(m, v[u].w);
+            }
+        }
+    }
+    m = __reduce_max_sync(0xFFFFFFFFu, fold_halves(m));
+    if (lane == 0)
+        s_warp[warp] = m;
+    if (threadIdx.x == 0)
+        s_m4 = 0;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t a = 0;
+        for (int w = 0; w < kSmallThreads / 32; ++w)
+            a = max(a, s_warp[w]);
+        s_amax = a;
+    }
+    cluster.sync();                                     // every CTA's s_amax is written
+    if (threadIdx.x == 0) {
+        uint32_t g = 0;
+        for (unsigned r = 0; r < P; ++r)
+            g = max(g, *cluster.map_shared_rank(&s_amax, r));
+        s_gc = make_group_const(g);
+        if (rank == 0) {
+            s2_out[0] = s_gc.s2;
+            if (g >= 0x7F80u)
+                atomicOr(status, MXQ_DEV_NONFINITE_INPUT);
+        }
+    }
+    cluster.sync();                                     // remote reads done; s_gc set
+    const GroupConst gc = s_gc;
+    uint32_t my_m4 = 0;
+    for (int base = 0; base < n; base += kSmallThreads) {
+        const int j = base + threadIdx.x;
+        const bool live = j < n;
+        BlockOut o;
+        o.m4 = false;
+        if (live) {
+            o = quantize_block<FOUR_SIX>(tile[2 * j], tile[2 * j + 1], gc);
+            const int64_t b = b0 + j;
+            codes[b] = o.codes;
+            scales[SWZ ? tiled_scale_offset(sl, 0, (uint32_t)b) : (uint64_t)b] = (uint8_t)o.scale;
+        }
+        if (mbits) {
+            const uint32_t word = __ballot_sync(0xFFFFFFFFu, o.m4);
+            const int64_t first = b0 + base + 32 * warp;   // first block of this warp's word
+            if (lane == 0 && first < b0 + n)
+                mbits[first >> 5] = word;
+        }
+        my_m4 += o.m4 ? 1u : 0u;
+    }
+    if (FOUR_SIX && m4_count) {
+        const uint32_t wsum = __reduce_add_sync(0xFFFFFFFFu, my_m4);
+        if (lane == 0 && wsum)
+            atomicAdd(&s_m4, wsum);
+        __syncthreads();
+        if (threadIdx.x == 0 && s_m4)
+            atomicAdd(m4_count, s_m4);
+    }
+}
+
+cudaError_t launch_nvfp4_small(const uint16_t *x, int64_t nb, int four_six, uint8_t *codes, uint8_t *scales,
+                               const ScaleLayout &sl, float *s2, uint32_t *mbits, uint32_t *m4_count,
+                               uint32_t *status, cudaStream_t s)
+{
+    if (nb <= 0 || nb > kSmallMaxBlocks)
+        return cudaErrorNotSupported;
+    int dev = 0, cluster_ok = 0, max_optin = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&cluster_ok, cudaDevAttrClusterLaunch, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+        !cluster_ok)
+        return cudaErrorNotSupported;
+    // about 16 KB of the tile per CTA (up to 16 CTAs), shares a multiple of
+    // 32 blocks
+    int P = (int)((nb * 32 + 16383) / 16384);
+    P = P < 1 ? 1 : (P > kSmallMaxCtas ? kSmallMaxCtas : P);
+    int64_t share = (nb + P - 1) / P;
+    share = (share + 31) / 32 * 32;
+    P = (int)((nb + share - 1) / share);
+    const size_t dyn = (size_t)share * 32;
+    if (dyn + 4096 > (size_t)max_optin)
+        return cudaErrorNotSupported;
+    const void *fn = four_six ? (sl.swz ? (const void *)nvfp4_small_kernel<true, true>
+                                        : (const void *)nvfp4_small_kernel<true, false>)
+                              : (sl.swz ? (const void *)nvfp4_small_kernel<false, true>
+                                        : (const void *)nvfp4_small_kernel<false, false>);
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
+    if (e == cudaSuccess && P > 8)
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        return cudaErrorNotSupported;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)P);
+    cfg.blockDim = dim3(kSmallThreads);
+    cfg.dynamicSmemBytes = dyn;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)P;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&clusters, fn, &cfg);
+    if (e != cudaSuccess || clusters < 1) {
+        (void)cudaGetLastError();
+        return cudaErrorNotSupported;
+    }
+    const uint4 *xv = reinterpret_cast<const uint4 *>(x);
+    uint2 *cv = reinterpret_cast<uint2 *>(codes);
+    if (four_six) {
+        if (sl.swz)
+            e = cudaLaunchKernelEx(&cfg, nvfp4_small_kernel<true, true>, xv, nb, share, cv, scales, sl, s2, mbits,
+                                   m4_count, status);
+        else
+            e = cudaLaunchKernelEx(&cfg, nvfp4_small_kernel<true, false>, xv, nb, share, cv, scales, sl, s2, mbits,
+                                   m4_count, status);
+    } else {
+        if (sl.swz)
+            e = cudaLaunchKernelEx(&cfg, nvfp4_small_kernel<false, true>, xv, nb, share, cv, scales, sl, s2,
+                                   mbits, m4_count, status);
+        else
+            e = cudaLaunchKernelEx(&cfg, nvfp4_small_kernel<false, false>, xv, nb, share, cv, scales, sl, s2,
+                                   mbits, m4_count, status);
+    }
+    return e;
 }
 
 } // namespace mxq
