@@ -908,6 +908,72 @@ __device__ __forceinline__ double block_wsse(const double (&xd)[16], const doubl
     return acc;
 }
 
+// The same objective in fp32 pairs, for the filter below:
+// W32 = sum h (x - RN32(qD s2))^2 with one rounding per operation.
+__device__ __forceinline__ float block_wsse32(const float2 (&xf)[8], const float2 (&h2)[8], uint2 c, float D,
+                                              float s2)
+{
+    uint32_t q[8];
+    e2m1x8_to_f16x2(c.x, *reinterpret_cast<uint32_t(*)[4]>(&q[0]));
+    e2m1x8_to_f16x2(c.y, *reinterpret_cast<uint32_t(*)[4]>(&q[4]));
+    const float2 D2 = make_float2(D, D), S2 = make_float2(s2, s2);
+    float2 acc = make_float2(0.0f, 0.0f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const float2 deq = __fmul2_rn(__fmul2_rn(f16x2_to_float2(q[j]), D2), S2);
+        const float2 e = __fadd2_rn(xf[j], make_float2(-deq.x, -deq.y));
+        acc = __ffma2_rn(h2[j], __fmul2_rn(e, e), acc);
+    }
+    return __fadd_rn(acc.x, acc.y);
+}
+
+// Error bound of W32 against the exact weighted error W, and against the
+// binary64 value the definition forms.  With u = 2^-24, A = sum h x^2 and
+// Cauchy-Schwarz on sum h |x| |e|, the rounding of deq and e costs at most
+// 2u (sqrt(A W) + 2 W) + O(u^2 A), the products and the eight-step pair
+// sums at most 10u W32; bounding W by W32 the same way gives
+// |W32 - W| <= 2.1u sqrt(A W32) + 14.7u W32 + 4.2u^2 A.  The constants
+// below take about twice that, which also covers the binary64 procedure's
+// own error (below 2^-48 W) and the error of forming the bound in fp32.
+// The last term covers terms that underflow, with every weight <= 2^40 and
+// s2 in [2^-50, 2^50] (every non-zero dequantized value normal).
+__device__ __forceinline__ float wsse_bound(float W, float sqrtA_scaled, float c_block)
+{
+    float r;
+    asm("sqrt.approx.f32 %0, %1;" : "=f"(r) : "f"(W));
+    return __fmaf_rn(sqrtA_scaled, r, __fmaf_rn(0x1p-19f, W, c_block));
+}
+
+// The binary64 search of the definition, for blocks the fp32 filter leaves
+// undecided (kept out of line: its doubles stay off the common path).
+__device__ __noinline__ void weighted_search_exact(const uint32_t (&w)[8], const float (&hh)[16], uint32_t lo,
+                                                   uint32_t hi, const GroupConst gc, uint32_t &best_sc,
+                                                   uint2 &best_c)
+{
+    float2 xf[8];
+    unpack_x(w, xf);
+    double xd[16], hd[16];                              // converted once, used by every candidate
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        xd[2 * k] = (double)xf[k].x;
+        xd[2 * k + 1] = (double)xf[k].y;
+    }
+#pragma unroll
+    for (int k = 0; k < 16; ++k)
+        hd[k] = (double)hh[k];
+    double best_w = 0.0;
+    for (uint32_t sc = lo; sc <= hi; ++sc) {
+        const float D = f16x2_to_float2(e4m3x2_to_f16x2(sc)).x;
+        const Plan p = make_plan_any(xf, __fmul_rn(D, gc.s2));
+        const double wv = block_wsse(xd, hd, p.codes, D, (double)gc.s2);
+        if (sc == lo || wv < best_w) {
+            best_w = wv;
+            best_sc = sc;
+            best_c = p.codes;
+        }
+    }
+}
+
 __global__ void __launch_bounds__(kNvThreads)
 nvfp4_weighted_kernel(const uint4 *__restrict__ x, int64_t n_groups, int64_t nb,
                       const uint32_t *__restrict__ amax_bits, const float *__restrict__ h,
@@ -947,17 +1013,17 @@ nvfp4_weighted_kernel(const uint4 *__restrict__ x, int64_t n_groups, int64_t nb,
                 bad_h = bad_h || !(hh[k] >= 0.0f && hh[k] <= 3.402823466e38f);
             if (bad_h)
                 atomicOr(status, MXQ_DEV_NONFINITE_INPUT);
-            float2 xf[8];
+            float2 xf[8], h2[8];
             unpack_x(w, xf);
-            double xd[16], hd[16];                      // converted once, used by every candidate
+            float2 a2 = make_float2(0.0f, 0.0f);
+            float hmax = 0.0f;
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
-                xd[2 * k] = (double)xf[k].x;
-                xd[2 * k + 1] = (double)xf[k].y;
+                h2[k] = make_float2(hh[2 * k], hh[2 * k + 1]);
+                a2 = __ffma2_rn(h2[k], __fmul2_rn(xf[k], xf[k]), a2);
+                hmax = fmaxf(hmax, fmaxf(h2[k].x, h2[k].y));
             }
-#pragma unroll
-            for (int k = 0; k < 16; ++k)
-                hd[k] = (double)hh[k];
+            const float A = __fadd_rn(a2.x, a2.y);
             uint32_t lo = 0, hi = 0;
             if (gc.s2 > 0.0f) {
                 float t6, t4;
@@ -972,20 +1038,37 @@ nvfp4_weighted_kernel(const uint4 *__restrict__ x, int64_t n_groups, int64_t nb,
                 lo = sb & 0xFFu;
                 hi = sb >> 8;
             }
+            // fp32 filter: the fp32 argmin is the binary64 argmin when it beats
+            // every other candidate by more than both error bounds
             uint32_t best_sc = lo;
             uint2 best_c = make_uint2(0u, 0u);
-            double best_w = 0.0;
-            for (uint32_t sc = lo; sc <= hi; ++sc) {
-                const float D = f16x2_to_float2(e4m3x2_to_f16x2(sc)).x;
-                const float d = __fmul_rn(D, gc.s2);
-                const Plan p = make_plan_any(xf, d);
-                const double wv = block_wsse(xd, hd, p.codes, D, (double)gc.s2);
-                if (sc == lo || wv < best_w) {
-                    best_w = wv;
-                    best_sc = sc;
-                    best_c = p.codes;
+            bool decided = gc.qfast && !bad_h && hmax <= 0x1p40f && A >= 0x1p-60f && A <= 0x1p100f;
+            if (decided) {
+                float sa;
+                asm("sqrt.approx.f32 %0, %1;" : "=f"(sa) : "f"(A));
+                const float sqrtA_scaled = 0x1p-22f * sa;
+                const float c_block = __fmaf_rn(0x1p-45f, A, 0x1p-100f);
+                float bw = 0.0f, be = 0.0f, lb = __int_as_float(0x7F800000);   // lb: min (W - eps) of the others
+                for (uint32_t sc = lo; sc <= hi; ++sc) {
+                    const float D = f16x2_to_float2(e4m3x2_to_f16x2(sc)).x;
+                    const Plan p = make_plan_any(xf, __fmul_rn(D, gc.s2));
+                    const float wv = block_wsse32(xf, h2, p.codes, D, gc.s2);
+                    const float ev = wsse_bound(wv, sqrtA_scaled, c_block);
+                    if (sc == lo || wv < bw) {
+                        if (sc != lo)
+                            lb = fminf(lb, __fsub_rn(bw, be));
+                        bw = wv;
+                        be = ev;
+                        best_sc = sc;
+                        best_c = p.codes;
+                    } else {
+                        lb = fminf(lb, __fsub_rn(wv, ev));
+                    }
                 }
+                decided = lb > __fadd_rn(bw, be);
             }
+            if (!decided)
+                weighted_search_exact(w, hh, lo, hi, gc, best_sc, best_c);
             codes[g * nb + b] = best_c;
             scales[sl.swz ? tiled_scale_offset(sl, (uint64_t)g, (uint32_t)b) : (uint64_t)(g * nb + b)] =
                 (uint8_t)best_sc;

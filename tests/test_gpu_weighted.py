@@ -77,3 +77,35 @@ def test_bad_weight_sets_status():
     out = mxq.quantize_nvfp4_weighted(x, h.cuda())
     torch.cuda.synchronize()
     assert int(out["status"].item()) & mxq.DEV_NONFINITE_INPUT
+
+
+def _grid_blocks(seed, nblocks):
+    """Blocks on grids several candidate scales represent exactly (ties of
+    the weighted error), mixed with random blocks; group amax 2.625 makes
+    s2 = 2^-10 exactly."""
+    rng = np.random.default_rng(seed)
+    x = np.zeros((nblocks, 16), np.float32)
+    for b in range(nblocks):
+        base = np.float32(2.0 ** -10 * rng.choice([2.0, 4.0, 8.0, 16.0]))
+        if b % 3 == 2:
+            x[b] = rng.standard_normal(16) * 0.2
+        else:
+            x[b] = rng.choice([0.0, 1.0, 2.0, 3.0, -1.0, -2.0, -4.0], 16) * base
+            x[b, 0] = 4.0 * base
+    x[0] = 0.0
+    x[0, 0] = 2.625
+    return torch.from_numpy(x.reshape(1, nblocks, 16)).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("kind", ["zero", "one_hot", "huge", "gamma"])
+def test_ties_and_unfiltered_weights_take_the_binary64_search(kind):
+    """Exact ties (all-zero weights: every candidate scores 0; one-hot
+    weights on grid blocks), weights beyond the fp32 filter's range and plain
+    weights on tie-rich blocks must all give the binary64 choice (ties to
+    the smaller code), bit-exact with the oracle."""
+    x = _grid_blocks(7, 96)
+    h = {"zero": torch.zeros(16),
+         "one_hot": torch.nn.functional.one_hot(torch.tensor(3), 16).float(),
+         "huge": torch.full((16,), 2.0 ** 60),
+         "gamma": torch.distributions.Gamma(torch.tensor(0.5), torch.tensor(1.0)).sample((16,))}[kind]
+    _check(x.cuda(), h.float().contiguous())
