@@ -242,6 +242,38 @@ def run_cpu_baseline(layer, budget_s=20.0):
             "elements_per_s": n_el / t_total}
 
 
+def run_cpu_parallel(layer, per_thread=3):
+    """The same oracle on every host core: one thread per core (the C calls
+    release the interpreter lock), each converting whole experts of the
+    layer (quantize + verify), `per_thread` experts per thread, at most 512."""
+    import concurrent.futures as cf
+    import oracle
+    from mxfp_block_scaled_b200 import workloads
+    oracle.build()
+    oracle.lib()                                        # load once, before the threads start
+    n = min(os.cpu_count() or 1, 128)
+    experts = min(EXPERTS, n * per_thread)
+    work = [(workloads.bf16_bits(layer.gu[e:e + 1]), workloads.bf16_bits(layer.dn[e:e + 1]))
+            for e in range(experts)]
+
+    def one(item):
+        gu, dn = item
+        c, s, s2, _ = oracle.quantize_nvfp4(gu, mode=1)
+        oracle.dequant_relerr(gu, c, s, s2, "nvfp4", 2, INTER, HIDDEN, 2)
+        c, s, s2, _ = oracle.quantize_nvfp4(dn, mode=1)
+        oracle.dequant_relerr(dn, c, s, s2, "nvfp4", 1, HIDDEN, INTER, 1)
+        return gu.size + dn.size
+
+    with cf.ThreadPoolExecutor(max_workers=n) as ex:
+        t0 = time.perf_counter()
+        n_el = sum(ex.map(one, work))
+        t = time.perf_counter() - t0
+    return {"value": n_el * STEP_BYTES_PER_ELEM / t / 1e9, "unit": "GB/s", "cores": n, "kind": "oracle",
+            "sample": "%d of %d experts (gate_up + down, %.1fM elements), quantize + verify, %.1f s "
+                      "on %d threads" % (experts, EXPERTS, n_el / 1e6, t, n),
+            "elements_per_s": n_el / t}
+
+
 def run_e2e(layer, steps, device, chunk=64):
     """Same metric through the public Python API with host buffers: every step
     copies the layer from pinned host memory, quantizes and verifies it, and
@@ -887,6 +919,7 @@ def main():
     if rank == 0 and world == 1 and not args.no_extras:
         result["e2e"] = run_e2e(layer, args.e2e_steps, device)
         result["cpu_baseline"] = run_cpu_baseline(layer, args.cpu_budget)
+        result["cpu_baseline_all_cores"] = run_cpu_parallel(layer)
     elif rank == 0:
         result["e2e"] = None
     if rank == 0:
