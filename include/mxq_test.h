@@ -1,0 +1,29 @@
+/* mxq_test.h -- test-only hooks of libmxq.so.  Not part of the conversion
+ * API (include/mxq.h); they exist so that tests can show, without faulting
+ * or hanging the GPU, that the library's failure paths answer as specified.
+ */
+#ifndef MXQ_TEST_H
+#define MXQ_TEST_H
+
+#include "mxq.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Make the next single-pass NVFP4 launch (mxq_quantize_nvfp4 on several
+ * groups whose shape the single-pass kernel holds) stall on purpose: its
+ * per-SM publisher never releases a group, so every inter-CTA wait of that
+ * launch runs into its iteration limit.  The launch then ORs
+ * MXQ_DEV_WAIT_TIMEOUT into *status, lets its copies in flight land and
+ * returns, well under a second; the outputs of that call are undefined and
+ * the device stays usable.  `on` = 0 withdraws a pending request.  The
+ * request is taken by exactly one launch (the next one of any thread of the
+ * process); it is ignored by the other kernels. */
+MXQ_API void mxq_test_stall_next_single_pass(int on);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MXQ_TEST_H */

@@ -27,7 +27,7 @@ NVCC_FLAGS = [
 
 def _inputs():
     files = [os.path.join(CSRC, s) for s in SOURCES + HEADERS]
-    files.append(os.path.join(INCLUDE, "mxq.h"))
+    files += [os.path.join(INCLUDE, f) for f in ("mxq.h", "mxq_test.h")]
     return files
 
 

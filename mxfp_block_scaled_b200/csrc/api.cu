@@ -5,6 +5,7 @@
 #include "mxq_internal.h"
 
 #include <limits.h>
+#include <nvtx3/nvToolsExt.h>
 
 namespace mxq {
 
@@ -53,6 +54,15 @@ static bool mul_ok(int64_t a, int64_t b, int64_t *out)
     *out = a * b;
     return true;
 }
+
+// NVTX range around one API call (visible in Nsight timelines; a no-op
+// without a tool attached).
+struct ApiRange {
+    explicit ApiRange(const char *name) { nvtxRangePushA(name); }
+    ~ApiRange() { nvtxRangePop(); }
+    ApiRange(const ApiRange &) = delete;
+    ApiRange &operator=(const ApiRange &) = delete;
+};
 
 } // namespace mxq
 
@@ -119,6 +129,7 @@ mxq_status mxq_quantize_nvfp4(const uint16_t *x, int64_t n_groups, int64_t rows,
                               uint32_t *mbits, uint32_t *m4_count, uint32_t *status,
                               void *workspace, size_t workspace_bytes, cudaStream_t stream)
 {
+    const ApiRange range_("mxq_quantize_nvfp4");
     if (n_groups < 0 || rows < 0 || cols < 0)
         return MXQ_ERR_INVALID_ARG;
     if (mode != MXQ_SCALE_RTN && mode != MXQ_SCALE_FOUR_SIX)
@@ -212,6 +223,7 @@ mxq_status mxq_quantize_nvfp4_weighted(const uint16_t *x, int64_t n_groups, int6
                                        uint32_t *status, void *workspace, size_t workspace_bytes,
                                        cudaStream_t stream)
 {
+    const ApiRange range_("mxq_quantize_nvfp4_weighted");
     if (n_groups < 0 || rows < 0 || cols < 0)
         return MXQ_ERR_INVALID_ARG;
     if (!layout_ok(layout) || (h_groups != 1 && h_groups != n_groups))
@@ -254,6 +266,7 @@ mxq_status mxq_quantize_mx(const uint16_t *x, int64_t rows, int64_t cols, mxq_fm
                            mxq_layout layout, uint8_t *codes, uint8_t *scales, uint32_t *status,
                            cudaStream_t stream)
 {
+    const ApiRange range_("mxq_quantize_mx");
     if (rows < 0 || cols < 0)
         return MXQ_ERR_INVALID_ARG;
     if (fmt != MXQ_FMT_MXFP4 && fmt != MXQ_FMT_MXFP8)
@@ -287,6 +300,7 @@ mxq_status mxq_requant_fp8_mx(const uint8_t *fp8, const float *bscale, int64_t r
                               int64_t brows, int64_t bcols, mxq_fmt fmt, mxq_layout layout,
                               uint8_t *codes, uint8_t *scales, uint32_t *status, cudaStream_t stream)
 {
+    const ApiRange range_("mxq_requant_fp8_mx");
     if (rows < 0 || cols < 0 || brows < 1 || bcols < 1)
         return MXQ_ERR_INVALID_ARG;
     if (fmt != MXQ_FMT_MXFP4 && fmt != MXQ_FMT_MXFP8)
@@ -319,6 +333,7 @@ mxq_status mxq_quantize_act(const uint16_t *tokens, int64_t T, int64_t hidden, m
                             uint8_t *scales, float *input_scale, uint32_t *status,
                             void *workspace, size_t workspace_bytes, cudaStream_t stream)
 {
+    const ApiRange range_("mxq_quantize_act");
     if (T < 0 || hidden < 0)
         return MXQ_ERR_INVALID_ARG;
     if (mode != MXQ_SCALE_RTN && mode != MXQ_SCALE_FOUR_SIX)
@@ -354,6 +369,7 @@ mxq_status mxq_dequant_relerr(const uint16_t *x, const uint8_t *codes, const uin
                               double *sum_sq_ref, double *relerr, void *workspace,
                               size_t workspace_bytes, cudaStream_t stream)
 {
+    const ApiRange range_("mxq_dequant_relerr");
     if (n_tensors < 0 || rows < 0 || cols < 0)
         return MXQ_ERR_INVALID_ARG;
     if (fmt != MXQ_FMT_NVFP4 && fmt != MXQ_FMT_MXFP4 && fmt != MXQ_FMT_MXFP8)

@@ -24,11 +24,14 @@
 // bits) are exact in fp64.  So the decision has no rounding at all.
 //
 // Pipeline: group_amax_kernel (pass 1) -> nvfp4_quant_kernel (pass 2).
+#include <atomic>
+
 #include <cooperative_groups.h>
 
 #include "mxq_device.cuh"
 #include "mxq_internal.h"
 #include "mxq.h"
+#include "mxq_test.h"
 
 namespace mxq {
 
@@ -421,6 +424,7 @@ struct FusedArgs {
     ScaleLayout sl;
     float *s2_out;
     uint32_t *mbits, *m4_count;
+    int test_stall;                // test hook: the publisher releases no group
 };
 
 constexpr uint32_t kSpinLimit = 1u << 22;   // polls of a flag / barrier before giving up
@@ -514,7 +518,7 @@ nvfp4_fused_kernel(const FusedArgs a)
         uint32_t idle = 0;
         while (next_ready < G) {
             bool progress = false;
-            const int npoll = min(kPollGroups, *scouted - next_ready);
+            const int npoll = a.test_stall ? 0 : min(kPollGroups, *scouted - next_ready);
             if (npoll > 0) {
                 uint32_t cnt = 0;
                 if (lane < npoll)
@@ -777,6 +781,10 @@ cudaError_t launch_group_amax(const uint16_t *x, int64_t n_groups, int64_t nb,
     return cudaGetLastError();
 }
 
+// Test hook (include/mxq_test.h): the next single-pass launch stalls on
+// purpose and must end with MXQ_DEV_WAIT_TIMEOUT.
+static std::atomic<int> g_test_stall{0};
+
 static int sm_count()
 {
     int dev = 0, n = 0;
@@ -872,6 +880,7 @@ cudaError_t launch_nvfp4_fused(const uint16_t *x, int64_t n_groups, int64_t nb, 
     args.s2_out = s2;
     args.mbits = mbits;
     args.m4_count = four_six ? m4_count : nullptr;
+    args.test_stall = g_test_stall.exchange(0) ? 1 : 0;
     void *params[] = {&args};
     return cudaLaunchCooperativeKernel(fn, dim3((unsigned)sms), dim3(kFusedThreads), params, dyn, s);
 }
@@ -1292,3 +1301,8 @@ cudaError_t launch_nvfp4_small(const uint16_t *x, int64_t nb, int four_six, uint
 }
 
 } // namespace mxq
+
+extern "C" MXQ_API void mxq_test_stall_next_single_pass(int on)
+{
+    mxq::g_test_stall.store(on ? 1 : 0);
+}

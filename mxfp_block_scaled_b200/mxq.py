@@ -78,6 +78,8 @@ def load(path=LIB_PATH):
                                      vp]
     L.mxq_dequant_relerr_noalloc.restype = i32
     L.mxq_dequant_relerr_noalloc.argtypes = [vp, vp, vp, vp, i32, i64, i64, i64, i64, vp, vp, vp, vp]
+    L.mxq_test_stall_next_single_pass.restype = None
+    L.mxq_test_stall_next_single_pass.argtypes = [i32]
     if path == LIB_PATH:
         _lib = L
     return L

@@ -1,5 +1,5 @@
-"""The C-ABI library loads and exports every entry point include/mxq.h
-declares; host-side argument checks answer before any CUDA work (these
+"""The C-ABI library loads and exports every entry point the headers under
+include/ declare; host-side argument checks answer before any CUDA work (these
 calls need no GPU)."""
 import ctypes
 import os
@@ -18,9 +18,13 @@ def lib():
 
 
 def declared_functions():
-    with open(os.path.join(ROOT, "include", "mxq.h")) as f:
-        text = f.read()
-    return re.findall(r"MXQ_API\s+[\w\s\*]+?\b(mxq_\w+)\s*\(", text)
+    """Every entry point the headers under include/ declare."""
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            with open(os.path.join(ROOT, "include", h)) as f:
+                names += re.findall(r"MXQ_API\s+[\w\s\*]+?\b(mxq_\w+)\s*\(", f.read())
+    return names
 
 
 def test_header_declares_the_entry_points():
