@@ -47,19 +47,6 @@ __device__ __forceinline__ uint32_t e2m1x2(float lo, float hi)
     return out;
 }
 
-// As e2m1x2, also returning the two decoded values as f16x2 (exact), taken
-// from the same byte register.
-__device__ __forceinline__ uint32_t e2m1x2_enc_dec(float lo, float hi, uint32_t &q)
-{
-    uint32_t out;
-    asm("{\n\t.reg .b8 t;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 t, %3, %2;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %1, t;\n\t"
-        "cvt.u32.u8 %0, t;\n\t}"
-        : "=r"(out), "=r"(q) : "f"(lo), "f"(hi));
-    return out;
-}
-
 // Eight fp32 values (four pairs) -> one word of eight E2M1 codes (pair j in
 // byte j, element 2j in its low nibble) and the four decoded pairs as f16x2,
 // decoded from the same byte registers.  The bytes are only ever packed into
@@ -257,14 +244,6 @@ __device__ __forceinline__ void named_barrier_sync(int id, int count)
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-// Bounded spin for inter-CTA flags: returns false after `limit` polls.
-__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p)
-{
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
 __device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t *p)
 {
     uint32_t v;
@@ -287,11 +266,6 @@ __device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long
 __device__ __forceinline__ void st_relaxed_u64(unsigned long long *p, unsigned long long v)
 {
     asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-
-__device__ __forceinline__ void red_release_add_u32(uint32_t *p, uint32_t v)
-{
-    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
 // ---- shared-memory barriers and bulk copies (PTX ISA, sm_90+) -----------
@@ -353,27 +327,6 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity)
                  "selp.u32 %0, 1, 0, p;\n\t}"
                  : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity) : "memory");
     return ok != 0;
-}
-
-// As mbar_try_wait, letting the hardware suspend the thread for up to about
-// `ns` nanoseconds while the phase is incomplete (fewer polling instructions).
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t ns)
-{
-    uint32_t ok;
-    asm volatile("{\n\t.reg .pred p;\n\t"
-                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-                 "selp.u32 %0, 1, 0, p;\n\t}"
-                 : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity), "r"(ns) : "memory");
-    return ok != 0;
-}
-
-// Wait for phase `parity` of `bar`, giving up after `limit` polls.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, uint32_t limit)
-{
-    for (uint32_t i = 0; i < limit; ++i)
-        if (mbar_try_wait(bar, parity))
-            return true;
-    return false;
 }
 
 } // namespace mxq

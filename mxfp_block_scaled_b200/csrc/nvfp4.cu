@@ -504,9 +504,6 @@ nvfp4_fused_kernel(const FusedArgs a)
     }
     __syncthreads();
 
-    const unsigned long long *src0 = reinterpret_cast<const unsigned long long *>(a.x);
-    (void)src0;
-
     if (warp == 0) {
         // -------------------------------------------------------- publisher
         // Releases group j to the compute warps once all P CTAs have counted
