@@ -111,6 +111,23 @@ struct RequantArgs {
     uint32_t *status;
 };
 
+// Running max of |v| over f16x2 words, per half (max.NaN.xorsign.abs; the
+// sign bits are dropped by the fold below, NaN propagates).
+__device__ __forceinline__ uint32_t absmax_f16x2(uint32_t acc, uint32_t v)
+{
+    uint32_t r;
+    asm("max.NaN.xorsign.abs.f16x2 %0, %1, %2;" : "=r"(r) : "r"(acc), "r"(v));
+    return r;
+}
+
+// Per MX block of 32: w_i = RN32(q_i * sc) (q_i the E4M3 source value, sc
+// its block scale) is MX-quantized.  Two exact shortcuts:
+//  - max |w_i| = RN32(max |q_i| * |sc|), RN being monotone, so the block
+//    amax comes from the decoded source (one f16x2 max per pair);
+//  - with |sc| in [2^-117, 2^100] every non-zero product q_i sc is a normal
+//    fp32, and with |e| < 127 the scale sc 2^-e is normal, so
+//    RN32(RN32(q_i sc) 2^-e) = RN32(q_i (sc 2^-e)): one multiply per value.
+//    Outside that range the two roundings are kept.
 template <int FMT>
 __global__ void __launch_bounds__(256) requant_fp8_mx_kernel(const RequantArgs a)
 {
@@ -120,27 +137,36 @@ __global__ void __launch_bounds__(256) requant_fp8_mx_kernel(const RequantArgs a
         const uint4 v0 = __ldg(a.fp8 + 2 * bb), v1 = __ldg(a.fp8 + 2 * bb + 1);
         const uint32_t r = fastdiv(b, a.cbdiv), j = b - r * a.cb;
         const float sc = __ldg(a.bscale + (uint64_t)fastdiv(r, a.browsdiv) * a.nbc + fastdiv(j, a.bcdiv));
-        const float2 sc2 = make_float2(sc, sc);
         const uint32_t w8[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-        float2 w[16];
-        uint32_t m = 0;
+        uint32_t qh[16];                                // the E4M3 values as f16x2 pairs (exact)
+        uint32_t m16 = 0;
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
-            // 4 E4M3 bytes -> two f16x2 pairs (exact) -> fp32, times the scale (one rounding)
-            w[2 * t] = __fmul2_rn(f16x2_to_float2(e4m3x2_to_f16x2(w8[t])), sc2);
-            w[2 * t + 1] = __fmul2_rn(f16x2_to_float2(e4m3x2_to_f16x2(w8[t] >> 16)), sc2);
-            m = max(m, max(__float_as_uint(w[2 * t].x) & 0x7FFFFFFFu, __float_as_uint(w[2 * t].y) & 0x7FFFFFFFu));
-            m = max(m, max(__float_as_uint(w[2 * t + 1].x) & 0x7FFFFFFFu,
-                           __float_as_uint(w[2 * t + 1].y) & 0x7FFFFFFFu));
+            qh[2 * t] = e4m3x2_to_f16x2(w8[t]);
+            qh[2 * t + 1] = e4m3x2_to_f16x2(w8[t] >> 16);
+            m16 = absmax_f16x2(absmax_f16x2(m16, qh[2 * t]), qh[2 * t + 1]);
         }
-        if (m >= 0x7F800000u && a.status)
+        const uint32_t mq = max(m16 & 0x7FFFu, (m16 >> 16) & 0x7FFFu);
+        const float asc = fabsf(sc);
+        const uint32_t m = __float_as_uint(__fmul_rn(__half2float(__ushort_as_half((unsigned short)mq)), asc));
+        if (m >= 0x7F800000u && a.status)               // Inf / NaN source value or scale
             atomicOr(a.status, MXQ_DEV_NONFINITE_INPUT);
         const int e = mx_exponent_f32<FMT>(m);
-        const float s = e == 127 ? 0x1p-127f : __uint_as_float((uint32_t)(127 - e) << 23);   // 2^-e
-        const float2 s2 = make_float2(s, s);
+        float2 w[16];
+        if (asc >= 0x1p-117f && asc <= 0x1p100f && e > -127 && e < 127) {
+            const float sce = __fmul_rn(sc, __uint_as_float((uint32_t)(127 - e) << 23));   // exact
+            const float2 s2 = make_float2(sce, sce);
 #pragma unroll
-        for (int t = 0; t < 16; ++t)
-            w[t] = __fmul2_rn(w[t], s2);                // exact (a power of two)
+            for (int t = 0; t < 16; ++t)
+                w[t] = __fmul2_rn(f16x2_to_float2(qh[t]), s2);
+        } else {
+            const float2 sc2 = make_float2(sc, sc);
+            const float s = e == 127 ? 0x1p-127f : __uint_as_float((uint32_t)(127 - e) << 23);   // 2^-e
+            const float2 s2 = make_float2(s, s);
+#pragma unroll
+            for (int t = 0; t < 16; ++t)
+                w[t] = __fmul2_rn(__fmul2_rn(f16x2_to_float2(qh[t]), sc2), s2);
+        }
         a.scales[a.sl.swz ? tiled_scale_offset(a.sl, 0, b) : (uint64_t)b] = (uint8_t)(e + 127);
         if (FMT == MXQ_FMT_MXFP8) {
             uint32_t o[8];

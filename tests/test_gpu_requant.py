@@ -51,3 +51,27 @@ def test_requant_nonfinite_source_sets_status():
     out = mxq.requant_fp8_mx(codes.cuda(), scales.cuda(), 128, 128, "mxfp4")
     torch.cuda.synchronize()
     assert int(out["status"].item()) & mxq.DEV_NONFINITE_INPUT
+
+
+@pytest.mark.parametrize("fmt", ["mxfp8", "mxfp4"])
+def test_requant_extreme_block_scales(fmt):
+    """Block scales outside the range where one multiply by sc 2^-e replaces
+    the two roundings (tiny scales whose products go subnormal, huge ones),
+    the range edges, a zero scale (an all-zero block: e = -127) and a
+    negative scale: still bit-exact with the oracle."""
+    codes, scales = workloads.block_fp8_source(256, 512, seed=21)
+    s = scales.clone()
+    s[0, 0] = 2.0 ** -120
+    s[0, 1] = 1e-38
+    s[0, 2] = 2.0 ** 101
+    s[0, 3] = 0.0
+    s[1, 0] = -0.75
+    s[1, 1] = 2.0 ** -117
+    s[1, 2] = 2.0 ** 100
+    s[1, 3] = 2.0 ** -126
+    out = mxq.requant_fp8_mx(codes.cuda(), s.cuda(), 128, 128, fmt)
+    torch.cuda.synchronize()
+    assert int(out["status"].item()) == 0
+    oc, os_ = oracle.requant_fp8_mx(codes.numpy(), s.numpy(), 128, 128, fmt)
+    assert np.array_equal(out["codes"].cpu().numpy(), oc)
+    assert np.array_equal(out["scales"].cpu().numpy(), os_)
