@@ -68,7 +68,7 @@ def measured_peak():
 
 def kernel_source_sha():
     h = hashlib.sha256()
-    for f in ("nvfp4.cu", "mxq_device.cuh"):
+    for f in ("nvfp4.cu", "nvfp4_block.cuh", "mxq_device.cuh"):
         with open(os.path.join(ROOT, "mxfp_block_scaled_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]

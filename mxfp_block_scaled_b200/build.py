@@ -11,8 +11,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libmxq.so")
-SOURCES = ["api.cu", "nvfp4.cu", "mx.cu", "verify.cu", "noalloc.cu"]
-HEADERS = ["mxq_device.cuh", "mxq_internal.h"]
+SOURCES = ["api.cu", "nvfp4.cu", "weighted.cu", "mx.cu", "verify.cu", "noalloc.cu"]
+HEADERS = ["mxq_device.cuh", "mxq_internal.h", "nvfp4_block.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 # No --use_fast_math: denormals are kept and every division / reciprocal
