@@ -421,8 +421,10 @@ def run_requant(args, device):
         "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": "one full-size routed-expert layer as block FP8 (E4M3 + fp32 scale per "
-                               "128x128) -> MXFP4: gate_up [512*1536, 2048] + down [512*2048, 768]",
+        "config": {"workload": ("one full-size routed-expert layer as block FP8 (E4M3 + fp32 scale per "
+                                "128x128) -> MXFP4: gate_up [512*1536, 2048] + down [512*2048, 768]")
+                   if args.experts == EXPERTS else
+                   "PROFILING CASE, %d experts (not the full-size layer)" % args.experts,
                    "elements_per_gpu": n, "algorithmic_bytes_per_element": REQ_BYTES,
                    "l2": "inputs 2.4 GB, larger than L2; no flush",
                    "call_ms": dict(zip(["requant_gate_up", "requant_down"], call_ms))},
@@ -491,9 +493,11 @@ def run_weighted(args, device):
         "metric": "NVFP4 weighted-SSE scale search, quantize HBM GB/s (1 GPU)",
         "value": n * Q_BYTES / (ms * 1e-3) / 1e9, "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "one full-size routed-expert layer, NVFP4 with the weighted-SSE scale "
-                               "search: gate_up bf16 [512,1536,2048] + down [512,2048,768]",
+        "vs_baseline": None, "dtype": "f32+f64", "data": "synthetic",
+        "config": {"workload": ("one full-size routed-expert layer, NVFP4 with the weighted-SSE scale "
+                                "search: gate_up bf16 [512,1536,2048] + down [512,2048,768]")
+                   if args.experts == EXPERTS else
+                   "PROFILING CASE, %d experts (not the full-size layer)" % args.experts,
                    "elements_per_gpu": n, "algorithmic_bytes_per_element": Q_BYTES,
                    "passes": "two (group amax, then the search): W is read twice",
                    "call_ms": dict(zip(["gate_up", "down"], call_ms))},
