@@ -1,0 +1,63 @@
+"""Host-side logic of bench.py that the reported numbers depend on, checked
+without a GPU: the clock-sample summary (median loaded clock, throttle
+reasons of the right GPU only) and the DRAM traffic record (used only while
+the kernel source it was captured from is unchanged)."""
+import os
+
+import bench
+
+
+def _write(tmp_path, lines):
+    p = tmp_path / "clocks.csv"
+    p.write_text("\n".join(lines) + "\n")
+    return str(p)
+
+
+def test_clock_summary_median_and_reasons(tmp_path):
+    rows = [
+        # index, uuid, sm, max, power, active, hw_slowdown, hw_thermal, sw_thermal, sw_power_cap
+        "0, GPU-a, 1965, 1965, 800, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "0, GPU-a, 1950, 1965, 990, 0x4, Not Active, Not Active, Not Active, Active",
+        "0, GPU-a, 1965, 1965, 900, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "0, GPU-a, 300, 1965, 100, 0x0, Not Active, Not Active, Not Active, Not Active",  # idle tail
+        "1, GPU-b, 900, 1965, 400, 0x8, Active, Not Active, Not Active, Not Active",      # other GPU
+    ]
+    s = bench.ClockSampler("GPU-a")
+    s.path = _write(tmp_path, rows)
+    out = s.summary()
+    assert out["sm_max_mhz"] == 1965.0
+    assert out["sm_mhz"] == 1965.0              # median of the loaded samples (> half the max)
+    assert out["reasons"] == ["sw_power_cap"]   # GPU-b's hw_slowdown is not ours
+    assert out["samples"] == 4
+    assert not os.path.exists(s.path)
+
+
+def test_clock_summary_without_samples(tmp_path):
+    s = bench.ClockSampler("GPU-a")
+    s.path = _write(tmp_path, ["garbage"])
+    assert s.summary() is None
+
+
+def test_traffic_record_follows_the_kernel_source(tmp_path, monkeypatch):
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    rec = prof / "nvfp4_quant_gate_up_fullsize_traffic.txt"
+    sha = bench.kernel_source_sha()
+    rec.write_text("# comment\nsource_sha %s\ndram_bytes_per_call 1234\n" % sha)
+    real_join = os.path.join
+
+    def join(*parts):
+        if len(parts) >= 3 and parts[1] == "profiles":
+            return real_join(str(tmp_path), *parts[1:])
+        return real_join(*parts)
+
+    monkeypatch.setattr(bench.os.path, "join", join)
+    assert bench.ncu_traffic_per_launch() == 1234.0
+    rec.write_text("source_sha 0000000000000000\ndram_bytes_per_call 1234\n")
+    assert bench.ncu_traffic_per_launch() is None
+
+
+def test_algorithmic_bytes_per_element():
+    assert bench.Q_BYTES == 2.5625 and bench.STEP_BYTES_PER_ELEM == 5.125
+    assert bench.MX_BYTES == {"mxfp8": 3.03125, "mxfp4": 2.53125}
+    assert bench.ACT_BYTES["nvfp4"] == 2.5625
