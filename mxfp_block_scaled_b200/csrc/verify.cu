@@ -104,8 +104,11 @@ __device__ __forceinline__ void cta_reduce_store(double err, double ref, double 
     __syncthreads();
 }
 
+// Four CTAs per SM (at most 64 registers): the loads a thread issues
+// before its arithmetic are what keeps HBM busy, so occupancy sets the
+// bytes in flight.
 template <int FMT, bool SWZ>
-__global__ void __launch_bounds__(kVerifyThreads)
+__global__ void __launch_bounds__(kVerifyThreads, 4)
 verify_chunk_kernel(const uint16_t *__restrict__ x, const uint8_t *__restrict__ codes,
                     const uint8_t *__restrict__ scales, const float *__restrict__ s2,
                     const ScaleLayout sl, int64_t n_tensors, int64_t rows, int64_t tsize,
