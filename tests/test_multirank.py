@@ -11,8 +11,6 @@ import subprocess
 import sys
 import types
 
-import pytest
-
 from conftest import ROOT
 
 

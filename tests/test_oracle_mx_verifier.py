@@ -15,7 +15,6 @@ from fractions import Fraction as F
 
 import numpy as np
 import pytest
-import torch
 
 from oracle import micro
 from mxfp_block_scaled_b200 import workloads
