@@ -273,12 +273,14 @@ def run_cpu_parallel(layer, per_thread=3):
             "elements_per_s": n_el / t}
 
 
-def run_e2e(layer, steps, device, chunk=64):
+def run_e2e(layer, steps, device, chunk=64, world=1):
     """Same metric through the public Python API with host buffers: every step
     copies the layer from pinned host memory, quantizes and verifies it, and
     copies codes, scales, global scales and per-tensor errors back
     (layers.HostLayerConverter: chunks of `chunk` experts, with the copies in
-    both directions overlapping the kernels of neighbouring chunks)."""
+    both directions overlapping the kernels of neighbouring chunks).  Under
+    torchrun every rank converts its own layer; the step time is the max
+    over ranks and the value counts every rank's elements."""
     from mxfp_block_scaled_b200 import layers
     h_gu = torch.empty(layer.gu.shape, dtype=torch.bfloat16, pin_memory=True)
     h_dn = torch.empty(layer.dn.shape, dtype=torch.bfloat16, pin_memory=True)
@@ -292,6 +294,10 @@ def run_e2e(layer, steps, device, chunk=64):
     torch.cuda.synchronize()
     if conv.status() != 0:
         raise RuntimeError("device status %#x in the e2e leg" % conv.status())
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record()
@@ -299,8 +305,8 @@ def run_e2e(layer, steps, device, chunk=64):
         conv.run(h_gu, h_dn, out)
     t1.record()
     torch.cuda.synchronize()
-    ms = t0.elapsed_time(t1) / steps
-    return {"value": layer.n_elems * STEP_BYTES_PER_ELEM / (ms * 1e-3) / 1e9, "unit": "GB/s",
+    ms = max_over_ranks(t0.elapsed_time(t1) / steps, world, device)
+    return {"value": layer.n_elems * world * STEP_BYTES_PER_ELEM / (ms * 1e-3) / 1e9, "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms,
             "pipeline": "chunks of %d experts, H2D / kernels / D2H on three streams" % chunk}
 
@@ -919,10 +925,13 @@ def main():
         "gpu_launches": args.steps * 2 * (KERNELS_PER_QUANTIZE_NVFP4 + KERNELS_PER_VERIFY),
         "clocks": clk.summary(),
     }
-    if rank == 0 and world == 1 and not args.no_extras:
-        result["e2e"] = run_e2e(layer, args.e2e_steps, device)
-        result["cpu_baseline"] = run_cpu_baseline(layer, args.cpu_budget)
-        result["cpu_baseline_all_cores"] = run_cpu_parallel(layer)
+    if not args.no_extras:
+        e2e = run_e2e(layer, args.e2e_steps, device, world=world)    # every rank: collectives inside
+        if rank == 0:
+            result["e2e"] = e2e
+        if rank == 0 and world == 1:
+            result["cpu_baseline"] = run_cpu_baseline(layer, args.cpu_budget)
+            result["cpu_baseline_all_cores"] = run_cpu_parallel(layer)
     elif rank == 0:
         result["e2e"] = None
     if rank == 0:
