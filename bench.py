@@ -280,32 +280,43 @@ def run_e2e(layer, steps, device, chunk=64, world=1):
     (layers.HostLayerConverter: chunks of `chunk` experts, with the copies in
     both directions overlapping the kernels of neighbouring chunks).  Under
     torchrun every rank converts its own layer; the step time is the max
-    over ranks and the value counts every rank's elements."""
+    over ranks and the value counts every rank's elements.  A rank that
+    cannot set the leg up (e.g. pinned host memory refused) still takes part
+    in the barrier and the reduction, and the leg reports itself unavailable."""
     from mxfp_block_scaled_b200 import layers
-    h_gu = torch.empty(layer.gu.shape, dtype=torch.bfloat16, pin_memory=True)
-    h_dn = torch.empty(layer.dn.shape, dtype=torch.bfloat16, pin_memory=True)
-    h_gu.copy_(layer.gu)
-    h_dn.copy_(layer.dn)
-    out = layers.host_outputs(h_gu, h_dn)
-    h2d = h_gu.numel() * 2 + h_dn.numel() * 2
-    d2h = sum(t.numel() * t.element_size() for o in out.values() for t in o.values())
-    conv = layers.HostLayerConverter(layer.gu.shape, layer.dn.shape, chunk=chunk, device=device)
-    conv.run(h_gu, h_dn, out)
-    torch.cuda.synchronize()
-    if conv.status() != 0:
-        raise RuntimeError("device status %#x in the e2e leg" % conv.status())
+    failed, h2d, d2h = None, 0, 0
+    try:
+        h_gu = torch.empty(layer.gu.shape, dtype=torch.bfloat16, pin_memory=True)
+        h_dn = torch.empty(layer.dn.shape, dtype=torch.bfloat16, pin_memory=True)
+        h_gu.copy_(layer.gu)
+        h_dn.copy_(layer.dn)
+        out = layers.host_outputs(h_gu, h_dn)
+        h2d = h_gu.numel() * 2 + h_dn.numel() * 2
+        d2h = sum(t.numel() * t.element_size() for o in out.values() for t in o.values())
+        conv = layers.HostLayerConverter(layer.gu.shape, layer.dn.shape, chunk=chunk, device=device)
+        conv.run(h_gu, h_dn, out)
+        torch.cuda.synchronize()
+        if conv.status() != 0:
+            failed = "device status %#x" % conv.status()
+    except (RuntimeError, MemoryError) as e:
+        failed = str(e).splitlines()[0][:200] if str(e) else type(e).__name__
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
-        torch.cuda.synchronize()
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record()
-    for _ in range(steps):
-        conv.run(h_gu, h_dn, out)
-    t1.record()
     torch.cuda.synchronize()
-    ms = max_over_ranks(t0.elapsed_time(t1) / steps, world, device)
+    ms = float("inf")
+    if failed is None:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for _ in range(steps):
+            conv.run(h_gu, h_dn, out)
+        t1.record()
+        torch.cuda.synchronize()
+        ms = t0.elapsed_time(t1) / steps
+    ms = max_over_ranks(ms, world, device)
+    if ms == float("inf"):
+        return {"unavailable": "e2e leg could not run on every rank: %s" % (failed or "another rank failed")}
     return {"value": layer.n_elems * world * STEP_BYTES_PER_ELEM / (ms * 1e-3) / 1e9, "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms,
             "pipeline": "chunks of %d experts, H2D / kernels / D2H on three streams" % chunk}
