@@ -9,7 +9,13 @@ round-to-nearest-even of the exact rational result, and the test asserts:
     against the exact comparison;
 on random blocks and on tie-rich and near-tie blocks (grid-exact blocks, then
 the same blocks with one element moved by one bf16 ulp).  The plans come
-from the exact-rational restatement in oracle/micro.py."""
+from the exact-rational restatement in oracle/micro.py.
+
+The same emulation covers the weighted scale search's fp32 filter: every
+candidate's fp32 weighted error W32 (the kernel's operation order) lies
+within half its error bound eps of both the exact weighted error and the
+binary64 value the definition forms, a block the filter decides gets the
+binary64 argmin, and blocks whose binary64 scores tie are never decided."""
 from fractions import Fraction as F
 
 import numpy as np
@@ -124,3 +130,99 @@ def test_ties_and_near_ties():
     # the exact ties are present and left to the exact comparison
     ties = sum(1 for xs in blocks[::2] if (r := filtered_decision(xs, s2)) and r[3])
     assert ties > 50
+
+
+# ---- the weighted search's fp32 scores and their bound -------------------
+def _wsse32(xs, hs, codes, D, s2):
+    """The kernel's fp32 weighted error of one candidate: per element
+    deq = RN(RN(q D) s2), e = RN(x - deq), then acc = RN(h RN(e e) + acc) in
+    two interleaved partial sums (even / odd elements), added at the end."""
+    acc = [F(0), F(0)]
+    for i, (x, h, c) in enumerate(zip(xs, hs, codes)):
+        deq = rn32(rn32(micro.e2m1_value(c) * D) * F(float(s2)))
+        e = rn32(F(float(x)) - deq)
+        acc[i & 1] = rn32(F(float(h)) * rn32(e * e) + acc[i & 1])
+    return rn32(acc[0] + acc[1])
+
+
+def _wsse64(xs, hs, codes, D, s2):
+    """The definition's binary64 procedure (Python floats are binary64)."""
+    acc = 0.0
+    for x, h, c in zip(xs, hs, codes):
+        deq = float(micro.e2m1_value(c) * D) * float(s2)     # exact: 4 + 24 bits
+        e = float(x) - deq
+        acc = acc + float(h) * (e * e)
+    return acc
+
+
+def _weighted_case(xs, hs, s2):
+    """One block of the weighted search: checks every candidate's fp32 score
+    against its bound and the filter's decision against the binary64 argmin.
+    Returns (candidates checked, decided, binary64 argmin was a tie)."""
+    # A as the kernel forms it: acc = RN(h RN(x x) + acc) in two partial sums
+    acc = [F(0), F(0)]
+    for i, (x, h) in enumerate(zip(xs, hs)):
+        acc[i & 1] = rn32(F(float(h)) * rn32(F(float(x)) ** 2) + acc[i & 1])
+    A = rn32(acc[0] + acc[1])
+    if not (F(2) ** -60 <= A <= F(2) ** 100):
+        return 0, False, False
+    sc6, _, _ = micro.plan(xs, s2, 6)
+    sc4, _, _ = micro.plan(xs, s2, 4)
+    cands = []
+    for sc in range(sc6, sc4 + 1):
+        codes, _ = micro.plan_with_scale_code(xs, s2, sc)
+        D = F(micro.e4m3_value(sc))
+        w32 = _wsse32(xs, hs, codes, D, s2)
+        exact = sum(F(float(h)) * (F(float(x)) - micro.e2m1_value(c) * D * F(float(s2))) ** 2
+                    for x, h, c in zip(xs, hs, codes))
+        w64 = F(_wsse64(xs, hs, codes, D, s2))
+        eps = (F(2.0 ** -22 * float(A * w32) ** 0.5) + F(2.0 ** -19) * w32
+               + F(2.0 ** -45) * A + F(2.0 ** -100))
+        # the constants take about twice the derived error: half of eps must do
+        assert abs(w32 - exact) <= eps / 2, (sc, float(w32), float(exact))
+        assert abs(w32 - w64) <= eps / 2, (sc, float(w32), float(w64))
+        cands.append((sc, w32, eps, w64))
+    # the filter: the fp32 argmin (first on equal scores) is kept when every
+    # other candidate's W - eps lies above the best's W + eps
+    best = min(range(len(cands)), key=lambda i: (cands[i][1], i))
+    bw, be = cands[best][1], cands[best][2]
+    lb = min((w - e for i, (_, w, e, _) in enumerate(cands) if i != best), default=None)
+    decided = lb is None or lb > bw + be
+    w64s = [c[3] for c in cands]
+    arg64 = min(range(len(cands)), key=lambda i: (w64s[i], i))
+    tie64 = w64s.count(w64s[arg64]) > 1
+    if decided:
+        assert cands[best][0] == cands[arg64][0]
+        assert not tie64
+    return len(cands), decided, tie64
+
+
+def test_weighted_fp32_bound_and_filter():
+    rng = np.random.default_rng(33)
+    s2 = micro.global_scale(np.float32(2.625))
+    checked = decided = 0
+    for _ in range(60):
+        xs = _bf16(np.clip(rng.standard_normal(16) * rng.choice([0.05, 0.3]), -2.625, 2.625))
+        hs = [np.float32(v) for v in rng.gamma(0.7, 1.0, 16)]
+        n, d, _ = _weighted_case(xs, hs, s2)
+        checked += n
+        decided += d
+    assert checked > 250 and decided > 40
+
+
+def test_weighted_filter_leaves_ties_to_binary64():
+    """One-hot weights on a grid-exact element: several candidates score the
+    same, and the filter must hand every such block to the binary64 search."""
+    rng = np.random.default_rng(34)
+    s2 = np.float32(2.0 ** -10)
+    ties = 0
+    for _ in range(60):
+        base = float(2.0 ** int(rng.integers(-3, 4))) * float(s2)
+        v = rng.choice([0.5, 1.0, 1.5, 2.0, 3.0, -1.0, -2.0], 16) * base
+        v[rng.integers(16)] = 6.0 * base
+        xs = _bf16(v)
+        hs = [np.float32(0.0)] * 16
+        hs[int(rng.integers(16))] = np.float32(rng.choice([0.25, 1.0, 3.0]))
+        _, _, tie = _weighted_case(xs, hs, s2)
+        ties += tie
+    assert ties > 20
