@@ -15,6 +15,7 @@ larger than L2, so no flush is needed between steps.
     python bench.py --workload mxfp8_shared    # MXFP8 rewrite of 48 shared experts (dense + padded)
     python bench.py --workload mxfp4_layer     # MXFP4 quantize + verify of a full-size layer
     python bench.py --workload act_sweep       # activation tiles [T, 2048], NVFP4 and MXFP8
+    python bench.py --workload mixed8          # 8 layers: NVFP4 4/6 (even) and MXFP4 (odd)
 
 Prints one JSON line on rank 0.  Under torchrun every rank converts its own
 layer (independent units, no data-path collective: weak scaling); the step
@@ -163,11 +164,14 @@ def device_uuid():
 class Layer:
     """Device-resident layer and preallocated outputs."""
 
-    def __init__(self, seed, device, experts=EXPERTS):
+    def __init__(self, seed, device, experts=EXPERTS, tensors=None):
         from mxfp_block_scaled_b200 import mxq, workloads
         self.mxq = mxq
-        self.gu, self.dn, _ = workloads.full_moe_layer(seed=seed, device=device, experts=experts,
-                                                        hidden=HIDDEN, inter=INTER)
+        if tensors is None:
+            self.gu, self.dn, _ = workloads.full_moe_layer(seed=seed, device=device, experts=experts,
+                                                            hidden=HIDDEN, inter=INTER)
+        else:
+            self.gu, self.dn = tensors
         self.n_elems = self.gu.numel() + self.dn.numel()
         self.out = {}
         for name, x in (("gu", self.gu), ("dn", self.dn)):
@@ -687,6 +691,103 @@ def run_mx(args, device):
     return result
 
 
+# Layer formats of the mixed-format conversion: layers 0, 2, 4, 6 NVFP4
+# 4/6-optimal, layers 1, 3, 5, 7 MXFP4 (each with its verifier pass).
+MIXED_FORMATS = ("nvfp4", "mxfp4") * 4
+
+
+def mixed_bytes_per_layer(fmt, n_elems):
+    """Algorithmic bytes of one layer's quantize + verify."""
+    return n_elems * (STEP_BYTES_PER_ELEM if fmt == "nvfp4" else 2 * MX_BYTES[fmt])
+
+
+def run_mixed8(args, device):
+    """Mixed-format conversion of eight full-size routed-expert layers, values
+    N(0, 0.02) with the Student-t(4) tail mix: every layer quantized (NVFP4
+    4/6-optimal or MXFP4 by MIXED_FORMATS) and verified over all its unstacked
+    tensors, all eight layers resident in HBM (38.7 GB of bf16 inputs)."""
+    from mxfp_block_scaled_b200 import mxq, workloads
+    calls, names, nv, mx = [], [], [], []
+    n_total, bytes_total = 0, 0.0
+    for L, fmt in enumerate(MIXED_FORMATS):
+        gu, dn = workloads.student_t_mix_layer(seed=L, device=device, experts=args.experts)
+        n = gu.numel() + dn.numel()
+        if fmt == "nvfp4":
+            lay = Layer(seed=L, device=device, experts=args.experts, tensors=(gu, dn))
+            nv.append(lay)
+            calls += [(lambda lay=lay, k=k, t=t: getattr(lay, k)(t)) for k, t in Layer.CALLS]
+        else:
+            st = [MXStack(mxq, gu.view(-1, gu.shape[-1]), fmt, gu.shape[1] // 2, device),
+                  MXStack(mxq, dn.view(-1, dn.shape[-1]), fmt, dn.shape[1], device)]
+            mx.append(st)
+            calls += [st[0].quantize, st[1].quantize, st[0].verify, st[1].verify]
+        names += ["L%d_%s_%s" % (L, k, t) for k, t in Layer.CALLS]
+        n_total += n
+        bytes_total += mixed_bytes_per_layer(fmt, n)
+    torch.cuda.synchronize()
+    ms, call_ms, clocks = time_calls(calls, args.steps, args.warmup)
+    for lay in nv:
+        for t in ("gu", "dn"):
+            if int(lay.out[t]["status"].item()) != 0:
+                raise RuntimeError("device status %#x" % int(lay.out[t]["status"].item()))
+    for st in mx:
+        for s in st:
+            if int(s.status.item()) != 0:
+                raise RuntimeError("device status %#x" % int(s.status.item()))
+    peak, peak_kind = measured_peak()
+    value = bytes_total / (ms * 1e-3) / 1e9
+    # dominant kernel: the NVFP4 gate_up quantize launch (call 0 of each NVFP4 layer)
+    q_ms = statistics.mean(call_ms[4 * L] for L, f in enumerate(MIXED_FORMATS) if f == "nvfp4")
+    gu_elems = nv[0].gu.numel()
+    achieved = gu_elems * Q_BYTES / (q_ms * 1e-3) / 1e9
+    traffic = ncu_traffic_per_launch() if args.experts == EXPERTS else None
+    rel_nv = torch.cat([lay.out[t]["rel"] for lay in nv for t in ("gu", "dn")]).cpu().numpy()
+    rel_mx = torch.cat([s.rel for st in mx for s in st]).cpu().numpy()
+    m4 = sum(int(lay.out[t]["m4"].sum().item()) for lay in nv for t in ("gu", "dn"))
+    nv_blocks = sum(lay.n_elems // 16 for lay in nv)
+    workload = ("mixed-format conversion of 8 full-size routed-expert layers (Student-t tail mix), "
+                "quantize + verify: layers 0,2,4,6 NVFP4 4/6-optimal, layers 1,3,5,7 MXFP4; each "
+                "gate_up bf16 [%d,1536,2048] + down [%d,2048,768]" % (args.experts, args.experts))
+    result = {
+        "metric": "mixed-format NVFP4 4/6 + MXFP4 quantize+verify HBM GB/s (1 GPU)", "value": value,
+        "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": workload if args.experts == EXPERTS else
+                   "PROFILING CASE, %d experts per layer (not the full-size workload)" % args.experts,
+                   "layers": len(MIXED_FORMATS), "formats": list(MIXED_FORMATS),
+                   "elements_per_gpu": n_total, "algorithmic_bytes_per_step": bytes_total,
+                   "l2": "inputs %.1f GB, larger than L2; no flush" % (n_total * 2 / 1e9),
+                   "fraction_of_peak": value / peak, "peak_gbs": peak, "peak_kind": peak_kind,
+                   "call_ms": dict(zip(names, call_ms)),
+                   "quality": {"nvfp4": {"relerr_mean": float(rel_nv.mean()), "relerr_max": float(rel_nv.max()),
+                                         "tensors": int(rel_nv.size), "m4_fraction": m4 / nv_blocks},
+                               "mxfp4": {"relerr_mean": float(rel_mx.mean()), "relerr_max": float(rel_mx.max()),
+                                         "tensors": int(rel_mx.size)}}},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "traffic_note": "DRAM bytes of the same kernel on the same shape (routed-layer values); "
+                                     "its traffic does not depend on the values",
+                     "kernel": "nvfp4_fused_kernel (gate_up stacks of the NVFP4 layers)",
+                     "algorithmic_bytes_per_launch": gu_elems * Q_BYTES, "peak_kind": peak_kind},
+        "gpu_launches": args.steps * sum(
+            2 * (KERNELS_PER_QUANTIZE_NVFP4 + KERNELS_PER_VERIFY) if f == "nvfp4" else 2 + 2 * KERNELS_PER_VERIFY
+            for f in MIXED_FORMATS),
+        "clocks": clocks,
+    }
+    if not args.no_extras:
+        a = run_cpu_baseline(nv[0], args.cpu_budget / 2)
+        b = mx_cpu_baseline(mx[0], "mxfp4", args.cpu_budget / 2)
+        # CPU time of one step at the two measured element rates
+        t_step = sum((lay.n_elems / a["elements_per_s"]) for lay in nv) + \
+            sum(sum(s.R * s.C for s in st) / b["elements_per_s"] for st in mx)
+        result["cpu_baseline"] = {"value": bytes_total / t_step / 1e9, "unit": "GB/s", "cores": 1,
+                                  "kind": "oracle",
+                                  "sample": "NVFP4: %s; MXFP4: %s; combined at the step's element mix"
+                                            % (a["sample"], b["sample"])}
+    return result
+
+
 def time_loop(call, reps, warmup):
     """Mean time (us) of `reps` back-to-back calls on the current stream,
     CUDA events around the whole loop, and the clock samples."""
@@ -824,11 +925,12 @@ def main():
                     help="skip the e2e and CPU-baseline legs (profiling runs)")
     ap.add_argument("--workload", default="nvfp4_layer",
                     choices=["nvfp4_layer", "fp8_requant", "nvfp4_weighted", "mxfp8_shared",
-                             "mxfp4_layer", "act_sweep"],
+                             "mxfp4_layer", "act_sweep", "mixed8"],
                     help="nvfp4_layer: the headline quantize + verify step; fp8_requant: block-FP8 "
                          "-> MXFP4 requantization of the same layer; nvfp4_weighted: weighted-SSE "
                          "scale search; mxfp8_shared / mxfp4_layer: MX quantize + verify; act_sweep: "
-                         "dynamic activation quantization over T")
+                         "dynamic activation quantization over T; mixed8: 8 layers, NVFP4 4/6 and "
+                         "MXFP4 alternating, quantize + verify")
     ap.add_argument("--experts", type=int, default=EXPERTS,
                     help="experts in the layer; fewer than 512 only for small profiling captures")
     args = ap.parse_args()
@@ -861,10 +963,10 @@ def main():
             raise SystemExit("--workload nvfp4_weighted runs on one GPU")
         print(json.dumps(run_weighted(args, device)), flush=True)
         return 0
-    if args.workload in ("mxfp8_shared", "mxfp4_layer", "act_sweep"):
+    if args.workload in ("mxfp8_shared", "mxfp4_layer", "act_sweep", "mixed8"):
         if world > 1:
             raise SystemExit("--workload %s runs on one GPU" % args.workload)
-        run = run_act if args.workload == "act_sweep" else run_mx
+        run = {"act_sweep": run_act, "mixed8": run_mixed8}.get(args.workload, run_mx)
         print(json.dumps(run(args, device)), flush=True)
         return 0
 

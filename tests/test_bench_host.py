@@ -61,3 +61,11 @@ def test_algorithmic_bytes_per_element():
     assert bench.Q_BYTES == 2.5625 and bench.STEP_BYTES_PER_ELEM == 5.125
     assert bench.MX_BYTES == {"mxfp8": 3.03125, "mxfp4": 2.53125}
     assert bench.ACT_BYTES["nvfp4"] == 2.5625
+
+
+def test_mixed_format_layers_and_bytes():
+    # layers 0, 2, 4, 6 NVFP4 4/6-optimal, layers 1, 3, 5, 7 MXFP4
+    assert bench.MIXED_FORMATS == ("nvfp4", "mxfp4", "nvfp4", "mxfp4", "nvfp4", "mxfp4", "nvfp4", "mxfp4")
+    n = 512 * 1536 * 2048 + 512 * 2048 * 768
+    step = sum(bench.mixed_bytes_per_layer(f, n) for f in bench.MIXED_FORMATS)
+    assert step == 4 * n * (5.125 + 5.0625)          # about 98.45 GB per step
