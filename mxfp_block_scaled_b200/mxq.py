@@ -116,28 +116,78 @@ def _workspace(op, n, rows, cols, device):
     return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device), nbytes
 
 
+def _nbytes(t):
+    return 0 if t is None else t.numel() * t.element_size()
+
+
+def _need(name, t, nbytes):
+    """The library sees only a pointer, so a buffer that is not contiguous or
+    is smaller than the call reads or writes is refused here, before anything
+    is enqueued (the kernels would otherwise touch memory past its end).
+    Sizes the library rejects (negative, misaligned shapes) give nbytes <= 0
+    here and are left to its status code."""
+    if t is None:
+        return
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if _nbytes(t) < nbytes:
+        raise ValueError("%s holds %d bytes; the call needs %d" % (name, _nbytes(t), nbytes))
+
+
+def _verify_scale_need(fmt, layout, n_tensors, rows, cols, tps):
+    """Scale bytes the verifier reads: n_tensors * rows * cols / block when
+    linear; tiled, each run of tps tensors is one scale matrix (the last run
+    may be shorter)."""
+    if layout == "linear" or tps < 1:
+        return scale_bytes(fmt, "linear", n_tensors, rows, cols)
+    full, rem = divmod(n_tensors, tps)
+    return (scale_bytes(fmt, layout, full, rows * tps, cols)
+            + (scale_bytes(fmt, layout, 1, rows * rem, cols) if rem else 0))
+
+
+def _code_bytes(fmt, n):
+    return n if fmt == "mxfp8" else n // 2
+
+
 # ---------------------------------------------------------------- C names --
 def mxq_quantize_nvfp4(x, n_groups, rows, cols, mode, layout, codes, scales, s2, mbits, m4_count,
                        status, workspace, stream=None):
+    n = n_groups * rows * cols
+    _need("x", x, 2 * n)
+    _need("codes", codes, n // 2)
+    _need("scales", scales, scale_bytes("nvfp4", layout, n_groups, rows, cols))
+    _need("s2", s2, 4 * n_groups)
+    _need("mbits", mbits, 4 * ((n // 16 + 31) // 32))
+    _need("m4_count", m4_count, 4 * n_groups)
+    _need("status", status, 4)
     rc = load().mxq_quantize_nvfp4(_p(x), n_groups, rows, cols, SCALE_MODE[mode], LAYOUT[layout],
                                    _p(codes),
                                    _p(scales), _p(s2), _p(mbits), _p(m4_count), _p(status),
-                                   _p(workspace), workspace.numel() if workspace is not None else 0,
-                                   _stream(stream))
+                                   _p(workspace), _nbytes(workspace), _stream(stream))
     _check("mxq_quantize_nvfp4", rc)
 
 
 def mxq_quantize_nvfp4_weighted(x, n_groups, rows, cols, h, h_groups, layout, codes, scales, s2,
                                 status, workspace, stream=None):
+    n = n_groups * rows * cols
+    _need("x", x, 2 * n)
+    _need("h", h, 4 * h_groups * cols)
+    _need("codes", codes, n // 2)
+    _need("scales", scales, scale_bytes("nvfp4", layout, n_groups, rows, cols))
+    _need("s2", s2, 4 * n_groups)
+    _need("status", status, 4)
     rc = load().mxq_quantize_nvfp4_weighted(_p(x), n_groups, rows, cols, _p(h), h_groups,
                                             LAYOUT[layout], _p(codes), _p(scales), _p(s2), _p(status),
-                                            _p(workspace),
-                                            workspace.numel() if workspace is not None else 0,
-                                            _stream(stream))
+                                            _p(workspace), _nbytes(workspace), _stream(stream))
     _check("mxq_quantize_nvfp4_weighted", rc)
 
 
 def mxq_quantize_mx(x, rows, cols, fmt, block, layout, codes, scales, status, stream=None):
+    n = rows * cols
+    _need("x", x, 2 * n)
+    _need("codes", codes, _code_bytes(fmt, n))
+    _need("scales", scales, scale_bytes(fmt, layout, 1, rows, cols))
+    _need("status", status, 4)
     rc = load().mxq_quantize_mx(_p(x), rows, cols, FMT[fmt], block, LAYOUT[layout], _p(codes),
                                 _p(scales), _p(status), _stream(stream))
     _check("mxq_quantize_mx", rc)
@@ -145,6 +195,13 @@ def mxq_quantize_mx(x, rows, cols, fmt, block, layout, codes, scales, status, st
 
 def mxq_requant_fp8_mx(fp8, bscale, rows, cols, brows, bcols, fmt, layout, codes, scales, status,
                        stream=None):
+    n = rows * cols
+    _need("fp8", fp8, n)
+    if brows > 0 and bcols > 0:
+        _need("bscale", bscale, 4 * (-(-rows // brows)) * (-(-cols // bcols)))
+    _need("codes", codes, _code_bytes(fmt, n))
+    _need("scales", scales, scale_bytes(fmt, layout, 1, rows, cols))
+    _need("status", status, 4)
     rc = load().mxq_requant_fp8_mx(_p(fp8), _p(bscale), rows, cols, brows, bcols, FMT[fmt],
                                    LAYOUT[layout], _p(codes), _p(scales), _p(status), _stream(stream))
     _check("mxq_requant_fp8_mx", rc)
@@ -152,20 +209,37 @@ def mxq_requant_fp8_mx(fp8, bscale, rows, cols, brows, bcols, fmt, layout, codes
 
 def mxq_quantize_act(tokens, T, hidden, fmt, mode, layout, codes, scales, input_scale, status,
                      workspace, stream=None):
+    n = T * hidden
+    _need("tokens", tokens, 2 * n)
+    _need("codes", codes, _code_bytes(fmt, n))
+    _need("scales", scales, scale_bytes(fmt, layout, 1, T, hidden))
+    _need("input_scale", input_scale, 4 if fmt == "nvfp4" else 0)
+    _need("status", status, 4)
     rc = load().mxq_quantize_act(_p(tokens), T, hidden, FMT[fmt], SCALE_MODE[mode], LAYOUT[layout],
                                  _p(codes), _p(scales),
                                  _p(input_scale), _p(status), _p(workspace),
-                                 workspace.numel() if workspace is not None else 0, _stream(stream))
+                                 _nbytes(workspace), _stream(stream))
     _check("mxq_quantize_act", rc)
+
+
+def _need_verify(x, codes, scales, s2, fmt, layout, n_tensors, rows, cols, tps, err, ref, rel):
+    n = n_tensors * rows * cols
+    _need("x", x, 2 * n)
+    _need("codes", codes, _code_bytes(fmt, n))
+    _need("scales", scales, _verify_scale_need(fmt, layout, n_tensors, rows, cols, tps))
+    if fmt == "nvfp4" and tps >= 1:
+        _need("s2", s2, 4 * (-(-n_tensors // tps)))
+    for name, t in (("sum_sq_err", err), ("sum_sq_ref", ref), ("relerr", rel)):
+        _need(name, t, 8 * n_tensors)
 
 
 def mxq_dequant_relerr(x, codes, scales, s2, fmt, layout, n_tensors, rows, cols,
                        tensors_per_scale, sum_sq_err, sum_sq_ref, relerr, workspace, stream=None):
+    _need_verify(x, codes, scales, s2, fmt, layout, n_tensors, rows, cols, tensors_per_scale,
+                 sum_sq_err, sum_sq_ref, relerr)
     rc = load().mxq_dequant_relerr(_p(x), _p(codes), _p(scales), _p(s2), FMT[fmt], LAYOUT[layout],
                                    n_tensors, rows, cols, tensors_per_scale, _p(sum_sq_err), _p(sum_sq_ref),
-                                   _p(relerr), _p(workspace),
-                                   workspace.numel() if workspace is not None else 0,
-                                   _stream(stream))
+                                   _p(relerr), _p(workspace), _nbytes(workspace), _stream(stream))
     _check("mxq_dequant_relerr", rc)
 
 
@@ -175,6 +249,8 @@ def mxq_dequant_relerr_noalloc(x, codes, scales, s2, fmt, n_tensors, rows, cols,
     device memory: its partial sums live in a fixed 2 MiB array inside the
     library (at most 131072 chunks of 16384 elements per call).  Calls whose
     GPU work overlaps in time share that array and race."""
+    _need_verify(x, codes, scales, s2, fmt, "linear", n_tensors, rows, cols, tensors_per_scale,
+                 sum_sq_err, sum_sq_ref, relerr)
     rc = load().mxq_dequant_relerr_noalloc(_p(x), _p(codes), _p(scales), _p(s2), FMT[fmt],
                                            n_tensors, rows, cols, tensors_per_scale,
                                            _p(sum_sq_err), _p(sum_sq_ref), _p(relerr),
