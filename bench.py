@@ -16,6 +16,8 @@ larger than L2, so no flush is needed between steps.
     python bench.py --workload mxfp4_layer     # MXFP4 quantize + verify of a full-size layer
     python bench.py --workload act_sweep       # activation tiles [T, 2048], NVFP4 and MXFP8
     python bench.py --workload mixed8          # 8 layers: NVFP4 4/6 (even) and MXFP4 (odd)
+    --layout swizzled_128x4   block scales in the 128x4 tiled layout (layer and MX workloads)
+    --act-mode four_six       4/6-optimal NVFP4 block scales in act_sweep
 
 Prints one JSON line on rank 0.  Under torchrun every rank converts its own
 layer (independent units, no data-path collective: weak scaling); the step
@@ -164,9 +166,10 @@ def device_uuid():
 class Layer:
     """Device-resident layer and preallocated outputs."""
 
-    def __init__(self, seed, device, experts=EXPERTS, tensors=None):
+    def __init__(self, seed, device, experts=EXPERTS, tensors=None, layout="linear"):
         from mxfp_block_scaled_b200 import mxq, workloads
         self.mxq = mxq
+        self.layout = layout
         if tensors is None:
             self.gu, self.dn, _ = workloads.full_moe_layer(seed=seed, device=device, experts=experts,
                                                             hidden=HIDDEN, inter=INTER)
@@ -185,7 +188,8 @@ class Layer:
             self.out[name] = dict(
                 x=x, G=G, R=R, C=C, nt=nt, rows=rows, cols=cols, tps=tps,
                 codes=torch.empty((G, R, C // 2), dtype=torch.uint8, device=device),
-                scales=torch.empty((G, R, C // 16), dtype=torch.uint8, device=device),
+                scales=torch.empty(mxq.scale_bytes("nvfp4", layout, G, R, C), dtype=torch.uint8,
+                                   device=device),
                 s2=torch.empty(G, dtype=torch.float32, device=device),
                 mbits=torch.empty((G * R * C // 16 + 31) // 32, dtype=torch.int32, device=device),
                 m4=torch.empty(G, dtype=torch.int32, device=device),
@@ -199,12 +203,12 @@ class Layer:
 
     def quantize(self, name):
         o = self.out[name]
-        self.mxq.mxq_quantize_nvfp4(o["x"], o["G"], o["R"], o["C"], "four_six", "linear", o["codes"],
+        self.mxq.mxq_quantize_nvfp4(o["x"], o["G"], o["R"], o["C"], "four_six", self.layout, o["codes"],
                                     o["scales"], o["s2"], o["mbits"], o["m4"], o["status"], o["wsq"])
 
     def verify(self, name):
         o = self.out[name]
-        self.mxq.mxq_dequant_relerr(o["x"], o["codes"], o["scales"], o["s2"], "nvfp4", "linear", o["nt"],
+        self.mxq.mxq_dequant_relerr(o["x"], o["codes"], o["scales"], o["s2"], "nvfp4", self.layout, o["nt"],
                                     o["rows"], o["cols"], o["tps"], o["err"], o["ref"], o["rel"],
                                     o["wsv"])
 
@@ -566,13 +570,14 @@ class MXStack:
     [rows, cols] matrix (MX scales are per 32 values: no per-tensor state)
     and verified per tensor of `trows` rows."""
 
-    def __init__(self, mxq, x2d, fmt, trows, device):
-        self.mxq, self.x, self.fmt, self.trows = mxq, x2d, fmt, trows
+    def __init__(self, mxq, x2d, fmt, trows, device, layout="linear"):
+        self.mxq, self.x, self.fmt, self.trows, self.layout = mxq, x2d, fmt, trows, layout
         self.R, self.C = x2d.shape
         self.nt = self.R // trows
         self.codes = torch.empty((self.R, self.C if fmt == "mxfp8" else self.C // 2), dtype=torch.uint8,
                                  device=device)
-        self.scales = torch.empty((self.R, self.C // 32), dtype=torch.uint8, device=device)
+        self.scales = torch.empty(mxq.scale_bytes(fmt, layout, 1, self.R, self.C), dtype=torch.uint8,
+                                  device=device)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
         ws = mxq.workspace_bytes("dequant_relerr", self.nt, trows, self.C)
         self.wsv = torch.empty(max(ws, 256), dtype=torch.uint8, device=device)
@@ -580,12 +585,14 @@ class MXStack:
                                         for _ in range(3))
 
     def quantize(self):
-        self.mxq.mxq_quantize_mx(self.x, self.R, self.C, self.fmt, 32, "linear", self.codes, self.scales,
+        self.mxq.mxq_quantize_mx(self.x, self.R, self.C, self.fmt, 32, self.layout, self.codes, self.scales,
                                  self.status)
 
     def verify(self):
-        self.mxq.mxq_dequant_relerr(self.x, self.codes, self.scales, None, self.fmt, "linear", self.nt,
-                                    self.trows, self.C, 1, self.err, self.ref, self.rel, self.wsv)
+        # tiled: the stack was quantized as one matrix, so all its tensors share one scale matrix
+        tps = 1 if self.layout == "linear" else self.nt
+        self.mxq.mxq_dequant_relerr(self.x, self.codes, self.scales, None, self.fmt, self.layout, self.nt,
+                                    self.trows, self.C, tps, self.err, self.ref, self.rel, self.wsv)
 
 
 def mx_cpu_baseline(stacks, fmt, budget_s=15.0):
@@ -630,16 +637,16 @@ def run_mx(args, device):
                 dns.append(dn)
         GU, DN = torch.stack(gus), torch.stack(dns)
         del gus, dns
-        stacks = [MXStack(mxq, GU.view(-1, GU.shape[-1]), fmt, GU.shape[1] // 2, device),
-                  MXStack(mxq, DN.view(-1, DN.shape[-1]), fmt, DN.shape[1], device)]
+        stacks = [MXStack(mxq, GU.view(-1, GU.shape[-1]), fmt, GU.shape[1] // 2, device, args.layout),
+                  MXStack(mxq, DN.view(-1, DN.shape[-1]), fmt, DN.shape[1], device, args.layout)]
         workload = ("shared-expert MXFP8 rewrite, quantize + verify: 48 layers x {dense, padded} of "
                     "gate/up bf16 [2560,2048] + down [2048,1280] (gate and up verified separately)")
         check_pad = True
     else:
         fmt = "mxfp4"
         GU, DN = workloads.student_t_mix_layer(seed=0, device=device, experts=args.experts)
-        stacks = [MXStack(mxq, GU.view(-1, GU.shape[-1]), fmt, GU.shape[1] // 2, device),
-                  MXStack(mxq, DN.view(-1, DN.shape[-1]), fmt, DN.shape[1], device)]
+        stacks = [MXStack(mxq, GU.view(-1, GU.shape[-1]), fmt, GU.shape[1] // 2, device, args.layout),
+                  MXStack(mxq, DN.view(-1, DN.shape[-1]), fmt, DN.shape[1], device, args.layout)]
         workload = ("one full-size routed-expert layer (Student-t tail mix), MXFP4 quantize + verify: "
                     "gate_up bf16 [%d,1536,2048] + down [%d,2048,768]" % (args.experts, args.experts))
         check_pad = False
@@ -653,11 +660,14 @@ def run_mx(args, device):
         # the padded copies (odd stack entries) must quantize to exact zeros, codes and scale
         # bytes: gate rows [640, 1280) and up rows [1920, 2560) of gate/up, columns [640, 1280)
         # of down
+        # (value codes in every layout; scale bytes where they are linear)
         cg = stacks[0].codes.view(GU.shape[0], GU.shape[1], -1)[1::2]
-        sg = stacks[0].scales.view(GU.shape[0], GU.shape[1], -1)[1::2]
         cd = stacks[1].codes.view(DN.shape[0], DN.shape[1], -1)[1::2]
-        sd = stacks[1].scales.view(DN.shape[0], DN.shape[1], -1)[1::2]
-        zero = [cg[:, 640:1280], cg[:, 1920:], sg[:, 640:1280], sg[:, 1920:], cd[:, :, 640:], sd[:, :, 20:]]
+        zero = [cg[:, 640:1280], cg[:, 1920:], cd[:, :, 640:]]
+        if args.layout == "linear":
+            sg = stacks[0].scales.view(GU.shape[0], GU.shape[1], -1)[1::2]
+            sd = stacks[1].scales.view(DN.shape[0], DN.shape[1], -1)[1::2]
+            zero += [sg[:, 640:1280], sg[:, 1920:], sd[:, :, 20:]]
         if any(int(z.count_nonzero()) for z in zero):
             raise RuntimeError("padded regions did not quantize to zeros")
     n = sum(s.R * s.C for s in stacks)
@@ -673,7 +683,8 @@ def run_mx(args, device):
         "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": workload, "elements_per_gpu": n, "algorithmic_bytes_per_element": bpe,
+        "config": {"workload": workload, "scale_layout": args.layout, "elements_per_gpu": n,
+                   "algorithmic_bytes_per_element": bpe,
                    "l2": "inputs %.1f GB, larger than L2; no flush" % (n * 2 / 1e9),
                    "fraction_of_peak": value / peak, "peak_gbs": peak, "peak_kind": peak_kind,
                    "call_ms": dict(zip(names, call_ms)),
@@ -713,12 +724,12 @@ def run_mixed8(args, device):
         gu, dn = workloads.student_t_mix_layer(seed=L, device=device, experts=args.experts)
         n = gu.numel() + dn.numel()
         if fmt == "nvfp4":
-            lay = Layer(seed=L, device=device, experts=args.experts, tensors=(gu, dn))
+            lay = Layer(seed=L, device=device, experts=args.experts, tensors=(gu, dn), layout=args.layout)
             nv.append(lay)
             calls += [(lambda lay=lay, k=k, t=t: getattr(lay, k)(t)) for k, t in Layer.CALLS]
         else:
-            st = [MXStack(mxq, gu.view(-1, gu.shape[-1]), fmt, gu.shape[1] // 2, device),
-                  MXStack(mxq, dn.view(-1, dn.shape[-1]), fmt, dn.shape[1], device)]
+            st = [MXStack(mxq, gu.view(-1, gu.shape[-1]), fmt, gu.shape[1] // 2, device, args.layout),
+                  MXStack(mxq, dn.view(-1, dn.shape[-1]), fmt, dn.shape[1], device, args.layout)]
             mx.append(st)
             calls += [st[0].quantize, st[1].quantize, st[0].verify, st[1].verify]
         names += ["L%d_%s_%s" % (L, k, t) for k, t in Layer.CALLS]
@@ -740,7 +751,7 @@ def run_mixed8(args, device):
     q_ms = statistics.mean(call_ms[4 * L] for L, f in enumerate(MIXED_FORMATS) if f == "nvfp4")
     gu_elems = nv[0].gu.numel()
     achieved = gu_elems * Q_BYTES / (q_ms * 1e-3) / 1e9
-    traffic = ncu_traffic_per_launch() if args.experts == EXPERTS else None
+    traffic = ncu_traffic_per_launch() if args.experts == EXPERTS and args.layout == "linear" else None
     rel_nv = torch.cat([lay.out[t]["rel"] for lay in nv for t in ("gu", "dn")]).cpu().numpy()
     rel_mx = torch.cat([s.rel for st in mx for s in st]).cpu().numpy()
     m4 = sum(int(lay.out[t]["m4"].sum().item()) for lay in nv for t in ("gu", "dn"))
@@ -755,7 +766,7 @@ def run_mixed8(args, device):
         "data": "synthetic",
         "config": {"workload": workload if args.experts == EXPERTS else
                    "PROFILING CASE, %d experts per layer (not the full-size workload)" % args.experts,
-                   "layers": len(MIXED_FORMATS), "formats": list(MIXED_FORMATS),
+                   "layers": len(MIXED_FORMATS), "formats": list(MIXED_FORMATS), "scale_layout": args.layout,
                    "elements_per_gpu": n_total, "algorithmic_bytes_per_step": bytes_total,
                    "l2": "inputs %.1f GB, larger than L2; no flush" % (n_total * 2 / 1e9),
                    "fraction_of_peak": value / peak, "peak_gbs": peak, "peak_kind": peak_kind,
@@ -840,7 +851,8 @@ ACT_BYTES = {"nvfp4": 2.0 + 0.5 + 1.0 / 16, "mxfp8": 2.0 + 1.0 + 1.0 / 32}   # q
 def run_act(args, device):
     """Dynamic activation quantization of token tiles [T, 2048] (N(0, 1),
     four outlier channels x 30): NVFP4 (input_scale = amax/2688, amax/6
-    block scales) and MXFP8, each T timed as back-to-back calls on one
+    block scales, or the 4/6-optimal rule with --act-mode four_six) and
+    MXFP8, each T timed as back-to-back calls on one
     stream (the latency of a call in a stream of calls)."""
     from mxfp_block_scaled_b200 import mxq, workloads
     H = HIDDEN
@@ -851,13 +863,14 @@ def run_act(args, device):
         for fmt in ("nvfp4", "mxfp8"):
             blk = 16 if fmt == "nvfp4" else 32
             codes = torch.empty((T, H if fmt == "mxfp8" else H // 2), dtype=torch.uint8, device=device)
-            scales = torch.empty((T, H // blk), dtype=torch.uint8, device=device)
+            scales = torch.empty(mxq.scale_bytes(fmt, args.layout, 1, T, H), dtype=torch.uint8, device=device)
             isc = torch.empty(1, dtype=torch.float32, device=device)
             st = torch.zeros(1, dtype=torch.int32, device=device)
             ws, _ = mxq._workspace("quantize_act", T, H, 0, device)
+            mode = args.act_mode if fmt == "nvfp4" else "rtn"
 
-            def call(x=x, fmt=fmt, codes=codes, scales=scales, isc=isc, st=st, ws=ws, T=T):
-                mxq.mxq_quantize_act(x, T, H, fmt, "rtn", "linear", codes, scales, isc, st, ws)
+            def call(x=x, fmt=fmt, codes=codes, scales=scales, isc=isc, st=st, ws=ws, T=T, mode=mode):
+                mxq.mxq_quantize_act(x, T, H, fmt, mode, args.layout, codes, scales, isc, st, ws)
 
             reps = 2000 if T <= 256 else (400 if T <= 4096 else 50)
             us, clk = time_loop(call, reps, max(args.warmup, 3))
@@ -881,8 +894,10 @@ def run_act(args, device):
         "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": "token tiles bf16 [T,2048], T in {1,16,256,4096,65536}, N(0,1) with "
-                               "channels 101/717/1333/1949 x30; NVFP4 (RTN block scales, "
-                               "input_scale = amax/2688) and MXFP8",
+                               "channels 101/717/1333/1949 x30; NVFP4 (%s block scales, "
+                               "input_scale = amax/2688) and MXFP8" %
+                               ("RTN" if args.act_mode == "rtn" else "4/6-optimal"),
+                   "nvfp4_scale_mode": args.act_mode, "scale_layout": args.layout,
                    "algorithmic_bytes_per_element": ACT_BYTES,
                    "l2": "T=65536 tile 268 MB, larger than L2; smaller tiles are L2-resident by design",
                    "sweep": sweep, "peak_gbs": peak, "peak_kind": peak_kind},
@@ -902,7 +917,7 @@ def run_act(args, device):
         n_el, t = 0, 0.0
         while t < args.cpu_budget / 2:
             t0 = time.perf_counter()
-            oracle.quantize_nvfp4(xb, mode=0)
+            oracle.quantize_nvfp4(xb, mode=0 if args.act_mode == "rtn" else 1)
             t += time.perf_counter() - t0
             n_el += xb.size
         result["cpu_baseline"] = {"value": n_el * ACT_BYTES["nvfp4"] / t / 1e9, "unit": "GB/s", "cores": 1,
@@ -931,6 +946,11 @@ def main():
                          "scale search; mxfp8_shared / mxfp4_layer: MX quantize + verify; act_sweep: "
                          "dynamic activation quantization over T; mixed8: 8 layers, NVFP4 4/6 and "
                          "MXFP4 alternating, quantize + verify")
+    ap.add_argument("--layout", default="linear", choices=["linear", "swizzled_128x4"],
+                    help="block-scale layout written by the quantizers and read by the verifier "
+                         "(nvfp4_layer, mixed8, mxfp8_shared, mxfp4_layer)")
+    ap.add_argument("--act-mode", default="rtn", choices=["rtn", "four_six"],
+                    help="NVFP4 block-scale rule of the act_sweep workload")
     ap.add_argument("--experts", type=int, default=EXPERTS,
                     help="experts in the layer; fewer than 512 only for small profiling captures")
     args = ap.parse_args()
@@ -970,7 +990,7 @@ def main():
         print(json.dumps(run(args, device)), flush=True)
         return 0
 
-    layer = Layer(seed=rank, device=device, experts=args.experts)
+    layer = Layer(seed=rank, device=device, experts=args.experts, layout=args.layout)
     torch.cuda.synchronize()
 
     def barrier():
@@ -1008,7 +1028,7 @@ def main():
     gu_elems = layer.gu.numel()
     q_ms = call_ms[0]
     achieved = gu_elems * Q_BYTES / (q_ms * 1e-3) / 1e9
-    traffic = ncu_traffic_per_launch()
+    traffic = ncu_traffic_per_launch() if args.layout == "linear" else None
     quality = {}
     for name in ("gu", "dn"):
         o = layer.out[name]
@@ -1020,9 +1040,11 @@ def main():
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": WORKLOAD if args.experts == EXPERTS else
+        "config": {"workload": (WORKLOAD + ("" if args.layout == "linear" else
+                                            "; block scales in the 128x4 tiled layout"))
+                   if args.experts == EXPERTS else
                    "PROFILING CASE, %d experts (not the headline workload)" % args.experts,
-                   "experts": args.experts, "hidden": HIDDEN, "inter": INTER,
+                   "experts": args.experts, "hidden": HIDDEN, "inter": INTER, "scale_layout": args.layout,
                    "elements_per_gpu": layer.n_elems, "algorithmic_bytes_per_element": STEP_BYTES_PER_ELEM,
                    "l2": "inputs 4.8 GB per GPU, larger than L2; no flush",
                    "fraction_of_peak": value / peak, "peak_gbs": peak, "peak_kind": peak_kind,
