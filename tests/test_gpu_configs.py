@@ -44,10 +44,23 @@ def unpack_mbits(words, n):
     return np.unpackbits(w.view(np.uint8), bitorder="little")[:n]
 
 
+def group_s2_from_bits(x, chunk=64):
+    """RN32(amax_g / 2688) of every group (leading index), from the bf16 bit
+    patterns on the host: the magnitude bits of non-negative bf16 order like
+    their values, and numpy's fp32 division is correctly rounded."""
+    out = []
+    for e0 in range(0, x.shape[0], chunk):
+        b = x[e0:e0 + chunk].cpu().contiguous().view(torch.int16)
+        m = (b.reshape(b.shape[0], -1).to(torch.int32) & 0x7FFF).amax(dim=1).numpy().astype(np.uint32)
+        out.append((m << 16).view(np.float32))
+    return (np.concatenate(out) / np.float32(2688.0)).astype(np.float32)
+
+
 def test_full_size_routed_layer_sampled_experts():
     """The benchmark's exact launch: full 512-expert stacks through
     mxq_quantize_nvfp4 and mxq_dequant_relerr; experts 0, 255 and 511 (and
-    their unstacked tensors) checked against the oracle."""
+    their unstacked tensors) checked against the oracle, and every group's s2
+    and M=4 count checked against properties that hold at any size."""
     gu, dn, _ = workloads.full_moe_layer(seed=0, device="cuda")
     res = layers.quantize_routed_layer(gu, dn, fmt="nvfp4", mode="four_six")
     torch.cuda.synchronize()
@@ -58,6 +71,10 @@ def test_full_size_routed_layer_sampled_experts():
         nb = R * C // 16
         gm = unpack_mbits(q["mbits"], E * nb).reshape(E, nb)
         tps = 2 if name == "gate_up" else 1
+        # every group at full size: s2 from the group amax, M=4 count = M bits set
+        s2_all = group_s2_from_bits(x)
+        assert np.array_equal(q["s2"].cpu().numpy().view(np.uint32), s2_all.view(np.uint32)), name
+        assert np.array_equal(gm.sum(1), q["m4_count"][:E].cpu().numpy()), name
         for e in (0, 255, 511):
             xb = bits(x[e:e + 1])
             c, s, s2, m4 = oracle.quantize_nvfp4(xb, mode=1)
