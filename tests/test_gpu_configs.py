@@ -142,6 +142,45 @@ def test_mixed_format_layers_reduced_experts():
     assert n == 2 * 4 * 3 and mx < 0.25
 
 
+def check_mx_layer_sampled(gu, dn, res, fmt, seed=5, n_rows=48):
+    """Sampled rows of an MX layer against the oracle (MX blocks are
+    row-local: a row quantizes alone exactly as inside its stack), the
+    first and last rows always among them, and the verifier sums of the
+    first, a middle and the last unstacked tensor."""
+    rng = np.random.default_rng(seed)
+    for name, x in (("gate_up", gu), ("down", dn)):
+        q = res[name]
+        assert int(q["status"].item()) == 0
+        E, R, C = x.shape
+        x2 = x.reshape(E * R, C)
+        codes = q["codes"].reshape(E * R, -1)
+        scales = q["scales"].reshape(E * R, -1)
+        rows = sorted(set(rng.integers(0, E * R, n_rows).tolist()) | {0, E * R - 1})
+        c, s = oracle.quantize_mx(bits(x2[rows]), fmt)
+        assert np.array_equal(codes[rows].cpu().numpy(), c), (name, fmt)
+        assert np.array_equal(scales[rows].cpu().numpy(), s), (name, fmt)
+        tps = 2 if name == "gate_up" else 1
+        tr = R // tps
+        for t in (0, E * tps // 2, E * tps - 1):
+            xt = bits(x2[t * tr:(t + 1) * tr])
+            ct, st = oracle.quantize_mx(xt, fmt)
+            oe, orf = oracle.dequant_relerr(xt, ct, st, None, fmt, 1, tr, C, 1)
+            np.testing.assert_allclose(q["sum_sq_err"][t].item(), oe[0], rtol=RTOL_STATS)
+            np.testing.assert_allclose(q["sum_sq_ref"][t].item(), orf[0], rtol=RTOL_STATS)
+
+
+def test_full_size_mxfp4_layer_sampled_rows():
+    """An MXFP4 layer of the mixed-format conversion at full size, Student-t
+    tail mix, in the launch the benchmark times (each stack one
+    [rows, cols] matrix, every unstacked tensor verified)."""
+    gu, dn = workloads.student_t_mix_layer(seed=1, device="cuda")
+    res = layers.quantize_routed_layer(gu, dn, fmt="mxfp4")
+    torch.cuda.synchronize()
+    check_mx_layer_sampled(gu, dn, res, "mxfp4")
+    mean, mx, n = layers.relerr_census([res])
+    assert n == 512 * 3 and 0.1 < mean < 0.14 and mx < 0.2
+
+
 @pytest.mark.parametrize("T", [1, 16, 256, 4096])
 def test_activation_sweep_exact(T):
     a = workloads.activation_tile(T, seed=100 + T, device="cuda")
