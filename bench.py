@@ -394,13 +394,7 @@ def run_requant(args, device):
     E = args.experts
     srcs = []
     for name, rows, cols in (("gate_up", E * 2 * INTER, HIDDEN), ("down", E * HIDDEN, INTER)):
-        codes = torch.empty((rows, cols), dtype=torch.uint8, device=device)
-        bs = torch.empty((rows // 128, -(-cols // 128)), dtype=torch.float32, device=device)
-        step = 128 * 256
-        for i, r0 in enumerate(range(0, rows, step)):
-            c, b = workloads.block_fp8_source(min(step, rows - r0), cols, seed=1000 + i, device=device)
-            codes[r0:r0 + c.shape[0]] = c
-            bs[r0 // 128:r0 // 128 + b.shape[0]] = b
+        codes, bs = workloads.block_fp8_stack(rows, cols, device=device)
         out = {"codes": torch.empty((rows, cols // 2), dtype=torch.uint8, device=device),
                "scales": torch.empty((rows, cols // 32), dtype=torch.uint8, device=device),
                "status": torch.zeros(1, dtype=torch.int32, device=device)}

@@ -154,6 +154,22 @@ def block_fp8_source(rows, cols, seed=0, device="cpu", brows=128, bcols=128):
     return codes, scales.to(torch.float32)
 
 
+def block_fp8_stack(rows, cols, device="cpu", seed0=1000, chunk_rows=128 * 256):
+    """A full-size block-FP8 stack (128 x 128 source blocks) built from
+    block_fp8_source in runs of chunk_rows rows (a multiple of 128), seeds
+    seed0, seed0 + 1, ... per run, so the generator's temporaries stay small.
+    Returns codes [rows, cols] uint8 and scales [ceil(rows/128),
+    ceil(cols/128)] fp32."""
+    assert chunk_rows % 128 == 0
+    codes = torch.empty((rows, cols), dtype=torch.uint8, device=device)
+    scales = torch.empty((-(-rows // 128), -(-cols // 128)), dtype=torch.float32, device=device)
+    for i, r0 in enumerate(range(0, rows, chunk_rows)):
+        c, b = block_fp8_source(min(chunk_rows, rows - r0), cols, seed=seed0 + i, device=device)
+        codes[r0:r0 + c.shape[0]] = c
+        scales[r0 // 128:r0 // 128 + b.shape[0]] = b
+    return codes, scales
+
+
 def bf16_bits(t):
     """bf16 tensor -> numpy uint16 array of its bit patterns (host copy)."""
     return t.detach().contiguous().view(torch.int16).cpu().numpy().view("uint16")

@@ -75,3 +75,31 @@ def test_requant_extreme_block_scales(fmt):
     oc, os_ = oracle.requant_fp8_mx(codes.numpy(), s.numpy(), 128, 128, fmt)
     assert np.array_equal(out["codes"].cpu().numpy(), oc)
     assert np.array_equal(out["scales"].cpu().numpy(), os_)
+
+
+def check_requant_sampled_rows(codes, bs, out, fmt, seed=8, n_rows=40):
+    """Sampled output rows against the oracle.  A row's MX codes depend only
+    on its source row and that row's block scales, so the sampled source
+    rows form one small source whose every row is its own block row
+    (brows = 1, the original 128-column blocks)."""
+    rows = codes.shape[0]
+    rng = np.random.default_rng(seed)
+    sample = sorted(set(rng.integers(0, rows, n_rows).tolist()) | {0, rows - 1})
+    src = codes[sample].cpu().numpy()
+    sc = bs[[r // 128 for r in sample]].cpu().numpy()
+    oc, os_ = oracle.requant_fp8_mx(src, sc, 1, 128, fmt)
+    assert np.array_equal(out["codes"][sample].cpu().numpy(), oc)
+    assert np.array_equal(out["scales"][sample].cpu().numpy(), os_)
+
+
+def test_full_size_requant_sampled_rows():
+    """The benchmark's launches at full size: the gate_up [512 * 1536, 2048]
+    and down [512 * 2048, 768] stacks of a routed layer held as block FP8
+    (128 x 128 source blocks), requantized to MXFP4 with linear scales."""
+    for rows, cols in ((512 * 1536, 2048), (512 * 2048, 768)):
+        codes, bs = workloads.block_fp8_stack(rows, cols, device="cuda")
+        out = mxq.requant_fp8_mx(codes, bs, 128, 128, "mxfp4")
+        torch.cuda.synchronize()
+        assert int(out["status"].item()) == 0
+        check_requant_sampled_rows(codes, bs, out, "mxfp4")
+        del codes, bs, out
