@@ -109,3 +109,24 @@ def test_ties_and_unfiltered_weights_take_the_binary64_search(kind):
          "huge": torch.full((16,), 2.0 ** 60),
          "gamma": torch.distributions.Gamma(torch.tensor(0.5), torch.tensor(1.0)).sample((16,))}[kind]
     _check(x.cuda(), h.float().contiguous())
+
+
+def test_full_size_layer_sampled_experts():
+    """The benchmark's launch at full size: gate_up [512, 1536, 2048] and
+    down [512, 2048, 768], each stack with one row of per-channel weights
+    (the mean squared activation over a 4096-token tile).  Groups are
+    experts, so an expert's slab quantizes alone exactly as inside its
+    stack: sampled experts are checked against the oracle."""
+    gu, dn, _ = workloads.full_moe_layer(seed=0, device="cuda")
+    for x in (gu, dn):
+        G, R, C = x.shape
+        a = workloads.activation_tile(4096, seed=7, hidden=C).float()
+        h = (a * a).mean(0).contiguous()
+        out = mxq.quantize_nvfp4_weighted(x, h.cuda())
+        torch.cuda.synchronize()
+        assert int(out["status"].item()) == 0
+        for e in (0, 300, G - 1):
+            c, s, s2 = oracle.quantize_nvfp4_weighted(workloads.bf16_bits(x[e:e + 1]), h.numpy())
+            assert np.array_equal(out["codes"][e].cpu().numpy(), c[0]), e
+            assert np.array_equal(out["scales"][e].cpu().numpy(), s[0]), e
+            assert out["s2"][e].cpu().numpy().view(np.uint32) == s2.view(np.uint32)[0], e
