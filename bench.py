@@ -382,7 +382,7 @@ def run_reference(args, rank, world):
     return 0
 
 
-# ------------------------------------------------------------------ main --
+# ------------------------------------------------------- other workloads --
 REQ_BYTES = 1.0 + 0.5 + 1.0 / 32    # read E4M3, write E2M1 codes + UE8M0 scales (block scales ~0)
 
 
@@ -922,6 +922,7 @@ def run_act(args, device):
     return result
 
 
+# ------------------------------------------------------------------ main --
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
