@@ -282,7 +282,10 @@ MXQ_API mxq_status mxq_quantize_act(const uint16_t *tokens, int64_t T, int64_t h
  *            for MX pass n_tensors when the stack was quantized as one
  *            matrix, 1 when each tensor was).
  *   sum_sq_err, sum_sq_ref   out, fp64 [n_tensors]: sum (x - deq)^2 and
- *            sum x^2 with deq = RN32((q * D) * s2) (NVFP4) or q * 2^e (MX).
+ *            sum x^2 with deq = q * D * s2 (NVFP4) or q * 2^e (MX); each
+ *            x - deq is rounded once to fp32 and the squares are summed in
+ *            fp32 runs of 8 and fp64 across blocks, so both sums lie within
+ *            11 * 2^-24 (6.6e-7) relative of the exact ones.
  *   relerr   out, nullable, fp64 [n_tensors]: sqrt(err) / sqrt(ref)
  *            (0 when both are 0).
  *   workspace: mxq_workspace_bytes(MXQ_OP_DEQUANT_RELERR, n_tensors, rows, cols).

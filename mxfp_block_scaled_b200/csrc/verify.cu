@@ -4,9 +4,15 @@
 // of the quantized experts against the bf16 source, per tensor, mean and
 // max over the census; azampatti/Qwen3.8-Flash-Next-FP4-Local-AZ, "The
 // shared expert": error of the MXFP8 tensors against the bf16 master):
-//   deq_i = RN32((q_i * D) * s2)   NVFP4 (q_i * D is exact in f16)
-//   deq_i = q_i * 2^e              MXFP4 / MXFP8 (exact)
-//   err_t = sum (x_i - deq_i)^2, ref_t = sum x_i^2 per tensor t.
+//   deq_i = (q_i * D) * s2         NVFP4 (q_i * D is exact in f16)
+//   deq_i = q_i * 2^e              MXFP4 / MXFP8 (exact in fp32)
+//   err_t = sum (x_i - deq_i)^2, ref_t = sum x_i^2 per tensor t,
+// with e_i = RN32(x_i - deq_i) rounded once (for NVFP4 one FMA of the exact
+// q_i * D with -s2), so each e_i^2 is within 2^-23 of its exact value.
+// Squares are added by fp32 FMAs into pairs of partial sums of 8 terms
+// (one pair per NVFP4 block, two per MX block), each pair added once in
+// fp32 and then in fp64: err_t is within 11 * 2^-24 (6.6e-7) of the exact
+// sum and ref_t within 9 * 2^-24, whatever the data.
 //
 // Fixed summation order: every tensor is cut into chunks of kVerifyChunk
 // elements; one CTA reduces one chunk with a fixed thread -> element map,
@@ -34,7 +40,7 @@ __device__ __forceinline__ void nvfp4_block_sq(uint4 v0, uint4 v1, uint2 c, uint
     const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
     const uint32_t dh = e4m3x2_to_f16x2(sbyte);          // D in the low half
     const uint32_t dd = __byte_perm(dh, 0, 0x1010);      // D in both halves
-    const float2 s22 = make_float2(s2, s2);
+    const float2 s22 = make_float2(-s2, -s2);
     float2 e2 = make_float2(0.f, 0.f), r2 = make_float2(0.f, 0.f);
     uint32_t q[8];
     e2m1x8_to_f16x2(c.x, *reinterpret_cast<uint32_t(*)[4]>(&q[0]));
@@ -42,8 +48,10 @@ __device__ __forceinline__ void nvfp4_block_sq(uint4 v0, uint4 v1, uint2 c, uint
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         const float2 qd = f16x2_to_float2(hmul2_bits(q[j], dd));   // q * D, exact
-        const float2 deq = __fmul2_rn(qd, s22);
-        accum_sq(make_float2(bf16_lo(w[j]), bf16_hi(w[j])), deq, e2, r2);
+        const float2 x = make_float2(bf16_lo(w[j]), bf16_hi(w[j]));
+        const float2 e = __ffma2_rn(qd, s22, x);                    // RN32(x - q D s2)
+        e2 = __ffma2_rn(e, e, e2);
+        r2 = __ffma2_rn(x, x, r2);
     }
     err += (double)__fadd_rn(e2.x, e2.y);
     ref += (double)__fadd_rn(r2.x, r2.y);
@@ -71,8 +79,14 @@ __device__ __forceinline__ void mx_block_sq(const uint4 (&v)[4], const uint32_t 
         const uint32_t qh = (FMT == MXQ_FMT_MXFP8)
                                 ? e4m3x2_to_f16x2(j & 1 ? (cw[j >> 1] >> 16) : cw[j >> 1])
                                 : q4[j];
-        const float2 deq = __fmul2_rn(f16x2_to_float2(qh), sc2);
+        const float2 deq = __fmul2_rn(f16x2_to_float2(qh), sc2);   // exact
         accum_sq(make_float2(bf16_lo(w[j]), bf16_hi(w[j])), deq, e2, r2);
+        if (j == 7) {   // each fp32 partial sums at most 8 squares, as for NVFP4
+            err += (double)__fadd_rn(e2.x, e2.y);
+            ref += (double)__fadd_rn(r2.x, r2.y);
+            e2 = make_float2(0.f, 0.f);
+            r2 = make_float2(0.f, 0.f);
+        }
     }
     err += (double)__fadd_rn(e2.x, e2.y);
     ref += (double)__fadd_rn(r2.x, r2.y);

@@ -22,25 +22,7 @@ import numpy as np
 import torch
 
 from oracle import micro
-
-
-def rn32(q):
-    """Round a rational to the nearest fp32 (ties to even), as a Fraction.
-    Normal range only (the fast path keeps every operand there)."""
-    if q == 0:
-        return F(0)
-    sign = -1 if q < 0 else 1
-    a = abs(q)
-    e = a.numerator.bit_length() - a.denominator.bit_length()
-    if F(2) ** e > a:
-        e -= 1
-    assert -126 <= e <= 127
-    m = a / F(2) ** (e - 23)                    # in [2^23, 2^24)
-    n = m.numerator // m.denominator
-    r = m - n
-    if r > F(1, 2) or (r == F(1, 2) and n % 2 == 1):
-        n += 1
-    return sign * F(n) * F(2) ** (e - 23)
+from exact_fp import rn32
 
 
 def plan_sums(xs, s2, M):
