@@ -337,15 +337,6 @@ int oracle_quantize_mx(const uint16_t *x, int64_t rows, int64_t cols, int fmt,
     return 0;
 }
 
-/* Dequantize and measure the relative error of every unstacked tensor
- * [P3 metric table: relative error of quantized experts vs the bf16
- * source; P2 "The shared expert": error against the bf16 master].
- *   tensors t = 0..n_tensors-1, each [rows, cols], stored back to back;
- *   NVFP4 (fmt 0): deq = q * D * s2[t / tensors_per_scale] (so the gate
- *   and up halves of a fused slab read the same weight_scale_2);
- *   MXFP4 / MXFP8: deq = q * 2^(b - 127).
- * sum_sq_err[t] = sum (x - deq)^2, sum_sq_ref[t] = sum x^2, both as
- * binary64 sums in element order.  Returns 0 or -1. */
 /* Codes of one NVFP4 block for a given E4M3 scale code (the value half of
  * nvfp4_plan): d = RN32(D * s2), code_i = E2M1(RN32(x_i / d)); all codes 0
  * when D or d is 0. */
@@ -509,6 +500,15 @@ int oracle_requant_fp8_mx(const uint8_t *fp8, const float *bscale, int64_t rows,
     return 0;
 }
 
+/* Dequantize and measure the relative error of every unstacked tensor
+ * [P3 metric table: relative error of quantized experts vs the bf16
+ * source; P2 "The shared expert": error against the bf16 master].
+ *   tensors t = 0..n_tensors-1, each [rows, cols], stored back to back;
+ *   NVFP4 (fmt 0): deq = q * D * s2[t / tensors_per_scale] (so the gate
+ *   and up halves of a fused slab read the same weight_scale_2);
+ *   MXFP4 / MXFP8: deq = q * 2^(b - 127).
+ * sum_sq_err[t] = sum (x - deq)^2, sum_sq_ref[t] = sum x^2, both as
+ * binary64 sums in element order.  Returns 0 or -1. */
 int oracle_dequant_relerr(const uint16_t *x, const uint8_t *codes,
                           const uint8_t *scales, const float *s2, int fmt,
                           int64_t n_tensors, int64_t rows, int64_t cols,
