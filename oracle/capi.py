@@ -39,33 +39,39 @@ def lib():
     global _lib
     if _lib is None:
         build()
-        L = ctypes.CDLL(_LIB)
-        d, u, i, i64, vp = (ctypes.c_double, ctypes.c_uint, ctypes.c_int,
-                            ctypes.c_int64, ctypes.c_void_p)
-        L.oracle_e2m1_value.restype = d
-        L.oracle_e2m1_value.argtypes = [u]
-        L.oracle_e4m3_value.restype = d
-        L.oracle_e4m3_value.argtypes = [u]
-        L.oracle_ue8m0_value.restype = d
-        L.oracle_ue8m0_value.argtypes = [u]
-        L.oracle_e2m1_encode.restype = u
-        L.oracle_e2m1_encode.argtypes = [d]
-        L.oracle_e4m3_encode.restype = u
-        L.oracle_e4m3_encode.argtypes = [d]
-        L.oracle_mx_exponent.restype = i
-        L.oracle_mx_exponent.argtypes = [d, d]
-        L.oracle_quantize_nvfp4.restype = i
-        L.oracle_quantize_nvfp4.argtypes = [vp, i64, i64, i64, i, d, vp, vp, vp, vp]
-        L.oracle_quantize_mx.restype = i
-        L.oracle_quantize_mx.argtypes = [vp, i64, i64, i, vp, vp]
-        L.oracle_quantize_nvfp4_weighted.restype = i
-        L.oracle_quantize_nvfp4_weighted.argtypes = [vp, i64, i64, i64, vp, i64, vp, vp, vp]
-        L.oracle_requant_fp8_mx.restype = i
-        L.oracle_requant_fp8_mx.argtypes = [vp, vp, i64, i64, i64, i64, i, vp, vp]
-        L.oracle_dequant_relerr.restype = i
-        L.oracle_dequant_relerr.argtypes = [vp, vp, vp, vp, i, i64, i64, i64, i64, vp, vp]
-        _lib = L
+        _lib = load_library(_LIB)
     return _lib
+
+
+def load_library(path):
+    """Load a build of mxq_oracle.c and declare its signatures (the mutation
+    tests load deliberately broken copies this way)."""
+    L = ctypes.CDLL(path)
+    d, u, i, i64, vp = (ctypes.c_double, ctypes.c_uint, ctypes.c_int,
+                        ctypes.c_int64, ctypes.c_void_p)
+    L.oracle_e2m1_value.restype = d
+    L.oracle_e2m1_value.argtypes = [u]
+    L.oracle_e4m3_value.restype = d
+    L.oracle_e4m3_value.argtypes = [u]
+    L.oracle_ue8m0_value.restype = d
+    L.oracle_ue8m0_value.argtypes = [u]
+    L.oracle_e2m1_encode.restype = u
+    L.oracle_e2m1_encode.argtypes = [d]
+    L.oracle_e4m3_encode.restype = u
+    L.oracle_e4m3_encode.argtypes = [d]
+    L.oracle_mx_exponent.restype = i
+    L.oracle_mx_exponent.argtypes = [d, d]
+    L.oracle_quantize_nvfp4.restype = i
+    L.oracle_quantize_nvfp4.argtypes = [vp, i64, i64, i64, i, d, vp, vp, vp, vp]
+    L.oracle_quantize_mx.restype = i
+    L.oracle_quantize_mx.argtypes = [vp, i64, i64, i, vp, vp]
+    L.oracle_quantize_nvfp4_weighted.restype = i
+    L.oracle_quantize_nvfp4_weighted.argtypes = [vp, i64, i64, i64, vp, i64, vp, vp, vp]
+    L.oracle_requant_fp8_mx.restype = i
+    L.oracle_requant_fp8_mx.argtypes = [vp, vp, i64, i64, i64, i64, i, vp, vp]
+    L.oracle_dequant_relerr.restype = i
+    L.oracle_dequant_relerr.argtypes = [vp, vp, vp, vp, i, i64, i64, i64, i64, vp, vp]
+    return L
 
 
 def _ptr(a):

@@ -237,3 +237,23 @@ def test_exact_decision_values_match_rational_sse(orc):
         if e6 != 0 and abs(F(e4 - e6) / e6) < F(1, 50):
             found += 1
     assert found > 0
+
+
+def test_block_scale_divides_the_amax_once(orc):
+    """Reading of the plans' order of operations: t = RN32(amax_b / RN32(M s2)),
+    one rounded divisor and one division.  In the second block below (amax_b
+    1.0652e-8 in a group of amax 7.2718e-6) that gives t just above an E4M3
+    rounding tie, so scale code 51; the other order, RN32(RN32(amax_b / M) /
+    s2), lands exactly on the tie and would give the even code 50."""
+    amax_g, a = np.float32(7.271766662597656e-06), np.float32(1.0652001947164536e-08)
+    xf = np.zeros((1, 1, 32), np.float32)
+    xf[0, 0, 0] = amax_g
+    xf[0, 0, 16] = a
+    x = bits_of(xf)
+    _, s, s2, _ = orc.quantize_nvfp4(x, mode=0)
+    assert s2[0] == micro.global_scale(amax_g)
+    block = [np.float32(v) for v in xf[0, 0, 16:]]
+    sc, _, _ = micro.plan(block, s2[0], 6)
+    assert s.reshape(-1)[1] == sc == 51
+    other = micro.f32(micro.f32(a / micro.f32(6.0)) / s2[0])
+    assert micro.e4m3_encode(other) == 50
