@@ -1,9 +1,10 @@
 """Mutation check of the oracle's pins.  Each mutant below is one plausible
-mistake (a wrong tie rule, index, sign, operand, constant or comparison)
-planted in a copy of oracle/mxq_oracle.c on the CPU; the copy is built with
-the oracle's own flags and swapped in, and the pins of tests/test_oracle_*.py
-run against it until one fails.  Every mutant must be caught: a mutant that
-survives marks a part of the oracle that no pin fixes."""
+mistake (a wrong tie rule, index, sign, operand, constant, comparison or
+rounding) planted in a copy of oracle/mxq_oracle.c on the CPU; the copy is
+built with the oracle's own flags and swapped in, and the pins of
+tests/test_oracle_*.py run against it until one fails.  Every mutant must be
+caught: a mutant that survives marks a part of the oracle that no pin
+fixes."""
 import importlib
 import subprocess
 
@@ -44,6 +45,11 @@ MUTANTS = [
     ("weighted_ties_to_the_larger_code", "if (w < best_w) {", "if (w <= best_w) {"),
     ("weighted_candidates_stop_short", "for (unsigned sc = lo + 1; sc <= hi; ++sc) {",
      "for (unsigned sc = lo + 1; sc < hi; ++sc) {"),
+    ("s2_by_reciprocal", "float s2 = amax_g / (float)global_div;",
+     "float s2 = amax_g * (float)(1.0 / global_div);"),
+    ("quotient_by_reciprocal", "float y = x[i] / d;", "float y = x[i] * (1.0f / d);"),
+    ("requant_product_not_rounded", ("float w[32];", "w[i] = (float)(oracle_e4m3_value(q) * (double)sc);"),
+     ("double w[32];", "w[i] = oracle_e4m3_value(q) * (double)sc;")),
 ]
 
 
@@ -62,6 +68,7 @@ def _pins():
         lambda: n.test_global_scale_closed_form_and_amax_block_scale(o),
         lambda: n.test_gate_up_share_one_weight_scale_2(o),
         lambda: n.test_block_scale_divides_the_amax_once(o),
+        lambda: n.test_values_take_the_ieee_quotient_at_e2m1_ties(o),
         lambda: n.test_blocks_match_exact_rational_micro_oracle(o, 1.0),
         lambda: n.test_ties_keep_the_amax6_plan(o),
         lambda: n.test_rtn_mode_equals_plan6_of_four_six(o),
@@ -74,6 +81,7 @@ def _pins():
         lambda: m.test_nvfp4_verifier_reads_shared_scale_per_fused_slab(o),
         lambda: m.test_relerr_matches_independent_numpy_dequant(o),
         lambda: r.test_hand_worked_block(),
+        lambda: r.test_dequantized_value_is_rounded_to_fp32_once(),
         lambda: r.test_bf16_exact_case_reduces_to_the_bf16_quantizer("mxfp4"),
         lambda: w.test_matches_the_exact_argmin_away_from_near_ties(),
         lambda: w.test_one_hot_weight_reproduces_that_element_best(0),
@@ -89,9 +97,12 @@ def test_unmutated_oracle_passes_every_pin_used_here():
 def test_mutant_is_caught(tmp_path, monkeypatch, name, old, new):
     with open(capi._SRC) as f:
         src = f.read()
-    assert src.count(old) == 1, "the mutated text must occur exactly once"
+    olds, news = (old, new) if isinstance(old, tuple) else ((old,), (new,))
+    for o, n in zip(olds, news):
+        assert src.count(o) == 1, "the mutated text must occur exactly once"
+        src = src.replace(o, n)
     c_path, so_path = tmp_path / (name + ".c"), tmp_path / (name + ".so")
-    c_path.write_text(src.replace(old, new))
+    c_path.write_text(src)
     subprocess.check_call(["gcc", *capi.CFLAGS, "-o", str(so_path), str(c_path), "-lm"])
     monkeypatch.setattr(capi, "_lib", capi.load_library(str(so_path)))
     for pin in _pins():

@@ -257,3 +257,26 @@ def test_block_scale_divides_the_amax_once(orc):
     assert s.reshape(-1)[1] == sc == 51
     other = micro.f32(micro.f32(a / micro.f32(6.0)) / s2[0])
     assert micro.e4m3_encode(other) == 50
+
+
+def test_values_take_the_ieee_quotient_at_e2m1_ties(orc):
+    """Reading of the value step: code = E2M1(RN32(x / d)) with the IEEE
+    quotient.  With s2 = 2^-10 (group amax 2.625) the second block's scale
+    is D = 1.875 and its values lie exactly on every E2M1 tie (0.25 d,
+    0.75 d, ..., 5 d), each kept at the even code.  RN32(1 / 1.875) exceeds
+    1 / 1.875 by 0.875 * 2^-24 of its value, so a quotient formed as
+    x * RN32(1 / d) moves the ties at 1.25, 2.5 and 5 up to odd codes."""
+    s2 = np.float32(2.0 ** -10)
+    xf = np.zeros((1, 1, 32), np.float32)
+    xf[0, 0, 0] = 2.625                                  # group amax: s2 = 2^-10
+    ties = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]
+    xf[0, 0, 16:24] = np.array([6.0] + ties, np.float32) * np.float32(1.875) * s2
+    x = bits_of(xf)
+    c, s, s2o, _ = orc.quantize_nvfp4(x, mode=0)
+    assert s2o[0] == s2
+    assert micro.e4m3_value(int(s.reshape(-1)[1])) == F(15, 8)
+    block = [np.float32(v) for v in xf[0, 0, 16:]]
+    want, _ = micro.plan_with_scale_code(block, s2, int(s.reshape(-1)[1]))
+    got = [(int(b) >> (4 * h)) & 0xF for b in c.reshape(-1)[8:16] for h in (0, 1)]
+    assert got == list(want)
+    assert got[:8] == [7, 0, 2, 2, 4, 4, 6, 6]           # 6, then every tie at its even code

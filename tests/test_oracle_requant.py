@@ -64,3 +64,25 @@ def test_nan_source_is_rejected():
     q[0, 7] = 0xFF
     with pytest.raises(RuntimeError):
         oracle.requant_fp8_mx(q, np.ones((1, 1), np.float32), 128, 128, "mxfp8")
+
+
+def test_dequantized_value_is_rounded_to_fp32_once():
+    """Reading of the fp32 intermediate: w = RN32(E4M3(code) * scale).  With
+    scale = RN32(1.25 / 1.125), the value 1.125 dequantizes to exactly 1.25
+    after that rounding (an E2M1 tie once the block's exponent is 0, kept at
+    the even code 2), while the unrounded product lies 2^-24 above the tie
+    and would take the odd code 3."""
+    from fractions import Fraction as F
+    from oracle import micro
+    sc = np.float32(np.float32(1.25) / np.float32(1.125))
+    q = np.zeros((1, 32), np.uint8)
+    q[0, 0] = 0x48                                       # 4.0: w = 4.44, block exponent 0
+    q[0, 1] = 0x39                                       # 1.125
+    codes, scales = oracle.requant_fp8_mx(q, np.array([[sc]], np.float32), 128, 128, "mxfp4")
+    assert scales[0, 0] == 127
+    assert codes[0, 0] == 0x6 | (0x2 << 4)               # 4.44 -> 4 (code 6), 1.25 -> 1.0 (code 2)
+    assert np.all(codes[0, 1:] == 0)
+    exact = F(9, 8) * F(float(sc))
+    assert exact - F(5, 4) == F(1, 2 ** 24)
+    assert micro.e2m1_encode(np.float32(exact)) == 2     # rounded once: the tie
+    assert micro.E2M1_GRID[3] - exact < exact - micro.E2M1_GRID[2]   # unrounded: nearer 1.5
