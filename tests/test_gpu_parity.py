@@ -164,6 +164,26 @@ def test_exact_decision_at_ties(shape):
     assert 0 < m4.sum() < m4.size
 
 
+@pytest.mark.parametrize("mode", ["rtn", "four_six"])
+@pytest.mark.parametrize("G,R", [(1, 1), (8, 32)])
+def test_values_on_every_e2m1_tie(G, R, mode):
+    """Blocks whose values lie exactly on every E2M1 tie under a block scale
+    whose reciprocal is not a binary32 value (D = 1.875 with s2 = 2^-10):
+    the quotients must be the correctly rounded ones, so every tie keeps its
+    even code.  One group (the cluster kernel) and eight groups of 512
+    blocks (the single pass)."""
+    s2 = np.float32(2.0 ** -10)
+    ties = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]
+    vals = np.array([6.0] + ties + [-t for t in ties] + [0.0], np.float32) * np.float32(1.875) * s2
+    row = np.zeros(256, np.float32)
+    row[0] = 2.625                                       # group amax: s2 = 2^-10
+    for b in range(1, 16):
+        row[16 * b:16 * b + 16] = np.roll(vals, b)
+    x = torch.from_numpy(np.tile(row, (G, R, 1))).to(torch.bfloat16)
+    _, (_, s, s2o, _) = check_nvfp4(x.cuda(), mode=mode, label="e2m1 ties")
+    assert np.all(s2o == s2)
+
+
 def test_nonfinite_input_sets_status():
     x = torch.randn((2, 4, 32)).to(torch.bfloat16).cuda()
     x[1, 2, 5] = float("inf")

@@ -103,3 +103,24 @@ def test_full_size_requant_sampled_rows():
         assert int(out["status"].item()) == 0
         check_requant_sampled_rows(codes, bs, out, "mxfp4")
         del codes, bs, out
+
+
+def test_dequantized_values_on_e2m1_ties():
+    """Source values whose fp32 dequantization lands exactly on an E2M1 tie
+    (1.125 * RN32(1.25 / 1.125) = 1.25 + 2^-24, rounded once to 1.25): at
+    block exponent 0 (with a 4.0 in the block) and at exponent -2 (alone),
+    each tie keeps its even code, bit-exact with the oracle."""
+    sc = np.float32(np.float32(1.25) / np.float32(1.125))
+    q = np.zeros((128, 64), np.uint8)
+    q[:, 0] = 0x48                                       # 4.0
+    q[:, 1] = 0x39                                       # 1.125
+    q[:, 33] = 0x39
+    bs = np.full((1, 1), sc, np.float32)
+    out = mxq.requant_fp8_mx(torch.from_numpy(q).cuda(), torch.from_numpy(bs).cuda(), 128, 128, "mxfp4")
+    torch.cuda.synchronize()
+    assert int(out["status"].item()) == 0
+    oc, os_ = oracle.requant_fp8_mx(q, bs, 128, 128, "mxfp4")
+    assert np.array_equal(out["codes"].cpu().numpy(), oc)
+    assert np.array_equal(out["scales"].cpu().numpy(), os_)
+    assert oc[0, 0] == 0x26 and os_[0, 0] == 127         # 4.44 -> 4, 1.25 -> 1.0
+    assert oc[0, 16] == 0x60 and os_[0, 1] == 125        # 1.25 * 4 = 5 -> 4 (code 6)
