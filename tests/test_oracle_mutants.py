@@ -111,3 +111,43 @@ def test_mutant_is_caught(tmp_path, monkeypatch, name, old, new):
         except (AssertionError, RuntimeError, ValueError):
             return                                  # caught
     pytest.fail("mutant %s passed every pin" % name)
+
+
+# ---- the tiled scale layout (oracle/layout.py) ----------------------------
+def _rows_one_after_another(r, c, cols):
+    n = -(-cols // 4)
+    return ((r // 128) * n + c // 4) * 512 + 4 * (r % 128) + c % 4
+
+
+def _column_and_slab_swapped(r, c, cols):
+    n, rr = -(-cols // 4), r % 128
+    return ((r // 128) * n + c // 4) * 512 + 16 * (rr % 32) + (rr // 32) + 4 * (c % 4)
+
+
+def _line_and_slab_strides_swapped(r, c, cols):
+    n, rr = -(-cols // 4), r % 128
+    return ((r // 128) * n + c // 4) * 512 + 4 * (rr % 32) + 16 * (rr // 32) + c % 4
+
+
+def _column_tiles_rounded_down(r, c, cols):
+    n, rr = max(cols // 4, 1), r % 128
+    return ((r // 128) * n + c // 4) * 512 + 16 * (rr % 32) + 4 * (rr // 32) + c % 4
+
+
+@pytest.mark.parametrize("mutant", [_rows_one_after_another, _column_and_slab_swapped,
+                                    _line_and_slab_strides_swapped, _column_tiles_rounded_down],
+                         ids=lambda f: f.__name__.strip("_"))
+def test_layout_mutant_is_caught(monkeypatch, mutant):
+    from oracle import layout
+    lay = importlib.import_module("test_oracle_layout")
+    monkeypatch.setattr(layout, "tile_offset", mutant)
+    pins = [lay.test_hand_worked_offsets,
+            lambda: lay.test_bijection_onto_padded_matrix(130, 5),
+            lambda: lay.test_tiles_are_contiguous_submatrices_and_padding_is_zero(128, 4),
+            lay.test_round_trip_and_vectorised_path]
+    for pin in pins:
+        try:
+            pin()
+        except (AssertionError, IndexError):
+            return
+    pytest.fail("layout mutant %s passed every pin" % mutant.__name__)
