@@ -201,9 +201,9 @@ class Layer:
                 rel=torch.empty(nt, dtype=torch.float64, device=device),
             )
 
-    def quantize(self, name):
+    def quantize(self, name, mode="four_six"):
         o = self.out[name]
-        self.mxq.mxq_quantize_nvfp4(o["x"], o["G"], o["R"], o["C"], "four_six", self.layout, o["codes"],
+        self.mxq.mxq_quantize_nvfp4(o["x"], o["G"], o["R"], o["C"], mode, self.layout, o["codes"],
                                     o["scales"], o["s2"], o["mbits"], o["m4"], o["status"], o["wsq"])
 
     def verify(self, name):
@@ -1030,6 +1030,18 @@ def main():
         rel = o["rel"].cpu().numpy()
         quality[name] = {"relerr_mean": float(rel.mean()), "relerr_max": float(rel.max()),
                          "m4_fraction": float(o["m4"].sum().item()) / (o["G"] * o["R"] * o["C"] / 16)}
+    # SSE(chosen) / SSE(RTN) - 1 over the whole layer, after the timed region: the same stacks
+    # quantized with plain amax/6 block scales and verified, into the same buffers
+    try:
+        sse46 = sum(float(layer.out[n]["err"].cpu().numpy().sum()) for n in ("gu", "dn"))
+        for n in ("gu", "dn"):
+            layer.quantize(n, mode="rtn")
+            layer.verify(n)
+        torch.cuda.synchronize()
+        sse_rtn = sum(float(layer.out[n]["err"].cpu().numpy().sum()) for n in ("gu", "dn"))
+        quality["sse_vs_rtn"] = sse46 / sse_rtn - 1.0
+    except Exception as e:          # a quality figure only: the measured line stands without it
+        quality["sse_vs_rtn"] = {"unavailable": str(e)[:200]}
 
     result = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,

@@ -80,6 +80,30 @@ def relerr_census(results):
     return float(rel.mean()), float(rel.max()), int(rel.numel())
 
 
+def sse_vs_rtn(results, results_rtn):
+    """SSE(chosen) / SSE(RTN) - 1 over every unstacked tensor of the given
+    layer results (dabsLabs/Qwen3.8-Flash-Next-NVFP4, "What makes this
+    build different": the 4/6 choice against plain amax/6 block scales;
+    never above 0).  `results` and `results_rtn` are quantize_routed_layer
+    results of the same layers in "four_six" and "rtn" mode; the per-tensor
+    squared-error sums come from the verifier and are added on the host."""
+    def total(res):
+        return sum(float(q[k]["sum_sq_err"].cpu().numpy().sum()) for q in res for k in ("gate_up", "down"))
+    return total(results) / total(results_rtn) - 1.0
+
+
+def m4_fraction(results):
+    """Fraction of NVFP4 blocks that took the M=4 plan (from the per-group
+    M=4 counts)."""
+    m4 = blocks = 0
+    for q in results:
+        for k in ("gate_up", "down"):
+            E = q[k]["codes"].shape[0]
+            m4 += int(q[k]["m4_count"].cpu().numpy()[:E].sum())
+            blocks += q[k]["codes"].numel() // 8
+    return m4 / blocks
+
+
 # ------------------------------------------------ host-resident layers --
 def host_outputs(h_gate_up, h_down):
     """Pinned host buffers for convert_layer_from_host: per stack the codes,

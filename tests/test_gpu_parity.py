@@ -6,7 +6,7 @@ import pytest
 import torch
 
 import oracle
-from mxfp_block_scaled_b200 import mxq, workloads
+from mxfp_block_scaled_b200 import layers, mxq, workloads
 
 pytestmark = pytest.mark.gpu
 
@@ -87,6 +87,37 @@ def test_tiny_moe_layer_four_six_bit_exact_and_verified():
     check_verify(gu, o1["codes"], o1["scales"], o1["s2"], "nvfp4", 2 * E, R // 2, H, tps=2)
     check_verify(dn, o2["codes"], o2["scales"], o2["s2"], "nvfp4", E, dn.shape[1], dn.shape[2])
     assert 0.2 < m4.mean() < 0.7
+
+
+def test_sse_against_rtn_and_m4_fraction_of_a_layer():
+    """The layer figures the pages report beside the relative error:
+    SSE(chosen) / SSE(RTN) - 1 (never above 0) and the M=4 fraction, from
+    the GPU path against the oracle's own quantize + verify in both modes
+    (each error sum within 11 * 2^-24 of the exact one, so 1 + ratio within
+    2e-6)."""
+    gu, dn = workloads.tiny_moe_layer(seed=0)
+    g, d = gu.cuda(), dn.cuda()
+    res46 = layers.quantize_routed_layer(g, d, mode="four_six")
+    resrtn = layers.quantize_routed_layer(g, d, mode="rtn")
+    torch.cuda.synchronize()
+    ratio = layers.sse_vs_rtn([res46], [resrtn])
+    frac = layers.m4_fraction([res46])
+    tot = {0: 0.0, 1: 0.0}
+    m4s = blocks = 0
+    for x, tps in ((gu, 2), (dn, 1)):
+        E, R, C = x.shape
+        xb = bits(x)
+        for mode in (0, 1):
+            c, s, s2, m4 = oracle.quantize_nvfp4(xb, mode=mode)
+            oe, _ = oracle.dequant_relerr(xb, c, s, s2, "nvfp4", E * tps, R // tps, C, tps)
+            tot[mode] += float(oe.sum())
+            if mode == 1:
+                m4s += int(m4.sum())
+                blocks += m4.size
+    want = tot[1] / tot[0] - 1.0
+    assert ratio <= 0.0 and want <= 0.0
+    assert abs((1.0 + ratio) - (1.0 + want)) <= 2e-6 * (1.0 + want)
+    assert frac == m4s / blocks
 
 
 def test_tiny_moe_layer_rtn():
