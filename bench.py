@@ -1031,17 +1031,19 @@ def main():
         quality[name] = {"relerr_mean": float(rel.mean()), "relerr_max": float(rel.max()),
                          "m4_fraction": float(o["m4"].sum().item()) / (o["G"] * o["R"] * o["C"] / 16)}
     # SSE(chosen) / SSE(RTN) - 1 over the whole layer, after the timed region: the same stacks
-    # quantized with plain amax/6 block scales and verified, into the same buffers
-    try:
-        sse46 = sum(float(layer.out[n]["err"].cpu().numpy().sum()) for n in ("gu", "dn"))
-        for n in ("gu", "dn"):
-            layer.quantize(n, mode="rtn")
-            layer.verify(n)
-        torch.cuda.synchronize()
-        sse_rtn = sum(float(layer.out[n]["err"].cpu().numpy().sum()) for n in ("gu", "dn"))
-        quality["sse_vs_rtn"] = sse46 / sse_rtn - 1.0
-    except Exception as e:          # a quality figure only: the measured line stands without it
-        quality["sse_vs_rtn"] = {"unavailable": str(e)[:200]}
+    # quantized with plain amax/6 block scales and verified, into the same buffers (skipped by
+    # profiling runs, whose launch lists cover the measured step alone)
+    if not args.no_extras:
+        try:
+            sse46 = sum(float(layer.out[n]["err"].cpu().numpy().sum()) for n in ("gu", "dn"))
+            for n in ("gu", "dn"):
+                layer.quantize(n, mode="rtn")
+                layer.verify(n)
+            torch.cuda.synchronize()
+            sse_rtn = sum(float(layer.out[n]["err"].cpu().numpy().sum()) for n in ("gu", "dn"))
+            quality["sse_vs_rtn"] = sse46 / sse_rtn - 1.0
+        except Exception as e:      # a quality figure only: the measured line stands without it
+            quality["sse_vs_rtn"] = {"unavailable": str(e)[:200]}
 
     result = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
