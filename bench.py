@@ -750,6 +750,19 @@ def run_mixed8(args, device):
     rel_mx = torch.cat([s.rel for st in mx for s in st]).cpu().numpy()
     m4 = sum(int(lay.out[t]["m4"].sum().item()) for lay in nv for t in ("gu", "dn"))
     nv_blocks = sum(lay.n_elems // 16 for lay in nv)
+    sse_vs_rtn = None
+    if not args.no_extras:          # after the timed region: the NVFP4 layers again with RTN scales
+        try:
+            sse46 = sum(float(lay.out[t]["err"].cpu().numpy().sum()) for lay in nv for t in ("gu", "dn"))
+            for lay in nv:
+                for t in ("gu", "dn"):
+                    lay.quantize(t, mode="rtn")
+                    lay.verify(t)
+            torch.cuda.synchronize()
+            sse_rtn = sum(float(lay.out[t]["err"].cpu().numpy().sum()) for lay in nv for t in ("gu", "dn"))
+            sse_vs_rtn = sse46 / sse_rtn - 1.0
+        except Exception as e:      # a quality figure only
+            sse_vs_rtn = {"unavailable": str(e)[:200]}
     workload = ("mixed-format conversion of 8 full-size routed-expert layers (Student-t tail mix), "
                 "quantize + verify: layers 0,2,4,6 NVFP4 4/6-optimal, layers 1,3,5,7 MXFP4; each "
                 "gate_up bf16 [%d,1536,2048] + down [%d,2048,768]" % (args.experts, args.experts))
@@ -766,7 +779,8 @@ def run_mixed8(args, device):
                    "fraction_of_peak": value / peak, "peak_gbs": peak, "peak_kind": peak_kind,
                    "call_ms": dict(zip(names, call_ms)),
                    "quality": {"nvfp4": {"relerr_mean": float(rel_nv.mean()), "relerr_max": float(rel_nv.max()),
-                                         "tensors": int(rel_nv.size), "m4_fraction": m4 / nv_blocks},
+                                         "tensors": int(rel_nv.size), "m4_fraction": m4 / nv_blocks,
+                                         "sse_vs_rtn": sse_vs_rtn},
                                "mxfp4": {"relerr_mean": float(rel_mx.mean()), "relerr_max": float(rel_mx.max()),
                                          "tensors": int(rel_mx.size)}}},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
