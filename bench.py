@@ -223,6 +223,25 @@ class Layer:
                 events[i][1].record()
 
 
+def nvfp4_sse_vs_rtn(lays):
+    """SSE(chosen) / SSE(RTN) - 1 over Layer objects whose buffers hold their
+    4/6 results: the stacks are quantized again with plain amax/6 block
+    scales and verified into the same buffers, so call it after everything
+    that reads the 4/6 outputs.  A quality figure only: a failure is
+    reported, not raised."""
+    try:
+        sse46 = sum(float(lay.out[t]["err"].cpu().numpy().sum()) for lay in lays for t in ("gu", "dn"))
+        for lay in lays:
+            for t in ("gu", "dn"):
+                lay.quantize(t, mode="rtn")
+                lay.verify(t)
+        torch.cuda.synchronize()
+        sse_rtn = sum(float(lay.out[t]["err"].cpu().numpy().sum()) for lay in lays for t in ("gu", "dn"))
+        return sse46 / sse_rtn - 1.0
+    except Exception as e:
+        return {"unavailable": str(e)[:200]}
+
+
 def run_cpu_baseline(layer, budget_s=20.0):
     """The oracle as it stands, single-threaded on the host, on whole
     experts of the same layer until about budget_s of CPU work."""
@@ -750,19 +769,8 @@ def run_mixed8(args, device):
     rel_mx = torch.cat([s.rel for st in mx for s in st]).cpu().numpy()
     m4 = sum(int(lay.out[t]["m4"].sum().item()) for lay in nv for t in ("gu", "dn"))
     nv_blocks = sum(lay.n_elems // 16 for lay in nv)
-    sse_vs_rtn = None
-    if not args.no_extras:          # after the timed region: the NVFP4 layers again with RTN scales
-        try:
-            sse46 = sum(float(lay.out[t]["err"].cpu().numpy().sum()) for lay in nv for t in ("gu", "dn"))
-            for lay in nv:
-                for t in ("gu", "dn"):
-                    lay.quantize(t, mode="rtn")
-                    lay.verify(t)
-            torch.cuda.synchronize()
-            sse_rtn = sum(float(lay.out[t]["err"].cpu().numpy().sum()) for lay in nv for t in ("gu", "dn"))
-            sse_vs_rtn = sse46 / sse_rtn - 1.0
-        except Exception as e:      # a quality figure only
-            sse_vs_rtn = {"unavailable": str(e)[:200]}
+    # after the timed region (not in profiling runs): the NVFP4 layers again with RTN scales
+    sse_vs_rtn = None if args.no_extras else nvfp4_sse_vs_rtn(nv)
     workload = ("mixed-format conversion of 8 full-size routed-expert layers (Student-t tail mix), "
                 "quantize + verify: layers 0,2,4,6 NVFP4 4/6-optimal, layers 1,3,5,7 MXFP4; each "
                 "gate_up bf16 [%d,1536,2048] + down [%d,2048,768]" % (args.experts, args.experts))
@@ -1044,20 +1052,10 @@ def main():
         rel = o["rel"].cpu().numpy()
         quality[name] = {"relerr_mean": float(rel.mean()), "relerr_max": float(rel.max()),
                          "m4_fraction": float(o["m4"].sum().item()) / (o["G"] * o["R"] * o["C"] / 16)}
-    # SSE(chosen) / SSE(RTN) - 1 over the whole layer, after the timed region: the same stacks
-    # quantized with plain amax/6 block scales and verified, into the same buffers (skipped by
+    # SSE(chosen) / SSE(RTN) - 1 over the whole layer, after the timed region (skipped by
     # profiling runs, whose launch lists cover the measured step alone)
     if not args.no_extras:
-        try:
-            sse46 = sum(float(layer.out[n]["err"].cpu().numpy().sum()) for n in ("gu", "dn"))
-            for n in ("gu", "dn"):
-                layer.quantize(n, mode="rtn")
-                layer.verify(n)
-            torch.cuda.synchronize()
-            sse_rtn = sum(float(layer.out[n]["err"].cpu().numpy().sum()) for n in ("gu", "dn"))
-            quality["sse_vs_rtn"] = sse46 / sse_rtn - 1.0
-        except Exception as e:      # a quality figure only: the measured line stands without it
-            quality["sse_vs_rtn"] = {"unavailable": str(e)[:200]}
+        quality["sse_vs_rtn"] = nvfp4_sse_vs_rtn([layer])
 
     result = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
