@@ -69,3 +69,32 @@ def test_mixed_format_layers_and_bytes():
     n = 512 * 1536 * 2048 + 512 * 2048 * 768
     step = sum(bench.mixed_bytes_per_layer(f, n) for f in bench.MIXED_FORMATS)
     assert step == 4 * n * (5.125 + 5.0625)          # about 98.45 GB per step
+
+
+def test_sse_vs_rtn_pass(monkeypatch):
+    import torch
+    monkeypatch.setattr(bench.torch.cuda, "synchronize", lambda *a: None)
+
+    class FakeLayer:
+        """err holds the 4/6 sums until the RTN quantize + verify rewrites them."""
+        def __init__(self, e46, ertn):
+            self.out = {t: {"err": torch.tensor(e46[t], dtype=torch.float64)} for t in ("gu", "dn")}
+            self.ertn, self.mode = ertn, None
+
+        def quantize(self, t, mode="four_six"):
+            self.mode = mode
+
+        def verify(self, t):
+            assert self.mode == "rtn"
+            self.out[t]["err"] = torch.tensor(self.ertn[t], dtype=torch.float64)
+
+    a = FakeLayer({"gu": [1.0, 2.0], "dn": [1.0]}, {"gu": [2.0, 2.0], "dn": [4.0]})
+    b = FakeLayer({"gu": [0.5], "dn": [0.5]}, {"gu": [1.0], "dn": [1.0]})
+    assert abs(bench.nvfp4_sse_vs_rtn([a, b]) - (5.0 / 10.0 - 1.0)) < 1e-15
+
+    class Broken(FakeLayer):
+        def verify(self, t):
+            raise RuntimeError("device status 0x2")
+
+    r = bench.nvfp4_sse_vs_rtn([Broken({"gu": [1.0], "dn": [1.0]}, {})])
+    assert "unavailable" in r and "0x2" in r["unavailable"]
