@@ -1,4 +1,17 @@
 // weighted.cu -- NVFP4 with a weighted-SSE block-scale search (sm_100a).
+//
+// Method (josch15366/Qwen3.8-Flash-Next-NVFP4-LocalHessian-Experts, "What is
+// different about it": block scales chosen by a Hessian-weighted search
+// instead of the plain amax / MSE sweep; no formula is given).  Readings:
+// per-input-channel weights h >= 0 supplied by the caller (a diagonal
+// Hessian estimate); per block, every E4M3 scale code from the amax/6
+// plan's code to the four-over-six plan's code is a candidate; each
+// candidate's codes follow from its scale as in the 4/6 plans; the
+// objective sum h (x - q D s2)^2 is the binary64 sum in element order, the
+// lowest value wins and ties go to the smaller code.  The kernel scores
+// candidates in fp32 with a certified error bound and runs the binary64
+// procedure only where the bound cannot separate the best two, so its
+// choice is the binary64 argmin.
 #include "nvfp4_block.cuh"
 
 namespace mxq {
