@@ -16,9 +16,11 @@ from .capi import (  # noqa: F401
     e4m3_encode,
     mx_exponent,
     quantize_nvfp4,
+    quantize_nvfp4_s2,
     quantize_nvfp4_weighted,
     quantize_mx,
     requant_fp8_mx,
     dequant_relerr,
     relerr_from_sums,
+    census,
 )

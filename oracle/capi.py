@@ -63,6 +63,8 @@ def load_library(path):
     L.oracle_mx_exponent.argtypes = [d, d]
     L.oracle_quantize_nvfp4.restype = i
     L.oracle_quantize_nvfp4.argtypes = [vp, i64, i64, i64, i, d, vp, vp, vp, vp]
+    L.oracle_quantize_nvfp4_s2.restype = i
+    L.oracle_quantize_nvfp4_s2.argtypes = [vp, i64, i64, i64, i, vp, vp, vp, vp]
     L.oracle_quantize_mx.restype = i
     L.oracle_quantize_mx.argtypes = [vp, i64, i64, i, vp, vp]
     L.oracle_quantize_nvfp4_weighted.restype = i
@@ -123,6 +125,22 @@ def quantize_nvfp4(x_bits, mode=1, global_div=GLOBAL_DIVISOR):
     if rc != 0:
         raise RuntimeError("oracle_quantize_nvfp4 failed: %d" % rc)
     return codes, scales, s2, m4
+
+
+def quantize_nvfp4_s2(x_bits, s2_in, mode=1):
+    """x_bits: uint16 [G, R, C]; s2_in: float32 [G] caller-given global
+    scales.  Returns codes [G,R,C/2], scales [G,R,C/16], m4 [G, R*C/16]."""
+    x = _as_bits(x_bits)
+    G, R, C = x.shape
+    s2a = np.ascontiguousarray(s2_in, np.float32)
+    codes = np.zeros((G, R, C // 2), np.uint8)
+    scales = np.zeros((G, R, C // 16), np.uint8)
+    m4 = np.zeros((G, R * C // 16), np.uint8)
+    rc = lib().oracle_quantize_nvfp4_s2(_ptr(x), G, R, C, int(mode), _ptr(s2a), _ptr(codes),
+                                        _ptr(scales), _ptr(m4))
+    if rc != 0:
+        raise RuntimeError("oracle_quantize_nvfp4_s2 failed: %d" % rc)
+    return codes, scales, m4
 
 
 def quantize_mx(x_bits, fmt):
@@ -200,4 +218,32 @@ def relerr_from_sums(err, ref):
     nz = ref > 0
     out[nz] = np.sqrt(err[nz]) / np.sqrt(ref[nz])
     out[(~nz) & (err > 0)] = np.inf
+    return out
+
+
+def census(err, ref, err_rtn=None, m4_blocks=0, blocks=0):
+    """The census figures of a set of tensors, by their definitions
+    (dabsLabs/Qwen3.8-Flash-Next-NVFP4, metric table: mean and max relative
+    error over the tensors; "What makes this build different": total squared
+    error against plain RTN, share of 16-blocks that took M=4), from the
+    oracle's per-tensor sums: plain binary64 sums in tensor order.
+    Returns a dict with mean_relerr, max_relerr, n_tensors, sum_sq_err,
+    sum_sq_ref, sse_vs_rtn (None without err_rtn) and m4_fraction."""
+    err = [float(v) for v in np.asarray(err, np.float64).reshape(-1)]
+    ref = [float(v) for v in np.asarray(ref, np.float64).reshape(-1)]
+    rel = [float(v) for v in relerr_from_sums(err, ref)]
+    n = len(rel)
+    tot_err = tot_ref = tot_rel = 0.0
+    for k in range(n):
+        tot_err += err[k]
+        tot_ref += ref[k]
+        tot_rel += rel[k]
+    out = {"n_tensors": n, "mean_relerr": tot_rel / n if n else 0.0, "max_relerr": max(rel) if n else 0.0,
+           "sum_sq_err": tot_err, "sum_sq_ref": tot_ref, "sse_vs_rtn": None,
+           "m4_fraction": m4_blocks / blocks if blocks else 0.0}
+    if err_rtn is not None:
+        tot_rtn = 0.0
+        for v in np.asarray(err_rtn, np.float64).reshape(-1):
+            tot_rtn += float(v)
+        out["sse_vs_rtn"] = tot_err / tot_rtn - 1.0
     return out

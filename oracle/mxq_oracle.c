@@ -222,6 +222,49 @@ static int nvfp4_plan(const float x[16], float amax_b, float s2, float M,
     return ok ? 0 : -2;
 }
 
+/* The blocks of one NVFP4 group with global scale s2 [P3 "What makes this
+ * build different"]: per block of 16 the amax/6 plan and, in 4/6 mode
+ * (mode 1), the four-over-six plan; the M=4 plan wins only when its exact
+ * squared error is strictly lower, so ties keep the amax/6 plan and the
+ * result equals plain RTN unless it is strictly better.  xg holds the
+ * group's nblk * 16 bf16 values, g is the group's index in the stack (the
+ * outputs are written at its blocks).  Returns 0 or -2. */
+static int nvfp4_group(const uint16_t *xg, int64_t nblk, int64_t g, float s2, int mode,
+                       uint8_t *codes, uint8_t *scales, uint8_t *m4)
+{
+    int rc = 0;
+    for (int64_t b = 0; b < nblk; ++b) {
+        float xb[16];
+        float amax_b = 0.0f;
+        for (int i = 0; i < 16; ++i) {
+            xb[i] = bf16_to_float(xg[b * 16 + i]);
+            if (fabsf(xb[i]) > amax_b)
+                amax_b = fabsf(xb[i]);
+        }
+        unsigned sc6, sc4 = 0;
+        uint8_t c6[16], c4[16];
+        double G6, G4 = 0.0;
+        int r = nvfp4_plan(xb, amax_b, s2, 6.0f, &sc6, c6, &G6);
+        if (r)
+            rc = r;
+        int use4 = 0;
+        if (mode == 1) {
+            r = nvfp4_plan(xb, amax_b, s2, 4.0f, &sc4, c4, &G4);
+            if (r)
+                rc = r;
+            use4 = (G4 < G6);
+        }
+        const uint8_t *c = use4 ? c4 : c6;
+        int64_t gb = g * nblk + b;
+        for (int j = 0; j < 8; ++j)
+            codes[gb * 8 + j] = (uint8_t)((c[2 * j] & 0xF) | ((c[2 * j + 1] & 0xF) << 4));
+        scales[gb] = (uint8_t)(use4 ? sc4 : sc6);
+        if (m4)
+            m4[gb] = (uint8_t)use4;
+    }
+    return rc;
+}
+
 /* NVFP4 quantization of a stack of groups [P1 introduction; P3 "What
  * makes this build different"].
  *   x            bf16 bits, [n_groups, rows, cols] row-major
@@ -234,11 +277,9 @@ static int nvfp4_plan(const float x[16], float amax_b, float s2, float M,
  *   s2_out       [n_groups] fp32 global scale RN32(amax_g / global_div)
  *   m4           nullable, one byte per block: 1 if the M=4 plan won
  * Group = one expert's fused gate_up slab (gate and up share one
- * weight_scale_2), or one down slab, or one activation tile.
- * The M=4 plan wins only when its exact squared error is strictly lower;
- * ties keep the amax/6 plan, so the result equals plain RTN unless it is
- * strictly better.  Returns 0, -1 on bad shape, -2 on a failed
- * exactness premise, -3 on non-finite input. */
+ * weight_scale_2), or one down slab, or one activation tile.  Returns 0,
+ * -1 on bad shape, -2 on a failed exactness premise, -3 on non-finite
+ * input. */
 int oracle_quantize_nvfp4(const uint16_t *x, int64_t n_groups, int64_t rows,
                           int64_t cols, int mode, double global_div,
                           uint8_t *codes, uint8_t *scales, float *s2_out,
@@ -261,35 +302,38 @@ int oracle_quantize_nvfp4(const uint16_t *x, int64_t n_groups, int64_t rows,
         }
         float s2 = amax_g / (float)global_div;
         s2_out[g] = s2;
-        for (int64_t b = 0; b < nblk; ++b) {
-            float xb[16];
-            float amax_b = 0.0f;
-            for (int i = 0; i < 16; ++i) {
-                xb[i] = bf16_to_float(xg[b * 16 + i]);
-                if (fabsf(xb[i]) > amax_b)
-                    amax_b = fabsf(xb[i]);
-            }
-            unsigned sc6, sc4 = 0;
-            uint8_t c6[16], c4[16];
-            double G6, G4 = 0.0;
-            int r = nvfp4_plan(xb, amax_b, s2, 6.0f, &sc6, c6, &G6);
-            if (r)
-                rc = r;
-            int use4 = 0;
-            if (mode == 1) {
-                r = nvfp4_plan(xb, amax_b, s2, 4.0f, &sc4, c4, &G4);
-                if (r)
-                    rc = r;
-                use4 = (G4 < G6);
-            }
-            const uint8_t *c = use4 ? c4 : c6;
-            int64_t gb = g * nblk + b;
-            for (int j = 0; j < 8; ++j)
-                codes[gb * 8 + j] = (uint8_t)((c[2 * j] & 0xF) | ((c[2 * j + 1] & 0xF) << 4));
-            scales[gb] = (uint8_t)(use4 ? sc4 : sc6);
-            if (m4)
-                m4[gb] = (uint8_t)use4;
-        }
+        int r = nvfp4_group(xg, nblk, g, s2, mode, codes, scales, m4);
+        if (r)
+            rc = r;
+    }
+    return rc;
+}
+
+/* NVFP4 quantization with a caller-given global scale per group [P1
+ * introduction: gate and up share one weight_scale_2, so a caller that holds
+ * them apart passes the scale they share; an activation's input_scale may be
+ * reduced elsewhere].  As oracle_quantize_nvfp4 with s2 = s2_in[g] instead
+ * of RN32(amax_g / 2688).  s2_in must be finite and >= 0.  Returns 0, -1 on
+ * bad shape or scale, -2 on a failed exactness premise, -3 on non-finite
+ * input. */
+int oracle_quantize_nvfp4_s2(const uint16_t *x, int64_t n_groups, int64_t rows,
+                             int64_t cols, int mode, const float *s2_in,
+                             uint8_t *codes, uint8_t *scales, uint8_t *m4)
+{
+    if (n_groups < 0 || rows < 0 || cols < 0 || cols % 16 != 0)
+        return -1;
+    const int64_t gsize = rows * cols;
+    const int64_t nblk = gsize / 16;
+    int rc = 0;
+    for (int64_t g = 0; g < n_groups; ++g) {
+        if (!(s2_in[g] >= 0.0f) || !isfinite(s2_in[g]))
+            return -1;
+        for (int64_t i = 0; i < gsize; ++i)
+            if (!isfinite(bf16_to_float(x[g * gsize + i])))
+                return -3;
+        int r = nvfp4_group(x + g * gsize, nblk, g, s2_in[g], mode, codes, scales, m4);
+        if (r)
+            rc = r;
     }
     return rc;
 }
