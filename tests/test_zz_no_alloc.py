@@ -4,21 +4,18 @@ It serves callers that cannot allocate device memory (engines that reserve
 their whole memory budget up front, code that must not risk the
 synchronisation of a cudaMalloc): its partial sums live in a fixed array in
 the library instead of a caller workspace.  Checked here through the C ABI
-against the workspace-taking verifier on the same inputs, on two calls in a
-row (the second call reuses the array the first one left behind).  This file
-sorts last so that a run stopping at the first failure has run every other
-test first."""
+against the workspace-taking verifier on the same inputs, bit for bit, on
+calls in a row (each reuses the array the one before left behind, filled
+from another input in between).  This file sorts last so that a run
+stopping at the first failure has run every other test first."""
 import ctypes
 
-import numpy as np
 import pytest
 import torch
 
 from mxfp_block_scaled_b200 import mxq, workloads
 
 pytestmark = pytest.mark.gpu
-
-RTOL_STATS = 1e-6
 
 
 @pytest.fixture(scope="module")
@@ -38,31 +35,47 @@ def _stream():
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
 
+def _case(fmt, x, tps):
+    """Quantize x ([G, R, C] bf16 on the device) and return the verifier's
+    arguments for it plus the workspace verifier's results."""
+    G, R, C = x.shape
+    nt, rows = G * tps, R // tps
+    if fmt == "nvfp4":
+        q = mxq.quantize_nvfp4(x, mode="four_six")
+        s2 = q["s2"]
+    else:
+        q = mxq.quantize_mx(x.view(G * R, C), "mxfp8")
+        s2, tps = None, 1
+    want = mxq.dequant_relerr(x, q["codes"], q["scales"], s2, fmt, nt, rows, C, tps)
+    return (x, q["codes"], q["scales"], s2, nt, rows, C, tps), want
+
+
+def _noalloc(lib, fmt, args):
+    x, codes, scales, s2, nt, rows, C, tps = args
+    err = torch.full((nt,), -1.0, dtype=torch.float64, device="cuda")
+    sq = torch.full_like(err, -1.0)
+    rel = torch.full_like(err, -1.0)
+    rc = lib.mxq_dequant_relerr_noalloc(
+        _ptr(x), _ptr(codes), _ptr(scales), _ptr(s2), mxq.FMT[fmt], nt, rows, C, tps,
+        _ptr(err), _ptr(sq), _ptr(rel), _stream())
+    assert rc == 0, rc
+    torch.cuda.synchronize()
+    return err, sq, rel
+
+
 @pytest.mark.parametrize("fmt", ["nvfp4", "mxfp8"])
 def test_noalloc_verifier_matches_workspace_verifier_twice(lib, fmt):
+    """Same kernels, same fixed summation order as the workspace verifier, so
+    the results must be bit-identical, on two calls in a row; between them a
+    call on another input and shape fills the shared array with other
+    partials, and none of them may leak into the next call."""
     gu, dn = workloads.tiny_moe_layer(seed=5)
-    for x, tps in ((gu.cuda(), 2), (dn.cuda(), 1)):
-        G, R, C = x.shape
-        nt, rows = G * tps, R // tps
-        if fmt == "nvfp4":
-            q = mxq.quantize_nvfp4(x, mode="four_six")
-            s2 = q["s2"]
-        else:
-            q = mxq.quantize_mx(x.view(G * R, C), "mxfp8")
-            s2, tps = None, 1
-        ref = mxq.dequant_relerr(x, q["codes"], q["scales"], s2, fmt, nt, rows, C, tps)
-        for _ in range(2):
-            err = torch.full((nt,), -1.0, dtype=torch.float64, device="cuda")
-            sq = torch.full_like(err, -1.0)
-            rel = torch.full_like(err, -1.0)
-            rc = lib.mxq_dequant_relerr_noalloc(
-                _ptr(x), _ptr(q["codes"]), _ptr(q["scales"]), _ptr(s2), mxq.FMT[fmt], nt, rows,
-                C, tps, _ptr(err), _ptr(sq), _ptr(rel), _stream())
-            assert rc == 0, rc
-            torch.cuda.synchronize()
-            for got, want in zip((err, sq, rel), ref):
-                np.testing.assert_allclose(got.cpu().numpy(), want.cpu().numpy(),
-                                           rtol=RTOL_STATS, atol=0)
+    a_args, a_want = _case(fmt, gu.cuda(), 2)
+    b_args, b_want = _case(fmt, (dn.cuda() * 3).contiguous(), 1)
+    for args, want in ((a_args, a_want), (b_args, b_want), (a_args, a_want)):
+        got = _noalloc(lib, fmt, args)
+        for g, w in zip(got, want):
+            assert torch.equal(g, w), (g - w).abs().max().item()
 
 
 def test_noalloc_rejects_requests_beyond_its_array(lib):
