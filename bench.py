@@ -223,21 +223,42 @@ class Layer:
                 events[i][1].record()
 
 
-def nvfp4_sse_vs_rtn(lays):
-    """SSE(chosen) / SSE(RTN) - 1 over Layer objects whose buffers hold their
-    4/6 results: the stacks are quantized again with plain amax/6 block
-    scales and verified into the same buffers, so call it after everything
-    that reads the 4/6 outputs.  A quality figure only: a failure is
-    reported, not raised."""
+def nvfp4_census(lays, with_rtn=True):
+    """The census of Layer objects whose buffers hold their 4/6 results,
+    formed on the device (mxq_census_add): mean / max relative error over the
+    unstacked tensors and the M=4 fraction; with_rtn also SSE(chosen) /
+    SSE(RTN) - 1, for which the stacks are quantized again with plain amax/6
+    block scales and verified into the same buffers (so call it after
+    everything that reads the 4/6 outputs).  A quality figure only: a
+    failure is reported, not raised."""
+    from mxfp_block_scaled_b200 import mxq
     try:
-        sse46 = sum(float(lay.out[t]["err"].cpu().numpy().sum()) for lay in lays for t in ("gu", "dn"))
-        for lay in lays:
+        saved = [{t: (lay.out[t]["err"].clone(), lay.out[t]["rel"].clone(), lay.out[t]["m4"].clone())
+                  for t in ("gu", "dn")} for lay in lays]
+        rtn = None
+        if with_rtn:
+            try:
+                for lay in lays:
+                    for t in ("gu", "dn"):
+                        lay.quantize(t, mode="rtn")
+                        lay.verify(t)
+                torch.cuda.synchronize()
+                rtn = True
+            except Exception as e:
+                rtn = {"unavailable": str(e)[:200]}
+        c = mxq.Census(device=lays[0].gu.device)
+        for lay, sv in zip(lays, saved):
             for t in ("gu", "dn"):
-                lay.quantize(t, mode="rtn")
-                lay.verify(t)
-        torch.cuda.synchronize()
-        sse_rtn = sum(float(lay.out[t]["err"].cpu().numpy().sum()) for lay in lays for t in ("gu", "dn"))
-        return sse46 / sse_rtn - 1.0
+                o = lay.out[t]
+                err, rel, m4 = sv[t]
+                c.add(n_tensors=o["nt"], sum_sq_err=err, sum_sq_ref=o["ref"], relerr=rel,
+                      sum_sq_err_rtn=o["err"] if rtn is True else None, n_groups=o["G"], m4_count=m4,
+                      blocks_per_group=o["R"] * o["C"] // 16)
+        r = c.result()
+        out = {k: r[k] for k in ("mean_relerr", "max_relerr", "n_tensors", "m4_fraction")}
+        if with_rtn:
+            out["sse_vs_rtn"] = r["sse_vs_rtn"] if rtn is True else rtn
+        return out
     except Exception as e:
         return {"unavailable": str(e)[:200]}
 
@@ -765,12 +786,10 @@ def run_mixed8(args, device):
     gu_elems = nv[0].gu.numel()
     achieved = gu_elems * Q_BYTES / (q_ms * 1e-3) / 1e9
     traffic = ncu_traffic_per_launch() if args.experts == EXPERTS and args.layout == "linear" else None
-    rel_nv = torch.cat([lay.out[t]["rel"] for lay in nv for t in ("gu", "dn")]).cpu().numpy()
     rel_mx = torch.cat([s.rel for st in mx for s in st]).cpu().numpy()
-    m4 = sum(int(lay.out[t]["m4"].sum().item()) for lay in nv for t in ("gu", "dn"))
-    nv_blocks = sum(lay.n_elems // 16 for lay in nv)
-    # after the timed region (not in profiling runs): the NVFP4 layers again with RTN scales
-    sse_vs_rtn = None if args.no_extras else nvfp4_sse_vs_rtn(nv)
+    # after the timed region: the census of the NVFP4 layers, and (not in
+    # profiling runs) those layers again with RTN scales for SSE vs RTN
+    nv_census = nvfp4_census(nv, with_rtn=not args.no_extras)
     workload = ("mixed-format conversion of 8 full-size routed-expert layers (Student-t tail mix), "
                 "quantize + verify: layers 0,2,4,6 NVFP4 4/6-optimal, layers 1,3,5,7 MXFP4; each "
                 "gate_up bf16 [%d,1536,2048] + down [%d,2048,768]" % (args.experts, args.experts))
@@ -786,9 +805,7 @@ def run_mixed8(args, device):
                    "l2": "inputs %.1f GB, larger than L2; no flush" % (n_total * 2 / 1e9),
                    "fraction_of_peak": value / peak, "peak_gbs": peak, "peak_kind": peak_kind,
                    "call_ms": dict(zip(names, call_ms)),
-                   "quality": {"nvfp4": {"relerr_mean": float(rel_nv.mean()), "relerr_max": float(rel_nv.max()),
-                                         "tensors": int(rel_nv.size), "m4_fraction": m4 / nv_blocks,
-                                         "sse_vs_rtn": sse_vs_rtn},
+                   "quality": {"nvfp4": nv_census,
                                "mxfp4": {"relerr_mean": float(rel_mx.mean()), "relerr_max": float(rel_mx.max()),
                                          "tensors": int(rel_mx.size)}}},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
@@ -1046,16 +1063,9 @@ def main():
     q_ms = call_ms[0]
     achieved = gu_elems * Q_BYTES / (q_ms * 1e-3) / 1e9
     traffic = ncu_traffic_per_launch() if args.layout == "linear" else None
-    quality = {}
-    for name in ("gu", "dn"):
-        o = layer.out[name]
-        rel = o["rel"].cpu().numpy()
-        quality[name] = {"relerr_mean": float(rel.mean()), "relerr_max": float(rel.max()),
-                         "m4_fraction": float(o["m4"].sum().item()) / (o["G"] * o["R"] * o["C"] / 16)}
-    # SSE(chosen) / SSE(RTN) - 1 over the whole layer, after the timed region (skipped by
-    # profiling runs, whose launch lists cover the measured step alone)
-    if not args.no_extras:
-        quality["sse_vs_rtn"] = nvfp4_sse_vs_rtn([layer])
+    # census of the layer's 1536 tensors, after the timed region; SSE(chosen) / SSE(RTN) - 1
+    # (an RTN pass) is skipped by profiling runs, whose launch lists cover the measured step alone
+    quality = nvfp4_census([layer], with_rtn=not args.no_extras)
 
     result = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,

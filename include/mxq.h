@@ -28,8 +28,10 @@
  *
  * Conventions for every entry point
  *   - All pointers are DEVICE pointers unless stated; the caller owns every
- *     buffer.  The library allocates nothing and keeps no state between
- *     calls, except a per-device cache of the SM count.
+ *     buffer.  The library allocates nothing.  State kept between calls:
+ *     the device address of the fixed scratch array of
+ *     mxq_dequant_relerr_noalloc (per device and context, see there) and the
+ *     one-shot request flag of the test hook in mxq_test.h; nothing else.
  *   - All work is enqueued asynchronously on `stream` (0 = legacy default
  *     stream).  The call returns after enqueueing; results are valid once
  *     the stream has reached that point.
@@ -40,7 +42,8 @@
  *     caller zeroes and reads after synchronising): MXQ_DEV_NONFINITE_INPUT
  *     when an input element is Inf or NaN (outputs are then undefined),
  *     MXQ_DEV_WAIT_TIMEOUT when a bounded inter-CTA wait gave up (outputs
- *     are then undefined).  `status` may be NULL on the MX entry point
+ *     are then undefined), MXQ_DEV_INVALID_SCALE when a caller-given global
+ *     scale is negative or not finite (that group's outputs are undefined).  `status` may be NULL on the MX entry point
  *     only (the check is then skipped); elsewhere it is required.
  *   - Input bf16 data must be 16-byte aligned; code and scale outputs
  *     must be 16-byte aligned; fp32 / fp64 arrays naturally aligned.
@@ -94,6 +97,7 @@ typedef enum mxq_status {
 /* Bits of the device status word. */
 #define MXQ_DEV_NONFINITE_INPUT 0x1u
 #define MXQ_DEV_WAIT_TIMEOUT 0x2u
+#define MXQ_DEV_INVALID_SCALE 0x4u
 
 typedef enum mxq_fmt {
     MXQ_FMT_NVFP4 = 0,
@@ -116,6 +120,31 @@ typedef enum mxq_op {
     MXQ_OP_QUANTIZE_ACT = 1,
     MXQ_OP_DEQUANT_RELERR = 2
 } mxq_op;
+
+/* Census of a conversion, accumulated on the device by mxq_census_add
+ * (device memory, caller-owned, 8-byte aligned; 13 fields of 8 bytes).
+ * Source: dabsLabs/Qwen3.8-Flash-Next-NVFP4, metric table (mean and max
+ * relative error of the quantized expert tensors against the bf16 source,
+ * over the census of 48 x 512 x 3 tensors) and "What makes this build
+ * different" (total squared error of the 4/6 choice against plain RTN block
+ * scales; share of 16-blocks that chose the four-over-six plan). */
+typedef struct mxq_census {
+    double sum_relerr;       /* sum of the tensors' relative errors */
+    double max_relerr;       /* largest relative error (0 before any tensor) */
+    double sum_sq_err;       /* sum over the tensors of sum (x - deq)^2 */
+    double sum_sq_ref;       /* sum over the tensors of sum x^2 */
+    double sum_sq_err_rtn;   /* the same error total of the RTN comparison tensors */
+    uint64_t n_tensors;      /* tensors added */
+    uint64_t n_tensors_rtn;  /* of which added with an RTN counterpart */
+    uint64_t blocks;         /* NVFP4 blocks of the groups added */
+    uint64_t blocks_m4;      /* of which took the M=4 plan */
+    double mean_relerr;      /* sum_relerr / n_tensors (0 when none) */
+    double sse_vs_rtn;       /* sum_sq_err / sum_sq_err_rtn - 1: NaN unless
+                                every tensor came with its RTN counterpart and
+                                that total is > 0 */
+    double m4_fraction;      /* blocks_m4 / blocks (0 when none) */
+    double reserved;         /* 0 */
+} mxq_census;
 
 /* Version of this ABI (major * 10000 + minor * 100 + patch). */
 MXQ_API int mxq_version(void);
@@ -172,6 +201,28 @@ MXQ_API mxq_status mxq_quantize_nvfp4(const uint16_t *x, int64_t n_groups, int64
                               uint8_t *scales, float *s2, uint32_t *mbits,
                               uint32_t *m4_count, uint32_t *status, void *workspace,
                               size_t workspace_bytes, cudaStream_t stream);
+
+/* NVFP4 quantization with a caller-given global scale per group.
+ * Source: josch15366/Qwen3.8-Flash-Next-NVFP4-LocalHessian-Experts,
+ * introduction: gate and up share one weight_scale_2, and an activation's
+ * input_scale is amax / 2688.  This entry point serves callers that hold the
+ * two halves of a shared group apart (gate and up as separate tensors, which
+ * must both use RN32(max(amax_gate, amax_up) / 2688)), or that reduced a
+ * tile's amax elsewhere (a token-sharded activation tile).
+ *   x, n_groups, rows, cols, mode, layout, codes, scales, mbits, m4_count,
+ *            status: as mxq_quantize_nvfp4.
+ *   s2_in    fp32 [n_groups], the global scale of each group, finite and
+ *            >= 0 (a negative or non-finite scale sets
+ *            MXQ_DEV_INVALID_SCALE; s2 = 0 gives all-zero codes and scales).
+ * No workspace: the block quantizer of mxq_quantize_nvfp4 runs with s2 taken
+ * from s2_in instead of RN32(amax_g / 2688), in one read of x.  With s2_in
+ * equal to what mxq_quantize_nvfp4 writes, the outputs are byte-identical to
+ * its outputs. */
+MXQ_API mxq_status mxq_quantize_nvfp4_s2(const uint16_t *x, int64_t n_groups, int64_t rows,
+                                         int64_t cols, const float *s2_in, mxq_scale_mode mode,
+                                         mxq_layout layout, uint8_t *codes, uint8_t *scales,
+                                         uint32_t *mbits, uint32_t *m4_count, uint32_t *status,
+                                         cudaStream_t stream);
 
 /* NVFP4 quantization with a weighted-SSE block-scale search.
  * Source: josch15366/Qwen3.8-Flash-Next-NVFP4-LocalHessian-Experts, "What is
@@ -310,8 +361,11 @@ MXQ_API mxq_status mxq_dequant_relerr(const uint16_t *x, const uint8_t *codes,
  *   example 1024 tensors of 768 x 2048, or 512 of 2048 x 768); larger
  *   requests return MXQ_ERR_WORKSPACE before anything is enqueued.
  *   The first call on a device looks up the array's device address on that
- *   device (cudaGetSymbolAddress) and caches it; make that first call before
- *   any stream capture.  It allocates nothing: no cudaMalloc, no cudaFree.
+ *   device (cudaGetSymbolAddress) and caches it with the id of the device's
+ *   current context; a later call made in another context (after a
+ *   cudaDeviceReset, say) looks it up again.  Make the first call on a
+ *   device, and the first after such a reset, before any stream capture.
+ *   It allocates nothing: no cudaMalloc, no cudaFree.
  *   Every call on a device uses the same array and leaves its last contents
  *   there (each call writes every partial it reads, so nothing needs to
  *   start at zero); calls whose GPU work overlaps in time, on any streams,
@@ -322,6 +376,31 @@ MXQ_API mxq_status mxq_dequant_relerr_noalloc(const uint16_t *x, const uint8_t *
                                               int64_t cols, int64_t tensors_per_scale,
                                               double *sum_sq_err, double *sum_sq_ref,
                                               double *relerr, cudaStream_t stream);
+
+/* Zero a census (enqueued on `stream`).  census: device mxq_census. */
+MXQ_API mxq_status mxq_census_reset(mxq_census *census, cudaStream_t stream);
+
+/* Add one verifier call's per-tensor figures, and one quantizer call's M=4
+ * counts, to a census (see mxq_census for the source passages).
+ *   census          device mxq_census, 8-byte aligned.
+ *   n_tensors       tensors to add (0: none); then sum_sq_err, sum_sq_ref and
+ *                   relerr (fp64 [n_tensors], as mxq_dequant_relerr writes
+ *                   them) are required.
+ *   sum_sq_err_rtn  nullable, fp64 [n_tensors]: the verifier's sum_sq_err of
+ *                   the same tensors quantized with MXQ_SCALE_RTN, for
+ *                   sse_vs_rtn.
+ *   n_groups        groups whose M=4 counts to add (0: none); then m4_count
+ *                   (uint32 [n_groups], as mxq_quantize_nvfp4 writes it) is
+ *                   required and blocks_per_group >= 0 gives their blocks.
+ * One CTA adds the arrays in a fixed order (element i to partial i % 256,
+ * in order, then a fixed tree) and then adds the totals to the census and
+ * recomputes its derived fields, so the same sequence of calls gives the
+ * same bits.  Calls on one census must be ordered (one stream). */
+MXQ_API mxq_status mxq_census_add(mxq_census *census, int64_t n_tensors, const double *sum_sq_err,
+                                  const double *sum_sq_ref, const double *relerr,
+                                  const double *sum_sq_err_rtn, int64_t n_groups,
+                                  const uint32_t *m4_count, int64_t blocks_per_group,
+                                  cudaStream_t stream);
 
 #ifdef __cplusplus
 }

@@ -1,6 +1,6 @@
 // api.cu -- the C ABI declared in include/mxq.h: argument checks,
 // workspace carving and kernel launches.  No allocation, no host-device
-// synchronisation, no state beyond a per-device SM-count cache.
+// synchronisation; no state (the no-alloc verifier keeps its own, in noalloc.cu).
 #include "mxq.h"
 #include "mxq_internal.h"
 
@@ -70,7 +70,7 @@ using namespace mxq;
 
 extern "C" {
 
-int mxq_version(void) { return 10100; }
+int mxq_version(void) { return 10200; }
 
 const char *mxq_status_string(mxq_status s)
 {
@@ -211,9 +211,54 @@ mxq_status mxq_quantize_nvfp4(const uint16_t *x, int64_t n_groups, int64_t rows,
     if (e == cudaSuccess)
         e = launch_group_amax(x, n_groups, nb, amax_bits, status, stream);
     if (e == cudaSuccess)
-        e = launch_nvfp4_quant(x, n_groups, nb, mode == MXQ_SCALE_FOUR_SIX, amax_bits, codes, scales,
+        e = launch_nvfp4_quant(x, n_groups, nb, mode == MXQ_SCALE_FOUR_SIX, amax_bits, nullptr, codes, scales,
                                sl, s2, mbits, mbits_atomic, mode == MXQ_SCALE_FOUR_SIX ? m4_count : nullptr,
-                               stream);
+                               status, stream);
+    return e == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
+}
+
+mxq_status mxq_quantize_nvfp4_s2(const uint16_t *x, int64_t n_groups, int64_t rows, int64_t cols,
+                                 const float *s2_in, mxq_scale_mode mode, mxq_layout layout,
+                                 uint8_t *codes, uint8_t *scales, uint32_t *mbits, uint32_t *m4_count,
+                                 uint32_t *status, cudaStream_t stream)
+{
+    const ApiRange range_("mxq_quantize_nvfp4_s2");
+    if (n_groups < 0 || rows < 0 || cols < 0)
+        return MXQ_ERR_INVALID_ARG;
+    if (mode != MXQ_SCALE_RTN && mode != MXQ_SCALE_FOUR_SIX)
+        return MXQ_ERR_INVALID_ARG;
+    if (!layout_ok(layout))
+        return MXQ_ERR_INVALID_ARG;
+    if (cols % 16 != 0)
+        return MXQ_ERR_SHAPE;
+    int64_t gsize, total;
+    if (!mul_ok(rows, cols, &gsize) || !mul_ok(gsize, n_groups, &total) || total > (INT64_MAX / 4))
+        return MXQ_ERR_SHAPE;
+    const bool swz = layout == MXQ_LAYOUT_SWIZZLED_128X4;
+    if (swz && gsize / 16 > 0x7FFFFFFF)
+        return MXQ_ERR_SHAPE;
+    if (n_groups == 0)
+        return MXQ_OK;
+    if (!x || !s2_in || !codes || !scales || !status)
+        return MXQ_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(scales, 16) || !aligned(s2_in, 4) ||
+        !aligned(status, 4) || (mbits && !aligned(mbits, 4)) || (m4_count && !aligned(m4_count, 4)))
+        return MXQ_ERR_ALIGN;
+    const int64_t nb = gsize / 16;
+    const int64_t total_blocks = total / 16;
+    const ScaleLayout sl = make_scale_layout(swz ? 1 : 0, rows, cols / 16);
+    const int mbits_atomic = (nb % 32) != 0;
+    cudaError_t e = cudaSuccess;
+    if (swz)
+        e = zero_tiled_padding(scales, n_groups, rows, cols / 16, stream);
+    if (e == cudaSuccess && m4_count)
+        e = cudaMemsetAsync(m4_count, 0, (size_t)n_groups * sizeof(uint32_t), stream);
+    if (e == cudaSuccess && mbits && mbits_atomic)
+        e = cudaMemsetAsync(mbits, 0, (size_t)((total_blocks + 31) / 32) * sizeof(uint32_t), stream);
+    if (e == cudaSuccess)
+        e = launch_nvfp4_quant(x, n_groups, nb, mode == MXQ_SCALE_FOUR_SIX, nullptr, s2_in, codes, scales, sl,
+                               nullptr, mbits, mbits_atomic, mode == MXQ_SCALE_FOUR_SIX ? m4_count : nullptr,
+                               status, stream);
     return e == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
 }
 
@@ -409,6 +454,44 @@ mxq_status mxq_dequant_relerr(const uint16_t *x, const uint8_t *codes, const uin
     cudaError_t e = launch_verify(x, codes, scales, s2, (int)fmt, sl, n_tensors, rows, tsize,
                                   tensors_per_scale < 1 ? 1 : tensors_per_scale,
                                   static_cast<double *>(workspace), sum_sq_err, sum_sq_ref, relerr, stream);
+    return e == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
+}
+
+mxq_status mxq_census_reset(mxq_census *census, cudaStream_t stream)
+{
+    const ApiRange range_("mxq_census_reset");
+    if (!census)
+        return MXQ_ERR_INVALID_ARG;
+    if (!aligned(census, 8))
+        return MXQ_ERR_ALIGN;
+    return cudaMemsetAsync(census, 0, sizeof(mxq_census), stream) == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
+}
+
+mxq_status mxq_census_add(mxq_census *census, int64_t n_tensors, const double *sum_sq_err,
+                          const double *sum_sq_ref, const double *relerr, const double *sum_sq_err_rtn,
+                          int64_t n_groups, const uint32_t *m4_count, int64_t blocks_per_group,
+                          cudaStream_t stream)
+{
+    const ApiRange range_("mxq_census_add");
+    if (!census || n_tensors < 0 || n_groups < 0 || blocks_per_group < 0)
+        return MXQ_ERR_INVALID_ARG;
+    if (n_tensors > 0 && (!sum_sq_err || !sum_sq_ref || !relerr))
+        return MXQ_ERR_INVALID_ARG;
+    if (n_groups > 0 && !m4_count)
+        return MXQ_ERR_INVALID_ARG;
+    int64_t blocks;
+    if (!mul_ok(n_groups, blocks_per_group, &blocks))
+        return MXQ_ERR_SHAPE;
+    if (!aligned(census, 8) || (n_tensors > 0 && (!aligned(sum_sq_err, 8) || !aligned(sum_sq_ref, 8) ||
+                                                  !aligned(relerr, 8) ||
+                                                  (sum_sq_err_rtn && !aligned(sum_sq_err_rtn, 8)))) ||
+        (n_groups > 0 && !aligned(m4_count, 4)))
+        return MXQ_ERR_ALIGN;
+    if (n_tensors == 0 && n_groups == 0)
+        return MXQ_OK;
+    const cudaError_t e = launch_census_add(census, n_tensors, sum_sq_err, sum_sq_ref, relerr,
+                                            n_tensors > 0 ? sum_sq_err_rtn : nullptr, n_groups, m4_count,
+                                            blocks_per_group, stream);
     return e == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
 }
 

@@ -7,6 +7,7 @@
 #include <stdint.h>
 
 #include "mxq_device.cuh"
+#include "mxq.h"
 
 namespace mxq {
 
@@ -76,11 +77,12 @@ size_t nvfp4_slots_offset(int64_t n_groups);
 
 cudaError_t launch_group_amax(const uint16_t *x, int64_t n_groups, int64_t nb,
                               uint32_t *amax_bits, uint32_t *status, cudaStream_t s);
+// Block quantizer of the two-pass schedule; the group scale comes from
+// amax_bits (s2_in NULL; s2 written) or from the caller's s2_in.
 cudaError_t launch_nvfp4_quant(const uint16_t *x, int64_t n_groups, int64_t nb, int four_six,
-                               const uint32_t *amax_bits, uint8_t *codes, uint8_t *scales,
-                               const ScaleLayout &sl,
-                               float *s2, uint32_t *mbits, int mbits_atomic,
-                               uint32_t *m4_count, cudaStream_t s);
+                               const uint32_t *amax_bits, const float *s2_in, uint8_t *codes,
+                               uint8_t *scales, const ScaleLayout &sl, float *s2, uint32_t *mbits,
+                               int mbits_atomic, uint32_t *m4_count, uint32_t *status, cudaStream_t s);
 cudaError_t launch_nvfp4_fused(const uint16_t *x, int64_t n_groups, int64_t nb, int four_six,
                                unsigned long long *slots, uint32_t *arrived, uint8_t *codes, uint8_t *scales,
                                const ScaleLayout &sl,
@@ -102,6 +104,9 @@ cudaError_t launch_requant_fp8_mx(const uint8_t *fp8, const float *bscale, int64
                                   int64_t brows, int64_t bcols, int fmt, uint8_t *codes,
                                   uint8_t *scales, const ScaleLayout &sl, uint32_t *status,
                                   cudaStream_t s);
+cudaError_t launch_census_add(mxq_census *c, int64_t n_tensors, const double *err, const double *ref,
+                              const double *rel, const double *err_rtn, int64_t n_groups, const uint32_t *m4,
+                              int64_t blocks_per_group, cudaStream_t s);
 cudaError_t launch_verify(const uint16_t *x, const uint8_t *codes, const uint8_t *scales,
                           const float *s2, int fmt, const ScaleLayout &sl, int64_t n_tensors,
                           int64_t rows, int64_t tsize, int64_t tensors_per_scale, double *partials, double *sum_sq_err,

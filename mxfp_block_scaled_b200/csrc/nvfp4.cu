@@ -57,22 +57,36 @@ group_amax_kernel(const uint4 *__restrict__ x, int64_t n_groups, int64_t nb,
 
 // grid = (tiles of 512 blocks, groups).  Thread t of a tile handles blocks
 // t and t + 256, so each warp covers 32 consecutive blocks per step and its
-// M bits form one 32-bit word.
-template <bool FOUR_SIX>
+// M bits form one 32-bit word.  The group's global scale is either formed
+// from its amax (amax_bits, from group_amax_kernel; written to s2_out) or,
+// with S2IN, given by the caller (s2_in): then a scale that is negative or
+// not finite sets MXQ_DEV_INVALID_SCALE, and a non-finite element, found
+// through its block amax, sets MXQ_DEV_NONFINITE_INPUT.
+template <bool FOUR_SIX, bool S2IN>
 __global__ void __launch_bounds__(kNvThreads)
 nvfp4_quant_kernel(const uint4 *__restrict__ x, int64_t n_groups, int64_t nb,
-                   const uint32_t *__restrict__ amax_bits, uint2 *__restrict__ codes,
+                   const uint32_t *__restrict__ amax_bits, const float *__restrict__ s2_in,
+                   uint2 *__restrict__ codes,
                    uint8_t *__restrict__ scales, const ScaleLayout sl, float *__restrict__ s2_out,
-                   uint32_t *__restrict__ mbits, int mbits_atomic, uint32_t *__restrict__ m4_count)
+                   uint32_t *__restrict__ mbits, int mbits_atomic, uint32_t *__restrict__ m4_count,
+                   uint32_t *__restrict__ status)
 {
     __shared__ GroupConst s_gc;
     __shared__ uint32_t s_m4;
     const int lane = threadIdx.x & 31;
     for (int64_t g = blockIdx.y; g < n_groups; g += gridDim.y) {
         if (threadIdx.x == 0) {
-            s_gc = make_group_const(amax_bits[g]);
-            if (blockIdx.x == 0)
-                s2_out[g] = s_gc.s2;
+            if (S2IN) {
+                const float v = s2_in[g];
+                const bool valid = v >= 0.0f && v <= 0x1.fffffep127f;   // false for NaN
+                s_gc = make_group_const_from_s2(valid ? v : 0.0f);
+                if (!valid && blockIdx.x == 0)
+                    atomicOr(status, MXQ_DEV_INVALID_SCALE);
+            } else {
+                s_gc = make_group_const(amax_bits[g]);
+                if (blockIdx.x == 0)
+                    s2_out[g] = s_gc.s2;
+            }
             s_m4 = 0;
         }
         __syncthreads();
@@ -98,6 +112,8 @@ nvfp4_quant_kernel(const uint4 *__restrict__ x, int64_t n_groups, int64_t nb,
                 o.m4 = false;
                 if (live) {
                     o = quantize_block<FOUR_SIX>(v[k][0], v[k][1], gc);
+                    if (S2IN && !(o.amax <= 0x1.fep127f))       // Inf or NaN element
+                        atomicOr(status, MXQ_DEV_NONFINITE_INPUT);
                     const int64_t gb = g * nb + b;
                     codes[gb] = o.codes;
                     scales[sl.swz ? tiled_scale_offset(sl, (uint64_t)g, (uint32_t)b) : (uint64_t)gb] =
@@ -628,9 +644,9 @@ cudaError_t launch_nvfp4_fused(const uint16_t *x, int64_t n_groups, int64_t nb, 
 }
 
 cudaError_t launch_nvfp4_quant(const uint16_t *x, int64_t n_groups, int64_t nb, int four_six,
-                               const uint32_t *amax_bits, uint8_t *codes, uint8_t *scales,
-                               const ScaleLayout &sl, float *s2, uint32_t *mbits, int mbits_atomic,
-                               uint32_t *m4_count, cudaStream_t s)
+                               const uint32_t *amax_bits, const float *s2_in, uint8_t *codes,
+                               uint8_t *scales, const ScaleLayout &sl, float *s2, uint32_t *mbits,
+                               int mbits_atomic, uint32_t *m4_count, uint32_t *status, cudaStream_t s)
 {
     if (n_groups == 0)
         return cudaSuccess;
@@ -639,12 +655,15 @@ cudaError_t launch_nvfp4_quant(const uint16_t *x, int64_t n_groups, int64_t nb, 
               (unsigned)(n_groups < 65535 ? n_groups : 65535));
     const uint4 *xv = reinterpret_cast<const uint4 *>(x);
     uint2 *cv = reinterpret_cast<uint2 *>(codes);
-    if (four_six)
-        nvfp4_quant_kernel<true><<<grid, kNvThreads, 0, s>>>(xv, n_groups, nb, amax_bits, cv, scales,
-                                                             sl, s2, mbits, mbits_atomic, m4_count);
-    else
-        nvfp4_quant_kernel<false><<<grid, kNvThreads, 0, s>>>(xv, n_groups, nb, amax_bits, cv, scales,
-                                                              sl, s2, mbits, mbits_atomic, m4_count);
+#define MXQ_QUANT(F, S)                                                                                  \
+    nvfp4_quant_kernel<F, S><<<grid, kNvThreads, 0, s>>>(xv, n_groups, nb, amax_bits, s2_in, cv, scales, sl, \
+                                                         s2, mbits, mbits_atomic, m4_count, status)
+    if (s2_in) {
+        if (four_six) MXQ_QUANT(true, true); else MXQ_QUANT(false, true);
+    } else {
+        if (four_six) MXQ_QUANT(true, false); else MXQ_QUANT(false, false);
+    }
+#undef MXQ_QUANT
     return cudaGetLastError();
 }
 

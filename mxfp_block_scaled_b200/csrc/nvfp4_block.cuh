@@ -48,11 +48,11 @@ struct GroupConst {
                      // reciprocal quotient of the block values is exact
 };
 
-__device__ __forceinline__ GroupConst make_group_const(uint32_t amax_bits)
+// Constants of a group from its global scale s2 (finite, >= 0).
+__device__ __forceinline__ GroupConst make_group_const_from_s2(float s2)
 {
     GroupConst c;
-    const float amax = __uint_as_float(amax_bits << 16);
-    c.s2 = __fdiv_rn(amax, kGlobalDivisor);
+    c.s2 = s2;
     c.den = make_float2(__fmul_rn(6.0f, c.s2), __fmul_rn(4.0f, c.s2));
     c.tfast = (c.s2 >= 0x1p-100f && c.s2 <= 0x1p100f) ? 1 : 0;
     c.qfast = (c.s2 >= 0x1p-50f && c.s2 <= 0x1p50f) ? 1 : 0;
@@ -60,6 +60,13 @@ __device__ __forceinline__ GroupConst make_group_const(uint32_t amax_bits)
     c.s2h = 0.5 * (double)c.s2;
     c.s2hf = 0.5f * c.s2;
     return c;
+}
+
+// Constants of a group from its amax (bf16 magnitude bits): s2 = RN32(amax / 2688).
+__device__ __forceinline__ GroupConst make_group_const(uint32_t amax_bits)
+{
+    const float amax = __uint_as_float(amax_bits << 16);
+    return make_group_const_from_s2(__fdiv_rn(amax, kGlobalDivisor));
 }
 
 struct Plan {
@@ -172,6 +179,7 @@ struct BlockOut {
     uint2 codes;
     uint32_t scale;
     bool m4;
+    float amax;   // the block amax (Inf or NaN when an element is not finite)
 };
 
 __device__ __forceinline__ void unpack_x(const uint32_t (&w)[8], float2 (&x)[8])
@@ -188,6 +196,7 @@ template <bool FOUR_SIX>
 __device__ __noinline__ BlockOut quantize_block_general(uint4 v0, uint4 v1, float amax_b, const GroupConst gc)
 {
     BlockOut o;
+    o.amax = amax_b;
     if (!(gc.s2 > 0.0f)) {  // all-zero group
         o.codes = make_uint2(0u, 0u);
         o.scale = 0u;
@@ -247,6 +256,7 @@ __device__ __forceinline__ BlockOut quantize_block(uint4 v0, uint4 v1, const Gro
     float2 x[8];
     unpack_x(w, x);
     BlockOut o;
+    o.amax = amax_b;
     if (!FOUR_SIX) {
         const Plan p6 = make_plan_fast(x, d.x, __frcp_rn(d.x));
         o.codes = p6.codes;

@@ -230,6 +230,87 @@ __global__ void verify_finalize_kernel(const double *__restrict__ partials, int6
     }
 }
 
+// ---------------------------------------------------------------------------
+// Census of a conversion: the verifier's per-tensor figures reduced to the
+// pages' summary figures (dabsLabs/Qwen3.8-Flash-Next-NVFP4, metric table:
+// mean and max relative error over the expert tensors; "What makes this
+// build different": total squared error of the 4/6 choice against plain
+// RTN block scales, share of 16-blocks that chose M=4).  One CTA: thread t
+// adds elements t, t + 256, ... in order, then a fixed tree, then the call's
+// totals are added to the census; so a sequence of calls gives the same
+// bits every time.
+// ---------------------------------------------------------------------------
+constexpr int kCensusThreads = 256;
+
+__global__ void __launch_bounds__(kCensusThreads)
+census_add_kernel(mxq_census *__restrict__ c, int64_t n_tensors, const double *__restrict__ err,
+                  const double *__restrict__ ref, const double *__restrict__ rel,
+                  const double *__restrict__ err_rtn, int64_t n_groups, const uint32_t *__restrict__ m4,
+                  int64_t blocks_per_group)
+{
+    __shared__ double s_sum[4][kCensusThreads];
+    __shared__ double s_max[kCensusThreads];
+    __shared__ unsigned long long s_m4[kCensusThreads];
+    const int t = threadIdx.x;
+    double a = 0.0, b = 0.0, r = 0.0, q = 0.0, mx = 0.0;
+    for (int64_t i = t; i < n_tensors; i += kCensusThreads) {
+        r += rel[i];
+        a += err[i];
+        b += ref[i];
+        if (err_rtn)
+            q += err_rtn[i];
+        mx = fmax(mx, rel[i]);
+    }
+    unsigned long long k = 0;
+    for (int64_t g = t; g < n_groups; g += kCensusThreads)
+        k += m4[g];
+    s_sum[0][t] = r;
+    s_sum[1][t] = a;
+    s_sum[2][t] = b;
+    s_sum[3][t] = q;
+    s_max[t] = mx;
+    s_m4[t] = k;
+    __syncthreads();
+    for (int off = kCensusThreads / 2; off > 0; off >>= 1) {
+        if (t < off) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                s_sum[j][t] += s_sum[j][t + off];
+            s_max[t] = fmax(s_max[t], s_max[t + off]);
+            s_m4[t] += s_m4[t + off];
+        }
+        __syncthreads();
+    }
+    if (t == 0) {
+        c->sum_relerr += s_sum[0][0];
+        c->sum_sq_err += s_sum[1][0];
+        c->sum_sq_ref += s_sum[2][0];
+        if (n_tensors > 0)
+            c->max_relerr = fmax(c->max_relerr, s_max[0]);
+        c->n_tensors += (uint64_t)n_tensors;
+        if (err_rtn) {
+            c->sum_sq_err_rtn += s_sum[3][0];
+            c->n_tensors_rtn += (uint64_t)n_tensors;
+        }
+        c->blocks += (uint64_t)(n_groups * blocks_per_group);
+        c->blocks_m4 += s_m4[0];
+        c->mean_relerr = c->n_tensors ? c->sum_relerr / (double)c->n_tensors : 0.0;
+        c->sse_vs_rtn = (c->n_tensors > 0 && c->n_tensors_rtn == c->n_tensors && c->sum_sq_err_rtn > 0.0)
+                            ? c->sum_sq_err / c->sum_sq_err_rtn - 1.0
+                            : __longlong_as_double(0x7FF8000000000000LL);
+        c->m4_fraction = c->blocks ? (double)c->blocks_m4 / (double)c->blocks : 0.0;
+    }
+}
+
+cudaError_t launch_census_add(mxq_census *c, int64_t n_tensors, const double *err, const double *ref,
+                              const double *rel, const double *err_rtn, int64_t n_groups, const uint32_t *m4,
+                              int64_t blocks_per_group, cudaStream_t s)
+{
+    census_add_kernel<<<1, kCensusThreads, 0, s>>>(c, n_tensors, err, ref, rel, err_rtn, n_groups, m4,
+                                                   blocks_per_group);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_verify(const uint16_t *x, const uint8_t *codes, const uint8_t *scales,
                           const float *s2, int fmt, const ScaleLayout &sl, int64_t n_tensors,
                           int64_t rows, int64_t tsize, int64_t tensors_per_scale, double *partials,

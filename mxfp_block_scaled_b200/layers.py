@@ -72,36 +72,52 @@ def quantize_mixed(layers, formats, stream=None):
     return [quantize_routed_layer(gu, dn, fmt=f, stream=stream) for (gu, dn), f in zip(layers, formats)]
 
 
+def census(results, results_rtn=None, stream=None):
+    """The census of the given layer results, formed on the device by
+    mxq_census_add (dabsLabs/Qwen3.8-Flash-Next-NVFP4, metric table: mean
+    and max relative error over the unstacked tensors; "What makes this
+    build different": SSE(chosen) / SSE(RTN) - 1 and the share of 16-blocks
+    that chose M=4).  `results` are quantize_routed_layer results; with
+    `results_rtn` (the same layers quantized in "rtn" mode) each tensor is
+    added with its RTN error sum, which gives sse_vs_rtn.  Returns the
+    struct's fields as a dict (mxq.CENSUS_FIELDS)."""
+    dev = results[0]["gate_up"]["codes"].device if results else "cuda"
+    c = mxq.Census(device=dev, stream=stream)
+    for i, q in enumerate(results):
+        for k in ("gate_up", "down"):
+            s = q[k]
+            rtn = results_rtn[i][k]["sum_sq_err"] if results_rtn is not None else None
+            nvfp4 = s["fmt"] == "nvfp4"
+            E, R, C2 = s["codes"].shape
+            C = C2 * 2 if s["fmt"] != "mxfp8" else C2
+            c.add(n_tensors=s["relerr"].numel(), sum_sq_err=s["sum_sq_err"], sum_sq_ref=s["sum_sq_ref"],
+                  relerr=s["relerr"], sum_sq_err_rtn=rtn, n_groups=E if nvfp4 else 0,
+                  m4_count=s["m4_count"] if nvfp4 else None, blocks_per_group=R * C // 16 if nvfp4 else 0,
+                  stream=stream)
+    return c.result()
+
+
 def relerr_census(results):
     """Mean and max relative error over every unstacked tensor of the given
-    layer results (the metric-table figures: mean / max rel-err over the
-    expert census)."""
-    rel = torch.cat([q[k]["relerr"] for q in results for k in ("gate_up", "down")])
-    return float(rel.mean()), float(rel.max()), int(rel.numel())
+    layer results, and the tensor count (the metric-table figures)."""
+    r = census(results)
+    return r["mean_relerr"], r["max_relerr"], r["n_tensors"]
 
 
 def sse_vs_rtn(results, results_rtn):
     """SSE(chosen) / SSE(RTN) - 1 over every unstacked tensor of the given
-    layer results (dabsLabs/Qwen3.8-Flash-Next-NVFP4, "What makes this
-    build different": the 4/6 choice against plain amax/6 block scales;
-    never above 0).  `results` and `results_rtn` are quantize_routed_layer
-    results of the same layers in "four_six" and "rtn" mode; the per-tensor
-    squared-error sums come from the verifier and are added on the host."""
-    def total(res):
-        return sum(float(q[k]["sum_sq_err"].cpu().numpy().sum()) for q in res for k in ("gate_up", "down"))
-    return total(results) / total(results_rtn) - 1.0
+    layer results ("four_six" and "rtn" quantize_routed_layer results of the
+    same layers).  The 4/6 rule is never worse than RTN per block on the exact
+    error, so the exact figure is never above 0; from the verifier's sums,
+    each within 11 * 2^-24 relative of its exact value, it can come out above
+    0 by at most about 1.4e-6 (a layer whose blocks nearly all tie)."""
+    return census(results, results_rtn)["sse_vs_rtn"]
 
 
 def m4_fraction(results):
     """Fraction of NVFP4 blocks that took the M=4 plan (from the per-group
-    M=4 counts)."""
-    m4 = blocks = 0
-    for q in results:
-        for k in ("gate_up", "down"):
-            E = q[k]["codes"].shape[0]
-            m4 += int(q[k]["m4_count"].cpu().numpy()[:E].sum())
-            blocks += q[k]["codes"].numel() // 8
-    return m4 / blocks
+    M=4 counts of the quantizer)."""
+    return census(results)["m4_fraction"]
 
 
 # ------------------------------------------------ host-resident layers --

@@ -23,6 +23,7 @@ STATUS_NAMES = {0: "ok", 1: "invalid argument", 2: "shape", 3: "align", 4: "work
                 5: "cuda", 6: "unsupported"}
 DEV_NONFINITE_INPUT = 0x1
 DEV_WAIT_TIMEOUT = 0x2
+DEV_INVALID_SCALE = 0x4
 
 FMT = {"nvfp4": 0, "mxfp4": 1, "mxfp8": 2}
 SCALE_MODE = {"rtn": 0, "four_six": 1}
@@ -30,9 +31,15 @@ LAYOUT = {"linear": 0, "swizzled_128x4": 1}
 OP = {"quantize_nvfp4": 0, "quantize_act": 1, "dequant_relerr": 2}
 
 EXPORTED = ("mxq_version", "mxq_status_string", "mxq_scale_bytes", "mxq_workspace_bytes",
-            "mxq_quantize_nvfp4", "mxq_quantize_nvfp4_weighted",
+            "mxq_quantize_nvfp4", "mxq_quantize_nvfp4_s2", "mxq_quantize_nvfp4_weighted",
             "mxq_quantize_mx", "mxq_requant_fp8_mx", "mxq_quantize_act", "mxq_dequant_relerr",
-            "mxq_dequant_relerr_noalloc")
+            "mxq_dequant_relerr_noalloc", "mxq_census_reset", "mxq_census_add")
+
+# Fields of struct mxq_census (include/mxq.h), in order, each 8 bytes.
+CENSUS_FIELDS = ("sum_relerr", "max_relerr", "sum_sq_err", "sum_sq_ref", "sum_sq_err_rtn",
+                 "n_tensors", "n_tensors_rtn", "blocks", "blocks_m4",
+                 "mean_relerr", "sse_vs_rtn", "m4_fraction", "reserved")
+_CENSUS_INTS = ("n_tensors", "n_tensors_rtn", "blocks", "blocks_m4")
 
 
 class MxqError(RuntimeError):
@@ -64,6 +71,12 @@ def load(path=LIB_PATH):
     L.mxq_workspace_bytes.argtypes = [i32, i64, i64, i64]
     L.mxq_quantize_nvfp4.restype = i32
     L.mxq_quantize_nvfp4.argtypes = [vp, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.mxq_quantize_nvfp4_s2.restype = i32
+    L.mxq_quantize_nvfp4_s2.argtypes = [vp, i64, i64, i64, vp, i32, i32, vp, vp, vp, vp, vp, vp]
+    L.mxq_census_reset.restype = i32
+    L.mxq_census_reset.argtypes = [vp, vp]
+    L.mxq_census_add.restype = i32
+    L.mxq_census_add.argtypes = [vp, i64, vp, vp, vp, vp, i64, vp, i64, vp]
     L.mxq_quantize_nvfp4_weighted.restype = i32
     L.mxq_quantize_nvfp4_weighted.argtypes = [vp, i64, i64, i64, vp, i64, i32, vp, vp, vp, vp, vp, sz,
                                               vp]
@@ -165,6 +178,40 @@ def mxq_quantize_nvfp4(x, n_groups, rows, cols, mode, layout, codes, scales, s2,
                                    _p(scales), _p(s2), _p(mbits), _p(m4_count), _p(status),
                                    _p(workspace), _nbytes(workspace), _stream(stream))
     _check("mxq_quantize_nvfp4", rc)
+
+
+def mxq_quantize_nvfp4_s2(x, n_groups, rows, cols, s2_in, mode, layout, codes, scales, mbits, m4_count,
+                          status, stream=None):
+    n = n_groups * rows * cols
+    _need("x", x, 2 * n)
+    _need("s2_in", s2_in, 4 * n_groups)
+    _need("codes", codes, n // 2)
+    _need("scales", scales, scale_bytes("nvfp4", layout, n_groups, rows, cols))
+    _need("mbits", mbits, 4 * ((n // 16 + 31) // 32))
+    _need("m4_count", m4_count, 4 * n_groups)
+    _need("status", status, 4)
+    rc = load().mxq_quantize_nvfp4_s2(_p(x), n_groups, rows, cols, _p(s2_in), SCALE_MODE[mode],
+                                      LAYOUT[layout], _p(codes), _p(scales), _p(mbits), _p(m4_count),
+                                      _p(status), _stream(stream))
+    _check("mxq_quantize_nvfp4_s2", rc)
+
+
+def mxq_census_reset(census, stream=None):
+    _need("census", census, 8 * len(CENSUS_FIELDS))
+    _check("mxq_census_reset", load().mxq_census_reset(_p(census), _stream(stream)))
+
+
+def mxq_census_add(census, n_tensors, sum_sq_err, sum_sq_ref, relerr, sum_sq_err_rtn, n_groups,
+                   m4_count, blocks_per_group, stream=None):
+    _need("census", census, 8 * len(CENSUS_FIELDS))
+    for name, t in (("sum_sq_err", sum_sq_err), ("sum_sq_ref", sum_sq_ref), ("relerr", relerr),
+                    ("sum_sq_err_rtn", sum_sq_err_rtn)):
+        _need(name, t, 8 * n_tensors)
+    _need("m4_count", m4_count, 4 * n_groups)
+    rc = load().mxq_census_add(_p(census), n_tensors, _p(sum_sq_err), _p(sum_sq_ref), _p(relerr),
+                               _p(sum_sq_err_rtn), n_groups, _p(m4_count), blocks_per_group,
+                               _stream(stream))
+    _check("mxq_census_add", rc)
 
 
 def mxq_quantize_nvfp4_weighted(x, n_groups, rows, cols, h, h_groups, layout, codes, scales, s2,
@@ -287,6 +334,51 @@ def quantize_nvfp4(x, mode="four_six", with_mbits=True, stream=None, layout="lin
     mxq_quantize_nvfp4(x, G, R, C, mode, layout, out["codes"], out["scales"], out["s2"],
                        out["mbits"], out["m4_count"], out["status"], ws, stream)
     return out
+
+
+def quantize_nvfp4_s2(x, s2_in, mode="four_six", with_mbits=True, stream=None, layout="linear"):
+    """x: bf16 [G, R, C]; s2_in: fp32 [G] global scales on the device (gate
+    and up held apart pass the scale they share).  Returns a dict of device
+    tensors: codes, scales, mbits, m4_count, status (as quantize_nvfp4,
+    without s2)."""
+    _bf16(x)
+    G, R, C = x.shape
+    if s2_in.dtype != torch.float32 or not s2_in.is_contiguous() or s2_in.numel() < G:
+        raise ValueError("expected contiguous fp32 global scales [G]")
+    dev = x.device
+    out = {
+        "codes": torch.empty((G, R, C // 2), dtype=torch.uint8, device=dev),
+        "scales": torch.empty((G, R, C // 16), dtype=torch.uint8, device=dev) if layout == "linear"
+        else torch.empty(max(scale_bytes("nvfp4", layout, G, R, C), 1), dtype=torch.uint8, device=dev),
+        "mbits": torch.empty(((G * R * C // 16) + 31) // 32 or 1, dtype=torch.int32, device=dev)
+        if with_mbits else None,
+        "m4_count": torch.empty(max(G, 1), dtype=torch.int32, device=dev),
+        "status": torch.zeros(1, dtype=torch.int32, device=dev),
+    }
+    mxq_quantize_nvfp4_s2(x, G, R, C, s2_in, mode, layout, out["codes"], out["scales"], out["mbits"],
+                          out["m4_count"], out["status"], stream)
+    return out
+
+
+class Census:
+    """A device-resident struct mxq_census: reset on creation, filled by
+    add() (mxq_census_add), read by result() (one small device -> host
+    copy, after which the struct's fields come back as a dict)."""
+
+    def __init__(self, device="cuda", stream=None):
+        self.buf = torch.empty(len(CENSUS_FIELDS), dtype=torch.float64, device=device)
+        mxq_census_reset(self.buf, stream)
+
+    def add(self, n_tensors=0, sum_sq_err=None, sum_sq_ref=None, relerr=None, sum_sq_err_rtn=None,
+            n_groups=0, m4_count=None, blocks_per_group=0, stream=None):
+        mxq_census_add(self.buf, n_tensors, sum_sq_err, sum_sq_ref, relerr, sum_sq_err_rtn, n_groups,
+                       m4_count, blocks_per_group, stream)
+
+    def result(self):
+        raw = self.buf.cpu()
+        ints = raw.view(torch.int64)
+        return {k: (int(ints[i]) if k in _CENSUS_INTS else float(raw[i]))
+                for i, k in enumerate(CENSUS_FIELDS) if k != "reserved"}
 
 
 def quantize_nvfp4_weighted(x, h, stream=None, layout="linear"):

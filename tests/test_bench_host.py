@@ -71,14 +71,42 @@ def test_mixed_format_layers_and_bytes():
     assert step == 4 * n * (5.125 + 5.0625)          # about 98.45 GB per step
 
 
-def test_sse_vs_rtn_pass(monkeypatch):
+class FakeCensus:
+    """Stands in for mxq.Census on the CPU: keeps the arrays each add() got,
+    so the test sees which buffers the bench hands to the census."""
+    made = []
+
+    def __init__(self, device=None, stream=None):
+        self.adds = []
+        FakeCensus.made.append(self)
+
+    def add(self, **kw):
+        self.adds.append({k: (v.clone() if hasattr(v, "clone") else v) for k, v in kw.items()})
+
+    def result(self):
+        err = sum(float(a["sum_sq_err"].sum()) for a in self.adds)
+        rtn = [a["sum_sq_err_rtn"] for a in self.adds]
+        return {"mean_relerr": 0.0, "max_relerr": 0.0, "n_tensors": sum(a["n_tensors"] for a in self.adds),
+                "m4_fraction": 0.0,
+                "sse_vs_rtn": (err / sum(float(r.sum()) for r in rtn) - 1.0) if all(r is not None for r in rtn)
+                else float("nan")}
+
+
+def test_census_pass(monkeypatch):
     import torch
+    from mxfp_block_scaled_b200 import mxq
     monkeypatch.setattr(bench.torch.cuda, "synchronize", lambda *a: None)
+    monkeypatch.setattr(mxq, "Census", FakeCensus)
 
     class FakeLayer:
         """err holds the 4/6 sums until the RTN quantize + verify rewrites them."""
         def __init__(self, e46, ertn):
-            self.out = {t: {"err": torch.tensor(e46[t], dtype=torch.float64)} for t in ("gu", "dn")}
+            self.gu = torch.zeros(1)
+            self.out = {t: {"err": torch.tensor(e46[t], dtype=torch.float64),
+                            "ref": torch.ones(len(e46[t]), dtype=torch.float64),
+                            "rel": torch.zeros(len(e46[t]), dtype=torch.float64),
+                            "m4": torch.tensor([1], dtype=torch.int32), "nt": len(e46[t]), "G": 1,
+                            "R": 4, "C": 16} for t in ("gu", "dn")}
             self.ertn, self.mode = ertn, None
 
         def quantize(self, t, mode="four_six"):
@@ -90,11 +118,20 @@ def test_sse_vs_rtn_pass(monkeypatch):
 
     a = FakeLayer({"gu": [1.0, 2.0], "dn": [1.0]}, {"gu": [2.0, 2.0], "dn": [4.0]})
     b = FakeLayer({"gu": [0.5], "dn": [0.5]}, {"gu": [1.0], "dn": [1.0]})
-    assert abs(bench.nvfp4_sse_vs_rtn([a, b]) - (5.0 / 10.0 - 1.0)) < 1e-15
+    r = bench.nvfp4_census([a, b])
+    assert abs(r["sse_vs_rtn"] - (5.0 / 10.0 - 1.0)) < 1e-15
+    c = FakeCensus.made[-1]
+    # the 4/6 error sums were saved before the RTN pass rewrote the buffers
+    assert [a_["sum_sq_err"].tolist() for a_ in c.adds] == [[1.0, 2.0], [1.0], [0.5], [0.5]]
+    assert [a_["sum_sq_err_rtn"].tolist() for a_ in c.adds] == [[2.0, 2.0], [4.0], [1.0], [1.0]]
+    assert all(a_["blocks_per_group"] == 4 and a_["n_groups"] == 1 for a_ in c.adds)
+    # without the RTN pass, no RTN sums reach the census
+    r = bench.nvfp4_census([FakeLayer({"gu": [1.0], "dn": [1.0]}, {})], with_rtn=False)
+    assert "sse_vs_rtn" not in r and FakeCensus.made[-1].adds[0]["sum_sq_err_rtn"] is None
 
     class Broken(FakeLayer):
         def verify(self, t):
             raise RuntimeError("device status 0x2")
 
-    r = bench.nvfp4_sse_vs_rtn([Broken({"gu": [1.0], "dn": [1.0]}, {})])
-    assert "unavailable" in r and "0x2" in r["unavailable"]
+    r = bench.nvfp4_census([Broken({"gu": [1.0], "dn": [1.0]}, {})])
+    assert "unavailable" in r["sse_vs_rtn"] and "0x2" in r["sse_vs_rtn"]["unavailable"]

@@ -59,7 +59,9 @@ def test_allocating_wrappers_pass_the_checks(rec, layout):
                            layout=layout)
     for fmt, mode in (("nvfp4", "rtn"), ("nvfp4", "four_six"), ("mxfp8", "rtn"), ("mxfp4", "rtn")):
         mxq.quantize_act(_bf16(5, C), fmt, mode=mode, layout=layout)
+    mxq.quantize_nvfp4_s2(x, torch.ones(G), layout=layout)
     names = [c[0] for c in rec.calls]
+    assert names.count("mxq_quantize_nvfp4_s2") == 1
     assert names.count("mxq_quantize_nvfp4") == 1 and names.count("mxq_quantize_nvfp4_weighted") == 2
     assert names.count("mxq_quantize_mx") == 2 and names.count("mxq_requant_fp8_mx") == 2
     assert names.count("mxq_quantize_act") == 4 and names.count("mxq_dequant_relerr") == 3
@@ -177,3 +179,20 @@ def test_workspace_is_passed_in_bytes(rec):
     a["workspace"] = torch.zeros(1000, dtype=torch.float32)
     mxq.mxq_quantize_nvfp4(**a)
     assert rec.calls[0][1][-2] == 4000
+
+
+def test_s2_and_census_buffers_are_checked(rec):
+    G, R, C = 3, 16, 32
+    x = _bf16(G, R, C)
+    with pytest.raises(ValueError):
+        mxq.quantize_nvfp4_s2(x, torch.ones(G - 1))                      # one scale short
+    cen = torch.zeros(len(mxq.CENSUS_FIELDS), dtype=torch.float64)
+    mxq.mxq_census_reset(cen)
+    arr = torch.zeros(4, dtype=torch.float64)
+    mxq.mxq_census_add(cen, 4, arr, arr, arr, None, 2, torch.zeros(2, dtype=torch.int32), 8)
+    with pytest.raises(ValueError):
+        mxq.mxq_census_add(cen, 5, arr, arr, arr, None, 0, None, 0)      # arrays shorter than n_tensors
+    with pytest.raises(ValueError):
+        mxq.mxq_census_reset(cen[:12])                                    # struct is 13 fields
+    names = [c[0] for c in rec.calls]
+    assert names == ["mxq_census_reset", "mxq_census_add"]
