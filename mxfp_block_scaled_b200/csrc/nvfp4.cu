@@ -156,19 +156,20 @@ nvfp4_quant_kernel(const uint4 *__restrict__ x, int64_t n_groups, int64_t nb,
 //                  amax, publish it as one tagged 64-bit slot per group
 //                  and CTA (tag and value land together: no fence needed)
 //                  and then count the group's arrivals up by one;
-//   quantize copy  (ring of `qstages`), issued only after the scouts are
-//                  done with that group, `distance` groups behind them, so
-//                  it normally hits the L2 copy the scout read left behind:
-//                  20 compute warps quantize it once a publisher warp has
-//                  seen every CTA's slot for the group.  The publisher polls
+//   quantize copy  (ring of `qstages`), issued only after a publisher warp
+//                  has seen every CTA's slot for the group and released it
+//                  (group constants set), `distance` groups behind the
+//                  scouts, so it normally hits the L2 copy the scout read
+//                  left behind: 20 compute warps quantize it as soon as it
+//                  lands, one barrier per hand-over.  The publisher polls
 //                  only the one arrival word of a group; it reads the slots
 //                  (and checks their tags) once the count is complete, so
 //                  the polling of every CTA stays off the slots' L2 lines.
 // The grid-wide amax of a group is therefore resolved while the compute
 // warps work on earlier groups; its latency is off the critical path.
 // Roles hand over through mbarriers (sfull / sfreed: scout ring, qfull /
-// qfreed: quantize ring, ready: group amax known) and one shared counter
-// (groups scouted).  Every wait is bounded: on time-out the CTA sets
+// qfreed: quantize ring, ready: group released, which the loader waits for)
+// and one shared counter (groups scouted).  Every wait is bounded: on time-out the CTA sets
 // MXQ_DEV_WAIT_TIMEOUT, lets its copies in flight land (bounded) and
 // returns.
 // ---------------------------------------------------------------------------
@@ -326,12 +327,14 @@ nvfp4_fused_kernel(const FusedArgs a)
     if (warp == 1) {
         // ----------------------------------------------------------- loader
         // Scout copies run up to `distance` groups ahead of quantize copies;
-        // a group's quantize copy waits until the scouts are done with it.
+        // a group's quantize copy is issued once the publisher has released
+        // the group (its constants are set), so a compute warp that sees the
+        // copy land may use the group at once: one barrier per hand-over.
         if (lane != 0 || bytes == 0)
             return;
         // Stages and phase parities advance incrementally (no division).
-        int s_next = 0, q_next = 0, s_st = 0, q_st = 0;
-        uint32_t s_par = 0, q_par = 0;                  // parity of (next / ring size)
+        int s_next = 0, q_next = 0, s_st = 0, q_st = 0, q_rs = 0;
+        uint32_t s_par = 0, q_par = 0, q_rpar = 0;      // parity of (next / ring size)
         int s_last[kMaxStages], q_last[kMaxStages];     // phase parity of the copy in flight, or -1
         for (int k = 0; k < kMaxStages; ++k)
             s_last[k] = q_last[k] = -1;
@@ -353,7 +356,7 @@ nvfp4_fused_kernel(const FusedArgs a)
                     progress = true;
                 }
             }
-            if (q_next < *scouted) {
+            if (q_next < *scouted && mbar_test_wait(ready + q_rs, q_rpar)) {
                 if (q_next < LQ || mbar_test_wait(qfreed + q_st, q_par ^ 1u)) {
                     fence_proxy_async_smem();
                     mbar_arrive_expect_tx(qfull + q_st, bytes);
@@ -364,6 +367,10 @@ nvfp4_fused_kernel(const FusedArgs a)
                     if (++q_st == LQ) {
                         q_st = 0;
                         q_par ^= 1u;
+                    }
+                    if (++q_rs == kReadyRing) {
+                        q_rs = 0;
+                        q_rpar ^= 1u;
                     }
                     progress = true;
                 }
@@ -476,10 +483,11 @@ nvfp4_fused_kernel(const FusedArgs a)
     const int step = run % kWarpsPerPart;               // offset gained per group
     int first = li;                                     // this warp's first chunk of the run
     int st = 0, rs = 0;                                 // quantize stage and ready slot of group j
-    uint32_t qpar = 0, rpar = 0;                        // their phase parities
+    uint32_t qpar = 0;                                  // the stage's phase parity
     for (int j = 0; j < G; ++j) {
-        bool ok = wait_phase(ready + rs, rpar, abort_flag, 200u);
-        ok = ok && wait_phase(qfull + st, qpar, abort_flag, 200u);
+        // the stage's copy is issued only after the group's release, so its
+        // completion also orders the publisher's constants before their use
+        const bool ok = wait_phase(qfull + st, qpar, abort_flag, 200u);
         if (!__all_sync(0xFFFFFFFFu, ok))
             break;
         const GroupConst gc = s_gc[rs];
@@ -516,10 +524,8 @@ nvfp4_fused_kernel(const FusedArgs a)
             st = 0;
             qpar ^= 1u;
         }
-        if (++rs == kReadyRing) {
+        if (++rs == kReadyRing)
             rs = 0;
-            rpar ^= 1u;
-        }
         first -= step;                                  // (li - run * (j + 1)) mod warps
         if (first < 0)
             first += kWarpsPerPart;
