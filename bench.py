@@ -76,9 +76,9 @@ def kernel_source_sha():
     return h.hexdigest()[:16]
 
 
-def ncu_traffic_per_launch():
-    """DRAM bytes per quantize launch from the committed ncu summary, or None
-    when the kernel source changed since it was captured."""
+def _traffic_record():
+    """Fields of the committed ncu traffic summary, or None when the kernel
+    source changed since it was captured."""
     p = os.path.join(ROOT, "profiles", "nvfp4_quant_gate_up_fullsize_traffic.txt")
     try:
         kv = {}
@@ -90,9 +90,30 @@ def ncu_traffic_per_launch():
                     kv[k] = v
         if kv.get("source_sha") != kernel_source_sha():
             return None
-        return float(kv["dram_bytes_per_call"])
+        return kv
     except Exception:
         return None
+
+
+def ncu_traffic_per_launch():
+    """DRAM bytes (read + write) per quantize launch from the committed ncu
+    summary, or None when the kernel source changed since it was captured."""
+    kv = _traffic_record()
+    try:
+        return float(kv["dram_bytes_per_call"]) if kv else None
+    except (KeyError, ValueError):
+        return None
+
+
+def ncu_traffic_split():
+    """{"traffic_read": R, "traffic_write": W} per quantize launch from the
+    same summary (empty when unavailable)."""
+    kv = _traffic_record()
+    try:
+        return {"traffic_read": float(kv["dram_read_per_call"]),
+                "traffic_write": float(kv["dram_write_per_call"])} if kv else {}
+    except (KeyError, ValueError):
+        return {}
 
 
 class ClockSampler:
@@ -1085,6 +1106,7 @@ def main():
                    "quality": quality},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
+                     **(ncu_traffic_split() if traffic is not None else {}),
                      "kernel": "nvfp4_fused_kernel (mxq_quantize_nvfp4 on the gate_up stack)",
                      "algorithmic_bytes_per_launch": gu_elems * Q_BYTES,
                      "peak_kind": peak_kind},
