@@ -202,6 +202,22 @@ MXQ_API mxq_status mxq_quantize_nvfp4(const uint16_t *x, int64_t n_groups, int64
                               uint32_t *m4_count, uint32_t *status, void *workspace,
                               size_t workspace_bytes, cudaStream_t stream);
 
+/* The global scale of each NVFP4 group alone: s2 = RN32(amax_g / 2688).
+ * Source: josch15366/Qwen3.8-Flash-Next-NVFP4-LocalHessian-Experts,
+ * introduction (weight_scale_2 and input_scale are amax / 2688).
+ *   x       bf16 [n_groups, rows, cols], cols % 16 == 0 (as mxq_quantize_nvfp4).
+ *   s2      out, fp32 [n_groups]; the bits of s2 equal what mxq_quantize_nvfp4
+ *           writes for the same groups.  Rounding is monotone, so the scale of
+ *           a group split over two calls (gate and up held apart) is the
+ *           larger of its two parts' scales.
+ *   status  required: MXQ_DEV_NONFINITE_INPUT when an element is Inf or NaN.
+ * No workspace: s2 holds the running amax until the last kernel of the call
+ * turns it into the scale.  With mxq_quantize_nvfp4_s2 this is the two-pass
+ * form of mxq_quantize_nvfp4 (x is read twice). */
+MXQ_API mxq_status mxq_global_scale_nvfp4(const uint16_t *x, int64_t n_groups, int64_t rows,
+                                          int64_t cols, float *s2, uint32_t *status,
+                                          cudaStream_t stream);
+
 /* NVFP4 quantization with a caller-given global scale per group.
  * Source: josch15366/Qwen3.8-Flash-Next-NVFP4-LocalHessian-Experts,
  * introduction: gate and up share one weight_scale_2, and an activation's

@@ -217,6 +217,27 @@ mxq_status mxq_quantize_nvfp4(const uint16_t *x, int64_t n_groups, int64_t rows,
     return e == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
 }
 
+mxq_status mxq_global_scale_nvfp4(const uint16_t *x, int64_t n_groups, int64_t rows, int64_t cols, float *s2,
+                                  uint32_t *status, cudaStream_t stream)
+{
+    const ApiRange range_("mxq_global_scale_nvfp4");
+    if (n_groups < 0 || rows < 0 || cols < 0)
+        return MXQ_ERR_INVALID_ARG;
+    if (cols % 16 != 0)
+        return MXQ_ERR_SHAPE;
+    int64_t gsize, total;
+    if (!mul_ok(rows, cols, &gsize) || !mul_ok(gsize, n_groups, &total) || total > (INT64_MAX / 4))
+        return MXQ_ERR_SHAPE;
+    if (n_groups == 0)
+        return MXQ_OK;
+    if (!x || !s2 || !status)
+        return MXQ_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(s2, 4) || !aligned(status, 4))
+        return MXQ_ERR_ALIGN;
+    return launch_global_scale(x, n_groups, gsize / 16, s2, status, stream) == cudaSuccess ? MXQ_OK
+                                                                                          : MXQ_ERR_CUDA;
+}
+
 mxq_status mxq_quantize_nvfp4_s2(const uint16_t *x, int64_t n_groups, int64_t rows, int64_t cols,
                                  const float *s2_in, mxq_scale_mode mode, mxq_layout layout,
                                  uint8_t *codes, uint8_t *scales, uint32_t *mbits, uint32_t *m4_count,

@@ -77,6 +77,10 @@ size_t nvfp4_slots_offset(int64_t n_groups);
 
 cudaError_t launch_group_amax(const uint16_t *x, int64_t n_groups, int64_t nb,
                               uint32_t *amax_bits, uint32_t *status, cudaStream_t s);
+// s2 = RN32(amax_g / 2688) per group, written to s2 (which holds the running
+// amax bits in between).
+cudaError_t launch_global_scale(const uint16_t *x, int64_t n_groups, int64_t nb, float *s2, uint32_t *status,
+                                cudaStream_t s);
 // Block quantizer of the two-pass schedule; the group scale comes from
 // amax_bits (s2_in NULL; s2 written) or from the caller's s2_in.
 cudaError_t launch_nvfp4_quant(const uint16_t *x, int64_t n_groups, int64_t nb, int four_six,

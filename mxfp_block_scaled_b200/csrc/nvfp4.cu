@@ -55,6 +55,28 @@ group_amax_kernel(const uint4 *__restrict__ x, int64_t n_groups, int64_t nb,
     }
 }
 
+// s2 = RN32(amax / 2688) in place: word g holds the group's amax as bf16
+// magnitude bits (group_amax_kernel) and becomes its fp32 global scale.
+__global__ void global_scale_kernel(uint32_t *__restrict__ s2_bits, int64_t n_groups)
+{
+    const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (g < n_groups)
+        s2_bits[g] = __float_as_uint(__fdiv_rn(__uint_as_float(s2_bits[g] << 16), kGlobalDivisor));
+}
+
+cudaError_t launch_global_scale(const uint16_t *x, int64_t n_groups, int64_t nb, float *s2, uint32_t *status,
+                                cudaStream_t s)
+{
+    uint32_t *bits = reinterpret_cast<uint32_t *>(s2);
+    cudaError_t e = cudaMemsetAsync(bits, 0, (size_t)n_groups * sizeof(uint32_t), s);
+    if (e == cudaSuccess)
+        e = launch_group_amax(x, n_groups, nb, bits, status, s);
+    if (e != cudaSuccess)
+        return e;
+    global_scale_kernel<<<(unsigned)((n_groups + 255) / 256), 256, 0, s>>>(bits, n_groups);
+    return cudaGetLastError();
+}
+
 // grid = (tiles of 512 blocks, groups).  Thread t of a tile handles blocks
 // t and t + 256, so each warp covers 32 consecutive blocks per step and its
 // M bits form one 32-bit word.  The group's global scale is either formed

@@ -31,7 +31,7 @@ LAYOUT = {"linear": 0, "swizzled_128x4": 1}
 OP = {"quantize_nvfp4": 0, "quantize_act": 1, "dequant_relerr": 2}
 
 EXPORTED = ("mxq_version", "mxq_status_string", "mxq_scale_bytes", "mxq_workspace_bytes",
-            "mxq_quantize_nvfp4", "mxq_quantize_nvfp4_s2", "mxq_quantize_nvfp4_weighted",
+            "mxq_quantize_nvfp4", "mxq_global_scale_nvfp4", "mxq_quantize_nvfp4_s2", "mxq_quantize_nvfp4_weighted",
             "mxq_quantize_mx", "mxq_requant_fp8_mx", "mxq_quantize_act", "mxq_dequant_relerr",
             "mxq_dequant_relerr_noalloc", "mxq_census_reset", "mxq_census_add")
 
@@ -71,6 +71,8 @@ def load(path=LIB_PATH):
     L.mxq_workspace_bytes.argtypes = [i32, i64, i64, i64]
     L.mxq_quantize_nvfp4.restype = i32
     L.mxq_quantize_nvfp4.argtypes = [vp, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.mxq_global_scale_nvfp4.restype = i32
+    L.mxq_global_scale_nvfp4.argtypes = [vp, i64, i64, i64, vp, vp, vp]
     L.mxq_quantize_nvfp4_s2.restype = i32
     L.mxq_quantize_nvfp4_s2.argtypes = [vp, i64, i64, i64, vp, i32, i32, vp, vp, vp, vp, vp, vp]
     L.mxq_census_reset.restype = i32
@@ -178,6 +180,14 @@ def mxq_quantize_nvfp4(x, n_groups, rows, cols, mode, layout, codes, scales, s2,
                                    _p(scales), _p(s2), _p(mbits), _p(m4_count), _p(status),
                                    _p(workspace), _nbytes(workspace), _stream(stream))
     _check("mxq_quantize_nvfp4", rc)
+
+
+def mxq_global_scale_nvfp4(x, n_groups, rows, cols, s2, status, stream=None):
+    _need("x", x, 2 * n_groups * rows * cols)
+    _need("s2", s2, 4 * n_groups)
+    _need("status", status, 4)
+    rc = load().mxq_global_scale_nvfp4(_p(x), n_groups, rows, cols, _p(s2), _p(status), _stream(stream))
+    _check("mxq_global_scale_nvfp4", rc)
 
 
 def mxq_quantize_nvfp4_s2(x, n_groups, rows, cols, s2_in, mode, layout, codes, scales, mbits, m4_count,
@@ -358,6 +368,17 @@ def quantize_nvfp4_s2(x, s2_in, mode="four_six", with_mbits=True, stream=None, l
     mxq_quantize_nvfp4_s2(x, G, R, C, s2_in, mode, layout, out["codes"], out["scales"], out["mbits"],
                           out["m4_count"], out["status"], stream)
     return out
+
+
+def global_scale_nvfp4(x, stream=None):
+    """x: bf16 [G, R, C].  Returns (s2 [G] fp32, status [1]) on the device:
+    s2 = RN32(amax_g / 2688) per group."""
+    _bf16(x)
+    G, R, C = x.shape
+    s2 = torch.empty(max(G, 1), dtype=torch.float32, device=x.device)
+    status = torch.zeros(1, dtype=torch.int32, device=x.device)
+    mxq_global_scale_nvfp4(x, G, R, C, s2, status, stream)
+    return s2[:G], status
 
 
 class Census:

@@ -60,8 +60,9 @@ def test_allocating_wrappers_pass_the_checks(rec, layout):
     for fmt, mode in (("nvfp4", "rtn"), ("nvfp4", "four_six"), ("mxfp8", "rtn"), ("mxfp4", "rtn")):
         mxq.quantize_act(_bf16(5, C), fmt, mode=mode, layout=layout)
     mxq.quantize_nvfp4_s2(x, torch.ones(G), layout=layout)
+    mxq.global_scale_nvfp4(x)
     names = [c[0] for c in rec.calls]
-    assert names.count("mxq_quantize_nvfp4_s2") == 1
+    assert names.count("mxq_quantize_nvfp4_s2") == 1 and names.count("mxq_global_scale_nvfp4") == 1
     assert names.count("mxq_quantize_nvfp4") == 1 and names.count("mxq_quantize_nvfp4_weighted") == 2
     assert names.count("mxq_quantize_mx") == 2 and names.count("mxq_requant_fp8_mx") == 2
     assert names.count("mxq_quantize_act") == 4 and names.count("mxq_dequant_relerr") == 3

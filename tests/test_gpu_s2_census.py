@@ -1,4 +1,4 @@
-"""GPU parity of two C-ABI entry points with the CPU oracle.
+"""GPU parity of three C-ABI entry points with the CPU oracle.
 
 * mxq_quantize_nvfp4_s2, NVFP4 with a caller-given global scale per group
   (josch15366/Qwen3.8-Flash-Next-NVFP4-LocalHessian-Experts, introduction:
@@ -6,6 +6,8 @@
   quantized with the scale they share, equal the fused-slab call byte for
   byte and the oracle; scales the caller got elsewhere (saturating,
   zero, invalid) follow the oracle or set the status word.
+* mxq_global_scale_nvfp4, the global scale alone: the quantizer's bits and
+  the oracle's, and with mxq_quantize_nvfp4_s2 the quantizer's outputs.
 * mxq_census_add, the census of a conversion (dabsLabs/Qwen3.8-Flash-Next-
   NVFP4, metric table and "What makes this build different"): mean and max
   relative error, SSE(chosen) / SSE(RTN) - 1 and the M=4 fraction against the
@@ -158,3 +160,35 @@ def test_census_is_deterministic_and_accumulates_in_call_order():
     assert a["blocks"] == one["blocks"] and a["blocks_m4"] == one["blocks_m4"]   # MX adds no blocks
     assert a["max_relerr"] == max(one["max_relerr"], layers.census([mx])["max_relerr"])
     assert np.isnan(a["sse_vs_rtn"])                     # no RTN counterparts were given
+
+
+@pytest.mark.parametrize("shape", [(8, 256, 256), (3, 5, 48), (2, 70, 256)])
+def test_global_scale_alone_matches_the_quantizer_and_the_oracle(shape):
+    """mxq_global_scale_nvfp4 (steps a1-a2 alone) writes the bits
+    mxq_quantize_nvfp4 writes, and RN32(amax_g / 2688) of the oracle; with
+    mxq_quantize_nvfp4_s2 it reproduces mxq_quantize_nvfp4 byte for byte."""
+    G, R, C = shape
+    g = torch.Generator().manual_seed(G * 31 + R)
+    x = (torch.randn(shape, generator=g) * 0.05).to(torch.bfloat16).cuda()
+    s2, st = mxq.global_scale_nvfp4(x)
+    full = mxq.quantize_nvfp4(x, mode="four_six")
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    _, _, os2, _ = oracle.quantize_nvfp4(bits(x), mode=1)
+    assert np.array_equal(s2.cpu().numpy().view(np.uint32), os2.view(np.uint32))
+    assert np.array_equal(s2.cpu().numpy().view(np.uint32), full["s2"].cpu().numpy().view(np.uint32))
+    two = _run_s2(x, s2)
+    assert torch.equal(two["codes"], full["codes"]) and torch.equal(two["scales"], full["scales"])
+    # gate and up held apart: the larger of the halves' scales is the shared one
+    sg, _ = mxq.global_scale_nvfp4(x[:, :R // 2].contiguous()) if R % 2 == 0 else (s2, None)
+    su, _ = mxq.global_scale_nvfp4(x[:, R // 2:].contiguous()) if R % 2 == 0 else (s2, None)
+    assert torch.equal(torch.maximum(sg, su), s2)
+
+
+def test_global_scale_reports_nonfinite_input():
+    x = (torch.randn((2, 16, 64)) * 0.1).to(torch.bfloat16)
+    xb = bits(x).copy()
+    xb[1, 2, 3] = 0x7FC0                                   # NaN
+    _, st = mxq.global_scale_nvfp4(to_dev_bf16(xb))
+    torch.cuda.synchronize()
+    assert int(st.item()) & mxq.DEV_NONFINITE_INPUT
