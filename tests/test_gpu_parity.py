@@ -260,6 +260,26 @@ def test_deterministic_and_canaries():
         assert torch.equal(a, b)
 
 
+@pytest.mark.parametrize("shape", [(4, 64, 512), (3, 96, 16 * 64)])
+def test_m4_count_with_and_without_m_bits(shape):
+    """The M=4 count per group is the same whether the M bits are stored
+    (counted from them after the quantizer) or not (counted inside it), and
+    equals the oracle's."""
+    G, R, C = shape
+    x, _ = workloads.tiny_moe_layer(seed=11, experts=G, hidden=C, inter=R // 2)
+    x = x.cuda()
+    a = mxq.quantize_nvfp4(x, with_mbits=True)
+    b = mxq.quantize_nvfp4(x, with_mbits=False)
+    torch.cuda.synchronize()
+    assert int(a["status"].item()) == 0 and int(b["status"].item()) == 0
+    assert torch.equal(a["codes"], b["codes"]) and torch.equal(a["scales"], b["scales"])
+    _, _, _, m4 = oracle.quantize_nvfp4(bits(x).reshape(G, R, C), mode=1)
+    want = m4.reshape(G, -1).sum(1)
+    assert np.array_equal(a["m4_count"].cpu().numpy()[:G], want)
+    assert np.array_equal(b["m4_count"].cpu().numpy()[:G], want)
+    assert np.array_equal(mbits_to_bytes(a["mbits"], G * R * C // 16), m4.reshape(-1))
+
+
 # ------------------------------------------------------------------- MX --
 @pytest.mark.parametrize("fmt", ["mxfp8", "mxfp4"])
 def test_shared_expert_mx_bit_exact_dense_and_padded(fmt):
