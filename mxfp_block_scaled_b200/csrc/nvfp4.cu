@@ -114,7 +114,12 @@ nvfp4_quant_kernel(const uint4 *__restrict__ x, int64_t n_groups, int64_t nb,
         __syncthreads();
         const GroupConst gc = s_gc;
         uint32_t my_m4 = 0;
-        for (int64_t tile = blockIdx.x; tile * kNvTileBlocks < nb; tile += gridDim.x) {
+        // Tiles in reverse order: pass 1 read the group front to back, so
+        // its last part is the part still in L2 (a group larger than L2, an
+        // activation tile of many tokens, then reads that part from L2).
+        const int64_t ntiles = (nb + kNvTileBlocks - 1) / kNvTileBlocks;
+        for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
+            const int64_t tile = ntiles - 1 - t;
             const int64_t b0 = tile * kNvTileBlocks + threadIdx.x;
             uint4 v[2][2];
 #pragma unroll
