@@ -186,6 +186,15 @@ __device__ __forceinline__ float2 rcp2_rn_mid(float2 d)
     return __ffma2_rn(y0, e, y0);
 }
 
+// One lane of rcp2_rn_mid: the same operations on a single value.
+__device__ __forceinline__ float rcp_rn_mid(float d)
+{
+    float y0;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y0) : "f"(d));
+    const float e = __fmaf_rn(-d, y0, 1.0f);
+    return __fmaf_rn(y0, e, y0);
+}
+
 // ---- division by a run-time invariant divisor ---------------------------
 // q = n / d for unsigned 32-bit n and 1 <= d < 2^31 with one high multiply
 // (Granlund and Montgomery, "Division by invariant integers using

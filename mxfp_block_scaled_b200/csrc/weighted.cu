@@ -49,19 +49,21 @@ __device__ __forceinline__ double block_wsse(const double (&xd)[16], const doubl
 }
 
 // The same objective in fp32 pairs, for the filter below:
-// W32 = sum h RN32(x - q D s2)^2: q D is exact in fp32 (2 + 4 significant
-// bits) and each error term is one FMA of it with -s2 (one rounding), then
-// one rounding per product and sum.  q: the candidate's decoded values as
-// f16x2 pairs.
+// W32 = sum h RN32(x - q d)^2 with d = RN32(D s2), the candidate's divisor:
+// each error term is one FMA (the product q d exact inside it, one
+// rounding), then one rounding per product and sum.  Against the exact
+// error x - q D s2 the divisor's rounding moves a term by at most
+// 2^-24 |q D s2|, the same size as rounding the dequantized value before
+// the subtraction, which the bound below covers.  q: the candidate's
+// decoded values as f16x2 pairs.
 __device__ __forceinline__ float block_wsse32(const float2 (&xf)[8], const float2 (&h2)[8], const uint32_t (&q)[8],
-                                              float D, float s2)
+                                              float d)
 {
-    const float2 D2 = make_float2(D, D), NS2 = make_float2(-s2, -s2);
+    const float2 ND = make_float2(-d, -d);
     float2 acc = make_float2(0.0f, 0.0f);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-        const float2 qd = __fmul2_rn(f16x2_to_float2(q[j]), D2);           // exact
-        const float2 e = __ffma2_rn(qd, NS2, xf[j]);                        // RN32(x - q D s2)
+        const float2 e = __ffma2_rn(f16x2_to_float2(q[j]), ND, xf[j]);      // RN32(x - q d)
         acc = __ffma2_rn(h2[j], __fmul2_rn(e, e), acc);
     }
     return __fadd_rn(acc.x, acc.y);
@@ -83,16 +85,15 @@ __device__ __forceinline__ uint2 candidate_codes(const float2 (&x)[8], float d, 
 }
 
 // Error bound of W32 against the exact weighted error W, and against the
-// binary64 value the definition forms.  With u = 2^-24, A = sum h x^2 and
-// Cauchy-Schwarz on sum h |x| |e|, the one rounding of each error term costs
-// at most 2u W + u^2 W (it is relative to |e| itself), the products and the
-// eight-step pair sums at most 10u W32; bounding W by W32 the same way gives
-// |W32 - W| <= 12.1u W32 + O(u^2 W32).  The constants below were derived for
-// an earlier form that rounded the dequantized value before the subtraction,
-// |W32 - W| <= 2.1u sqrt(A W32) + 14.7u W32 + 4.2u^2 A, and take about twice
-// that; they cover the present form with room, as well as the binary64
-// procedure's own error (below 2^-48 W) and the error of forming the bound
-// in fp32.
+// binary64 value the definition forms.  With u = 2^-24 and A = sum h x^2:
+// each error term is (e + eta)(1 + delta) with |eta| <= u |q D s2| <=
+// u (|x| + |e|) (the divisor's rounding) and |delta| <= u, so by
+// Cauchy-Schwarz on sum h |x| |e| the terms cost at most
+// 2.1u sqrt(A W32) + 4.2u W32 + 4.2u^2 A, and the products and the
+// eight-step pair sums at most 10.5u W32: |W32 - W| <= 2.1u sqrt(A W32) +
+// 14.7u W32 + 4.2u^2 A.  The constants below take about twice that, which
+// also covers the binary64 procedure's own error (below 2^-48 W) and the
+// error of forming the bound in fp32.
 // The last term covers terms that underflow, with every weight <= 2^40 and
 // s2 in [2^-50, 2^50] (every non-zero dequantized value normal).
 __device__ __forceinline__ float wsse_bound(float W, float sqrtA_scaled, float c_block)
@@ -233,10 +234,9 @@ nvfp4_weighted_kernel(const uint4 *__restrict__ x, int64_t n_groups, int64_t nb,
                 for (; sc <= hi; ++sc) {
                     const float D = f16x2_to_float2(e4m3x2_to_f16x2(sc)).x;
                     const float d = __fmul_rn(D, gc.s2);
-                    const float r = rcp2_rn_mid(make_float2(d, d)).x;
                     uint32_t q[8];
-                    const uint2 c = candidate_codes(xf, d, r, q);
-                    consider(sc, block_wsse32(xf, h2, q, D, gc.s2), c);
+                    const uint2 c = candidate_codes(xf, d, rcp_rn_mid(d), q);
+                    consider(sc, block_wsse32(xf, h2, q, d), c);
                 }
                 decided = lb > __fadd_rn(bw, be);
             }

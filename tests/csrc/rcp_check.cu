@@ -1,7 +1,7 @@
-// Exhaustive device check of rcp2_rn_mid (mxq_device.cuh): for every fp32
-// significand at every exponent of [2^-60, 2^60), both signs, the refined
-// reciprocal pair must equal __frcp_rn (CUDA's correctly rounded
-// reciprocal) bit for bit.  Prints "mismatches N first 0x........" and
+// Exhaustive device check of rcp2_rn_mid and its one-lane form rcp_rn_mid
+// (mxq_device.cuh): for every fp32 significand at every exponent of
+// [2^-60, 2^60), both signs, the refined reciprocals must equal __frcp_rn
+// (CUDA's correctly rounded reciprocal) bit for bit.  Prints "mismatches N first 0x........" and
 // exits 0 when the run itself succeeded (the count is judged by the test).
 #include <stdio.h>
 #include "mxq_device.cuh"
@@ -14,8 +14,10 @@ __global__ void rcp_check_kernel(unsigned long long *bad, unsigned int *first)
             const float d = __uint_as_float((e << 23) | i);
             const float want = __frcp_rn(d);
             const float2 got = mxq::rcp2_rn_mid(make_float2(d, -d));
+            const float one = mxq::rcp_rn_mid(e & 1u ? -d : d);
             if (__float_as_uint(got.x) != __float_as_uint(want) ||
-                __float_as_uint(got.y) != (__float_as_uint(want) ^ 0x80000000u)) {
+                __float_as_uint(got.y) != (__float_as_uint(want) ^ 0x80000000u) ||
+                __float_as_uint(one) != (__float_as_uint(want) ^ (e & 1u ? 0x80000000u : 0u))) {
                 atomicAdd(bad, 1ull);
                 atomicMin(first, (e << 23) | i);
             }

@@ -116,15 +116,14 @@ def test_ties_and_near_ties():
 
 # ---- the weighted search's fp32 scores and their bound -------------------
 def _wsse32(xs, hs, codes, D, s2):
-    """The kernel's fp32 weighted error of one candidate: per element
-    e = RN(x - RN(q D) s2) (one FMA; q D is exact), then
-    acc = RN(h RN(e e) + acc) in two interleaved partial sums (even / odd
-    elements), added at the end."""
+    """The kernel's fp32 weighted error of one candidate: with the
+    candidate's divisor d = RN(D s2), per element e = RN(x - q d) (one FMA),
+    then acc = RN(h RN(e e) + acc) in two interleaved partial sums (even /
+    odd elements), added at the end."""
+    d = rn32(D * F(float(s2)))
     acc = [F(0), F(0)]
     for i, (x, h, c) in enumerate(zip(xs, hs, codes)):
-        qd = rn32(micro.e2m1_value(c) * D)
-        assert qd == micro.e2m1_value(c) * D               # exact, as the kernel relies on
-        e = rn32(F(float(x)) - qd * F(float(s2)))
+        e = rn32(F(float(x)) - micro.e2m1_value(c) * d)
         acc[i & 1] = rn32(F(float(h)) * rn32(e * e) + acc[i & 1])
     return rn32(acc[0] + acc[1])
 

@@ -1,5 +1,6 @@
-"""The refined reciprocal of the NVFP4 fast path (rcp2_rn_mid: hardware
-approximation + one Newton-Raphson step) equals CUDA's correctly rounded
+"""The refined reciprocal of the NVFP4 fast path (rcp2_rn_mid, and its
+one-lane form rcp_rn_mid of the weighted search: hardware approximation +
+one Newton-Raphson step) equals CUDA's correctly rounded
 reciprocal for every significand at every exponent of [2^-60, 2^60], both
 signs: the range every block-scale divisor of the fast path lies in."""
 import os
