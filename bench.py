@@ -106,13 +106,17 @@ def ncu_traffic_per_launch():
 
 
 def ncu_traffic_split():
-    """{"traffic_read": R, "traffic_write": W} per quantize launch from the
-    same summary (empty when unavailable)."""
+    """{"traffic_read": R, "traffic_write": W, "ncu_dram_gbs": G} per quantize
+    launch from the same summary (empty when unavailable); G is the captured
+    launch's DRAM bytes over its ncu duration (cold, serialised)."""
     kv = _traffic_record()
     try:
-        return {"traffic_read": float(kv["dram_read_per_call"]),
-                "traffic_write": float(kv["dram_write_per_call"])} if kv else {}
-    except (KeyError, ValueError):
+        out = {"traffic_read": float(kv["dram_read_per_call"]),
+               "traffic_write": float(kv["dram_write_per_call"])} if kv else {}
+        if kv and "ncu_capture_ns" in kv:
+            out["ncu_dram_gbs"] = float(kv["ncu_capture_dram_bytes"]) / float(kv["ncu_capture_ns"])
+        return out
+    except (KeyError, ValueError, ZeroDivisionError):
         return {}
 
 
