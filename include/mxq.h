@@ -48,6 +48,12 @@
  *   - Input bf16 data must be 16-byte aligned; code and scale outputs
  *     must be 16-byte aligned; fp32 / fp64 arrays naturally aligned.
  *     Otherwise MXQ_ERR_ALIGN.
+ *   - Inputs without elements are valid.  A group with no elements has
+ *     amax 0, so its s2 is 0 and its M=4 count 0; an empty activation tile
+ *     has input_scale 0; a tensor with no elements has both verifier sums
+ *     0 and a relative error of 0.  Pointers to data of zero bytes (x,
+ *     codes, scales, M bits, the workspace) may then be NULL; the global
+ *     scales, status and per-group or per-tensor outputs are still required.
  *   - Tensors are row-major and contiguous; blocks run along the last
  *     dimension (`cols`), which must be a multiple of the block size
  *     (16 for NVFP4, 32 for MX), otherwise MXQ_ERR_SHAPE.

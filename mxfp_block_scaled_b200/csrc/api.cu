@@ -123,6 +123,21 @@ size_t mxq_workspace_bytes(mxq_op op, int64_t n, int64_t rows, int64_t cols)
     return 0;
 }
 
+// Groups with no elements: their amax is 0, so s2 = RN32(0 / 2688) = 0 and
+// no block exists; x, codes, scales and the workspace are not needed.
+static mxq_status empty_groups(int64_t n_groups, float *s2, uint32_t *m4_count, uint32_t *status,
+                               cudaStream_t stream)
+{
+    if (!s2 || !status)
+        return MXQ_ERR_INVALID_ARG;
+    if (!aligned(s2, 4) || !aligned(status, 4) || (m4_count && !aligned(m4_count, 4)))
+        return MXQ_ERR_ALIGN;
+    cudaError_t e = cudaMemsetAsync(s2, 0, (size_t)n_groups * sizeof(float), stream);
+    if (e == cudaSuccess && m4_count)
+        e = cudaMemsetAsync(m4_count, 0, (size_t)n_groups * sizeof(uint32_t), stream);
+    return e == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
+}
+
 mxq_status mxq_quantize_nvfp4(const uint16_t *x, int64_t n_groups, int64_t rows, int64_t cols,
                               mxq_scale_mode mode, mxq_layout layout, uint8_t *codes,
                               uint8_t *scales, float *s2,
@@ -146,6 +161,8 @@ mxq_status mxq_quantize_nvfp4(const uint16_t *x, int64_t n_groups, int64_t rows,
         return MXQ_ERR_SHAPE;   // tiled offsets index the blocks of a group in 32 bits
     if (n_groups == 0)
         return MXQ_OK;
+    if (total == 0)   // groups without elements: amax 0, so s2 = 0 and M=4 count 0
+        return empty_groups(n_groups, s2, m4_count, status, stream);
     if (!x || !codes || !scales || !s2 || !status)
         return MXQ_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(scales, 16) || !aligned(s2, 4) ||
@@ -230,6 +247,8 @@ mxq_status mxq_global_scale_nvfp4(const uint16_t *x, int64_t n_groups, int64_t r
         return MXQ_ERR_SHAPE;
     if (n_groups == 0)
         return MXQ_OK;
+    if (total == 0)
+        return empty_groups(n_groups, s2, nullptr, status, stream);
     if (!x || !s2 || !status)
         return MXQ_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(s2, 4) || !aligned(status, 4))
@@ -260,7 +279,9 @@ mxq_status mxq_quantize_nvfp4_s2(const uint16_t *x, int64_t n_groups, int64_t ro
         return MXQ_ERR_SHAPE;
     if (n_groups == 0)
         return MXQ_OK;
-    if (!x || !s2_in || !codes || !scales || !status)
+    // without elements x, codes and scales are not read or written (the
+    // kernel still checks the given scales)
+    if ((total > 0 && (!x || !codes || !scales)) || !s2_in || !status)
         return MXQ_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(scales, 16) || !aligned(s2_in, 4) ||
         !aligned(status, 4) || (mbits && !aligned(mbits, 4)) || (m4_count && !aligned(m4_count, 4)))
@@ -304,6 +325,8 @@ mxq_status mxq_quantize_nvfp4_weighted(const uint16_t *x, int64_t n_groups, int6
         return MXQ_ERR_SHAPE;
     if (n_groups == 0)
         return MXQ_OK;
+    if (total == 0)
+        return empty_groups(n_groups, s2, nullptr, status, stream);
     if (!x || !h || !codes || !scales || !s2 || !status)
         return MXQ_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(h, 16) || !aligned(codes, 16) || !aligned(scales, 16) ||
@@ -466,6 +489,16 @@ mxq_status mxq_dequant_relerr(const uint16_t *x, const uint8_t *codes, const uin
     if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(scales, 16) || (s2 && !aligned(s2, 4)) ||
         !aligned(sum_sq_err, 8) || !aligned(sum_sq_ref, 8) || (relerr && !aligned(relerr, 8)))
         return MXQ_ERR_ALIGN;
+    if (total == 0) {
+        // tensors without elements: both sums 0 and a relative error of 0
+        // (the convention for a tensor reproduced exactly); nothing is read
+        cudaError_t e = cudaMemsetAsync(sum_sq_err, 0, (size_t)n_tensors * sizeof(double), stream);
+        if (e == cudaSuccess)
+            e = cudaMemsetAsync(sum_sq_ref, 0, (size_t)n_tensors * sizeof(double), stream);
+        if (e == cudaSuccess && relerr)
+            e = cudaMemsetAsync(relerr, 0, (size_t)n_tensors * sizeof(double), stream);
+        return e == cudaSuccess ? MXQ_OK : MXQ_ERR_CUDA;
+    }
     const size_t need = verify_workspace_bytes(n_tensors, rows, cols);
     if (!workspace || workspace_bytes < need)
         return MXQ_ERR_WORKSPACE;
