@@ -147,6 +147,38 @@ def test_empty_inputs_are_no_ops(lib):
                                   None) == 0
 
 
+def test_maximum_sizes_are_refused_before_any_launch(lib):
+    vp = ctypes.c_void_p
+    fake = vp(0x1000)
+    # element count beyond int64 / 4
+    assert lib.mxq_quantize_nvfp4(fake, 1 << 30, 1 << 20, 1 << 20, 1, 0, fake, fake, fake, None, None,
+                                  fake, fake, 4096, None) == 2
+    # tiled scales: a group of 2^32 blocks does not fit the 32-bit tile offsets
+    assert lib.mxq_quantize_nvfp4(fake, 1, 1 << 22, 1 << 14, 1, 1, fake, fake, fake, None, None, fake,
+                                  fake, 4096, None) == 2
+    assert lib.mxq_quantize_mx(fake, 1 << 22, 1 << 15, 2, 32, 1, fake, fake, None, None) == 2
+    # the verifier indexes its chunks in 32 bits
+    assert lib.mxq_dequant_relerr(fake, fake, fake, fake, 0, 0, 1 << 31, 16, 1024, 1, fake, fake, None,
+                                  fake, 1 << 40, None) == 2
+    # the largest layer of the workloads is accepted by the same checks (the workspace sizes agree)
+    assert lib.mxq_workspace_bytes(0, 512, 1536, 2048) > 0
+    assert lib.mxq_workspace_bytes(2, 1536, 768, 2048) > 0
+
+
+def test_groups_without_elements_still_need_their_scales(lib):
+    vp = ctypes.c_void_p
+    fake = vp(0x1000)
+    # no elements: x, codes, scales and the workspace may be NULL, but s2 and status are written
+    assert lib.mxq_quantize_nvfp4(None, 3, 0, 32, 1, 0, None, None, None, None, None, fake, None, 0,
+                                  None) == 1
+    assert lib.mxq_quantize_nvfp4(None, 3, 0, 32, 1, 0, None, None, fake, None, None, None, None, 0,
+                                  None) == 1
+    assert lib.mxq_global_scale_nvfp4(None, 3, 0, 32, None, fake, None) == 1
+    assert lib.mxq_quantize_nvfp4_s2(None, 3, 0, 32, None, 1, 0, None, None, None, None, fake, None) == 1
+    assert lib.mxq_quantize_nvfp4(None, 3, 0, 32, 1, 0, None, None, vp(0x1002), None, None, fake, None,
+                                  0, None) == 3
+
+
 def test_product_path_refuses_to_run_without_the_library(tmp_path):
     from mxfp_block_scaled_b200 import mxq
     with pytest.raises(RuntimeError, match="not built"):
