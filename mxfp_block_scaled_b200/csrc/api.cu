@@ -206,14 +206,16 @@ mxq_status mxq_quantize_nvfp4(const uint16_t *x, int64_t n_groups, int64_t rows,
         e = cudaMemsetAsync(m4_count, 0, (size_t)n_groups * sizeof(uint32_t), stream);
     if (e != cudaSuccess)
         return MXQ_ERR_CUDA;
-    // single pass (one HBM read of x) when the shape allows it and there
-    // are several groups: a lone group has nothing to overlap its grid-wide
-    // amax with, and two passes over a tile that stays in L2 are faster
+    // single pass (one HBM read of x) when the shape allows it: several
+    // groups overlap each group's grid-wide amax with the quantization of
+    // earlier ones; a lone group whose blocks fit the SMs' shared memory is
+    // read once into it by one grid
     if (n_groups > 1)
         e = launch_nvfp4_fused(x, n_groups, nb, mode == MXQ_SCALE_FOUR_SIX, slots, amax_bits, codes, scales, sl,
                                s2, mbits, m4_count, status, stream);
-    else
-        e = cudaErrorNotSupported;
+    else    // one group that fits the SMs' shared memory: one grid, one read
+        e = launch_nvfp4_grid(x, nb, mode == MXQ_SCALE_FOUR_SIX, codes, scales, sl, s2, mbits, m4_count, status,
+                              amax_bits, slots, stream);
     if (e == cudaSuccess)
         return MXQ_OK;
     if (e != cudaErrorNotSupported)

@@ -98,6 +98,14 @@ constexpr int64_t kSmallMaxBlocks = 96 * 1024;    // 3 MiB of bf16
 cudaError_t launch_nvfp4_small(const uint16_t *x, int64_t nb, int four_six, uint8_t *codes, uint8_t *scales,
                                const ScaleLayout &sl, float *s2, uint32_t *mbits, uint32_t *m4_count,
                                uint32_t *status, cudaStream_t s);
+// One group too large for a cluster whose blocks still fit the SMs' shared
+// memory (an activation tile of up to several thousand tokens): a
+// cooperative grid of one CTA per SM, one HBM read of the group
+// (cudaErrorNotSupported where the device or the size does not allow it).
+// `arrived` and `slots` (kMaxFusedCtas words) must start at zero.
+cudaError_t launch_nvfp4_grid(const uint16_t *x, int64_t nb, int four_six, uint8_t *codes, uint8_t *scales,
+                              const ScaleLayout &sl, float *s2, uint32_t *mbits, uint32_t *m4_count,
+                              uint32_t *status, uint32_t *arrived, unsigned long long *slots, cudaStream_t s);
 cudaError_t launch_nvfp4_weighted(const uint16_t *x, int64_t n_groups, int64_t nb, int64_t cols,
                                   const uint32_t *amax_bits, const float *h, int64_t h_stride,
                                   uint8_t *codes, uint8_t *scales, const ScaleLayout &sl, float *s2,

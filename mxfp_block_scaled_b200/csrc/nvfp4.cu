@@ -877,6 +877,213 @@ cudaError_t launch_nvfp4_small(const uint16_t *x, int64_t nb, int four_six, uint
     return e;
 }
 
+// ---------------------------------------------------------------------------
+// One group too large for a cluster whose blocks still fit the SMs' shared
+// memory (an activation tile of about 800 to 7000 tokens of 2048 values):
+// a cooperative grid of one CTA per SM (all resident at once).  Each CTA
+// brings its share into shared memory with bulk copies issued together (the
+// whole share in flight), reduces its amax piece by piece as the pieces
+// land, publishes it as a tagged 64-bit slot (tag and value in one store)
+// and counts its arrival; once every CTA has arrived and every slot shows
+// its tag (bounded waits), each CTA takes the group amax from the slots and
+// quantizes its share from shared memory.  One HBM read of the group, one
+// launch.  Shares are multiples of 32 blocks, so each warp's M bits fill one
+// word.  On a time-out the CTA sets MXQ_DEV_WAIT_TIMEOUT and returns.
+// ---------------------------------------------------------------------------
+constexpr int kGridThreads = 512;
+constexpr int kGridPieces = 4;
+
+template <bool FOUR_SIX, bool SWZ>
+__global__ void __launch_bounds__(kGridThreads, 1)
+nvfp4_grid_kernel(const uint4 *__restrict__ x, int64_t nb, int64_t share, uint2 *__restrict__ codes,
+                  uint8_t *__restrict__ scales, const ScaleLayout sl, float *__restrict__ s2_out,
+                  uint32_t *__restrict__ mbits, uint32_t *__restrict__ m4_count, uint32_t *__restrict__ status,
+                  uint32_t *arrived, unsigned long long *slots)
+{
+    extern __shared__ __align__(128) uint8_t gsmem[];
+    uint64_t *bar = reinterpret_cast<uint64_t *>(gsmem);            // kGridPieces barriers
+    uint4 *tile = reinterpret_cast<uint4 *>(gsmem + 128);           // 2 vectors per block of the share
+    __shared__ uint32_t s_warp[kGridThreads / 32];
+    __shared__ GroupConst s_gc;
+    __shared__ uint32_t s_m4;
+    __shared__ int s_arrived;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t P = gridDim.x;
+    const int64_t b0 = min(nb, (int64_t)blockIdx.x * share);
+    const int n = (int)(min(nb, b0 + share) - b0);
+    const int piece = ((n + kGridPieces - 1) / kGridPieces + 31) / 32 * 32;   // blocks, a multiple of 32
+
+    if (threadIdx.x == 0) {
+        for (int k = 0; k < kGridPieces; ++k)
+            mbar_init(bar + k, 1);
+        s_m4 = 0;
+        fence_mbar_init();
+        for (int k = 0; k < kGridPieces; ++k) {
+            const int lo = k * piece, cnt = min(n, lo + piece) - lo;
+            if (cnt > 0) {
+                mbar_arrive_expect_tx(bar + k, (uint32_t)cnt * 32u);
+                bulk_g2s(reinterpret_cast<uint8_t *>(tile) + (size_t)lo * 32, x + 2 * (b0 + lo),
+                         (uint32_t)cnt * 32u, bar + k);
+            }
+        }
+    }
+    __syncthreads();                                    // barriers initialised before anyone waits
+    // the CTA's amax, each piece as it lands
+    uint32_t m = 0;
+    bool landed = true;
+    for (int k = 0; k < kGridPieces && landed; ++k) {
+        const int lo = k * piece, cnt = min(n, lo + piece) - lo;
+        if (cnt <= 0)
+            break;
+        landed = false;
+        for (uint32_t i = 0; i < kSpinLimit && !landed; ++i)
+            landed = mbar_try_wait(bar + k, 0u);
+        if (landed)
+            for (int i = 2 * lo + (int)threadIdx.x; i < 2 * (lo + cnt); i += kGridThreads) {
+                const uint4 v = tile[i];
+                m = absmax_bf16x2(absmax_bf16x2(m, v.x), absmax_bf16x2(v.y, v.z));
+                m = absmax_bf16x2(m, v.w);
+            }
+    }
+    m = __reduce_max_sync(0xFFFFFFFFu, fold_halves(m));
+    if (lane == 0)
+        s_warp[warp] = m;
+    if (!__syncthreads_and(landed ? 1 : 0)) {
+        if (threadIdx.x == 0) {
+            atomicOr(status, MXQ_DEV_WAIT_TIMEOUT);
+            // let the copies still in flight land (bounded) before the CTA's
+            // shared memory is released
+            for (int k = 0; k < kGridPieces; ++k)
+                if (min(n, k * piece + piece) - k * piece > 0)
+                    for (uint32_t i = 0; i < kSpinLimit; ++i)
+                        if (mbar_try_wait(bar + k, 0u))
+                            break;
+        }
+        return;                                         // the other CTAs time out at the barrier below
+    }
+    if (threadIdx.x == 0) {
+        uint32_t a = 0;
+        for (int w = 0; w < kGridThreads / 32; ++w)
+            a = max(a, s_warp[w]);
+        st_relaxed_u64(slots + blockIdx.x, (1ull << 32) | a);
+        red_relaxed_add_u32(arrived, 1u);
+        bool all = false;
+        for (uint32_t i = 0; i < kSpinLimit && !all; ++i) {
+            all = ld_relaxed_u32(arrived) >= P;
+            if (!all)
+                __nanosleep(64);
+        }
+        s_arrived = all ? 1 : 0;
+    }
+    __syncthreads();
+    // every slot, one per thread (a slot whose store is not visible yet still
+    // reads tag 0: poll it again, bounded)
+    bool seen = s_arrived != 0;
+    uint32_t g = 0;
+    if (seen && threadIdx.x < P) {
+        unsigned long long v = ld_relaxed_u64(slots + threadIdx.x);
+        for (uint32_t i = 0; i < kSpinLimit && (v >> 32) != 1ull; ++i) {
+            __nanosleep(64);
+            v = ld_relaxed_u64(slots + threadIdx.x);
+        }
+        seen = (v >> 32) == 1ull;
+        g = (uint32_t)v;
+    }
+    g = __reduce_max_sync(0xFFFFFFFFu, g);
+    __syncthreads();                                    // s_warp is reused
+    if (lane == 0)
+        s_warp[warp] = g;
+    if (!__syncthreads_and(seen ? 1 : 0)) {
+        if (threadIdx.x == 0)
+            atomicOr(status, MXQ_DEV_WAIT_TIMEOUT);
+        return;
+    }
+    if (threadIdx.x == 0) {
+        uint32_t a = 0;
+        for (int w = 0; w < kGridThreads / 32; ++w)
+            a = max(a, s_warp[w]);
+        s_gc = make_group_const(a);
+        if (blockIdx.x == 0) {
+            s2_out[0] = s_gc.s2;
+            if (a >= 0x7F80u)
+                atomicOr(status, MXQ_DEV_NONFINITE_INPUT);
+        }
+    }
+    __syncthreads();
+    const GroupConst gc = s_gc;
+    uint32_t my_m4 = 0;
+    for (int base = 0; base < n; base += kGridThreads) {
+        const int j = base + threadIdx.x;
+        const bool live = j < n;
+        BlockOut o;
+        o.m4 = false;
+        if (live) {
+            o = quantize_block<FOUR_SIX>(tile[2 * j], tile[2 * j + 1], gc);
+            const int64_t b = b0 + j;
+            codes[b] = o.codes;
+            scales[SWZ ? tiled_scale_offset(sl, 0, (uint32_t)b) : (uint64_t)b] = (uint8_t)o.scale;
+        }
+        if (mbits) {
+            const uint32_t word = __ballot_sync(0xFFFFFFFFu, o.m4);
+            const int64_t first = b0 + base + 32 * warp;   // first block of this warp's word
+            if (lane == 0 && first < b0 + n)
+                mbits[first >> 5] = word;
+        }
+        my_m4 += o.m4 ? 1u : 0u;
+    }
+    if (FOUR_SIX && m4_count) {
+        const uint32_t wsum = __reduce_add_sync(0xFFFFFFFFu, my_m4);
+        if (lane == 0 && wsum)
+            atomicAdd(&s_m4, wsum);
+        __syncthreads();
+        if (threadIdx.x == 0 && s_m4)
+            atomicAdd(m4_count, s_m4);
+    }
+}
+
+cudaError_t launch_nvfp4_grid(const uint16_t *x, int64_t nb, int four_six, uint8_t *codes, uint8_t *scales,
+                              const ScaleLayout &sl, float *s2, uint32_t *mbits, uint32_t *m4_count,
+                              uint32_t *status, uint32_t *arrived, unsigned long long *slots, cudaStream_t s)
+{
+    if (nb <= 0 || !arrived || !slots)
+        return cudaErrorNotSupported;
+    int dev = 0, coop = 0, max_optin = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+        return cudaErrorNotSupported;
+    const int sms = sm_count();
+    if (!coop || sms <= 0 || sms > kMaxFusedCtas)
+        return cudaErrorNotSupported;
+    int64_t share = (nb + sms - 1) / sms;
+    share = (share + 31) / 32 * 32;
+    const int P = (int)((nb + share - 1) / share);
+    const size_t dyn = 128 + (size_t)share * 32;
+    if (dyn + 2048 > (size_t)max_optin)                 // + static shared memory
+        return cudaErrorNotSupported;
+    const void *fn = four_six ? (sl.swz ? (const void *)nvfp4_grid_kernel<true, true>
+                                        : (const void *)nvfp4_grid_kernel<true, false>)
+                              : (sl.swz ? (const void *)nvfp4_grid_kernel<false, true>
+                                        : (const void *)nvfp4_grid_kernel<false, false>);
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        return cudaErrorNotSupported;
+    }
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kGridThreads, dyn);
+    if (e != cudaSuccess || per_sm < 1) {
+        (void)cudaGetLastError();
+        return cudaErrorNotSupported;
+    }
+    const uint4 *xv = reinterpret_cast<const uint4 *>(x);
+    uint2 *cv = reinterpret_cast<uint2 *>(codes);
+    void *params[] = {(void *)&xv, (void *)&nb, (void *)&share, (void *)&cv, (void *)&scales,
+                      (void *)&sl, (void *)&s2, (void *)&mbits, (void *)&m4_count, (void *)&status,
+                      (void *)&arrived, (void *)&slots};
+    return cudaLaunchCooperativeKernel(fn, dim3((unsigned)P), dim3(kGridThreads), params, dyn, s);
+}
+
 } // namespace mxq
 
 extern "C" MXQ_API void mxq_test_stall_next_single_pass(int on)

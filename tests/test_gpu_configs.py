@@ -19,6 +19,7 @@ import torch
 
 import oracle
 from mxfp_block_scaled_b200 import layers, mxq, workloads
+from oracle.layout import to_tiled_128x4
 
 pytestmark = pytest.mark.gpu
 
@@ -227,6 +228,33 @@ def test_activation_sweep_exact(T):
     c8, s8 = oracle.quantize_mx(bits(a), "mxfp8")
     assert np.array_equal(o8["codes"].cpu().numpy(), c8)
     assert np.array_equal(o8["scales"].cpu().numpy(), s8)
+
+
+@pytest.mark.parametrize("T,H", [(1000, 2048), (2999, 1024), (7000, 2048), (9000, 2048)])
+@pytest.mark.parametrize("mode", ["rtn", "four_six"])
+@pytest.mark.parametrize("layout", ["linear", "swizzled_128x4"])
+def test_activation_tiles_one_grid(T, H, mode, layout):
+    """Tiles too large for one cluster whose blocks fit the SMs' shared
+    memory go through one cooperative grid (ragged shares, the last CTA
+    shorter; 9000 tokens exceed the shared memory and take two passes):
+    byte-exact, M bits and the M=4 count included."""
+    a = workloads.activation_tile(T, seed=T + H, device="cuda", hidden=H)
+    x = a.reshape(1, T, H)
+    o = mxq.quantize_nvfp4(x, mode=mode, layout=layout)
+    torch.cuda.synchronize()
+    assert int(o["status"].item()) == 0
+    c, s, s2, m4 = oracle.quantize_nvfp4(bits(a).reshape(1, T, H), mode=1 if mode == "four_six" else 0)
+    assert o["s2"].cpu().numpy().view(np.uint32)[0] == s2.view(np.uint32)[0]
+    assert np.array_equal(o["codes"].cpu().numpy().reshape(-1), c.reshape(-1))
+    gs = o["scales"].cpu().numpy().reshape(-1)
+    if layout == "linear":
+        assert np.array_equal(gs, s.reshape(-1))
+    else:
+        assert np.array_equal(gs, to_tiled_128x4(s.reshape(T, H // 16)))
+    gm = np.unpackbits(o["mbits"].cpu().numpy().view(np.uint8), bitorder="little")[:T * H // 16]
+    assert np.array_equal(gm, m4.reshape(-1))
+    if mode == "four_six":
+        assert int(o["m4_count"].cpu().numpy()[0]) == int(m4.sum())
 
 
 def test_activation_65536_tokens_sampled_rows():
