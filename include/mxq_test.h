@@ -11,10 +11,12 @@
 extern "C" {
 #endif
 
-/* Make the next single-pass NVFP4 launch (mxq_quantize_nvfp4 on several
- * groups whose shape the single-pass kernel holds) stall on purpose: its
- * per-SM publisher never releases a group, so every inter-CTA wait of that
- * launch runs into its iteration limit.  The launch then ORs
+/* Make the next single-pass NVFP4 launch stall on purpose.  On several
+ * groups (mxq_quantize_nvfp4 where the single-pass kernel holds the shape)
+ * its per-SM publisher never releases a group; on one group read once by a
+ * grid of CTAs (a tile too large for one cluster that fits the SMs' shared
+ * memory) the first CTA never reports its amax.  Either way every inter-CTA
+ * wait of that launch runs into its iteration limit.  The launch then ORs
  * MXQ_DEV_WAIT_TIMEOUT into *status, lets its copies in flight land and
  * returns, well under a second; the outputs of that call are undefined and
  * the device stays usable.  `on` = 0 withdraws a pending request.  The

@@ -898,7 +898,7 @@ __global__ void __launch_bounds__(kGridThreads, 1)
 nvfp4_grid_kernel(const uint4 *__restrict__ x, int64_t nb, int64_t share, uint2 *__restrict__ codes,
                   uint8_t *__restrict__ scales, const ScaleLayout sl, float *__restrict__ s2_out,
                   uint32_t *__restrict__ mbits, uint32_t *__restrict__ m4_count, uint32_t *__restrict__ status,
-                  uint32_t *arrived, unsigned long long *slots)
+                  uint32_t *arrived, unsigned long long *slots, int test_stall)
 {
     extern __shared__ __align__(128) uint8_t gsmem[];
     uint64_t *bar = reinterpret_cast<uint64_t *>(gsmem);            // kGridPieces barriers
@@ -965,10 +965,14 @@ nvfp4_grid_kernel(const uint4 *__restrict__ x, int64_t nb, int64_t share, uint2 
         uint32_t a = 0;
         for (int w = 0; w < kGridThreads / 32; ++w)
             a = max(a, s_warp[w]);
-        st_relaxed_u64(slots + blockIdx.x, (1ull << 32) | a);
-        red_relaxed_add_u32(arrived, 1u);
+        if (!test_stall || blockIdx.x != 0) {             // test hook: CTA 0 never arrives
+            st_relaxed_u64(slots + blockIdx.x, (1ull << 32) | a);
+            red_relaxed_add_u32(arrived, 1u);
+        }
+        // all CTAs are resident (cooperative launch) and arrive within
+        // microseconds; the limit is tens of milliseconds
         bool all = false;
-        for (uint32_t i = 0; i < kSpinLimit && !all; ++i) {
+        for (uint32_t i = 0; i < (kSpinLimit >> 4) && !all; ++i) {
             all = ld_relaxed_u32(arrived) >= P;
             if (!all)
                 __nanosleep(64);
@@ -982,7 +986,7 @@ nvfp4_grid_kernel(const uint4 *__restrict__ x, int64_t nb, int64_t share, uint2 
     uint32_t g = 0;
     if (seen && threadIdx.x < P) {
         unsigned long long v = ld_relaxed_u64(slots + threadIdx.x);
-        for (uint32_t i = 0; i < kSpinLimit && (v >> 32) != 1ull; ++i) {
+        for (uint32_t i = 0; i < (kSpinLimit >> 4) && (v >> 32) != 1ull; ++i) {
             __nanosleep(64);
             v = ld_relaxed_u64(slots + threadIdx.x);
         }
@@ -1078,9 +1082,10 @@ cudaError_t launch_nvfp4_grid(const uint16_t *x, int64_t nb, int four_six, uint8
     }
     const uint4 *xv = reinterpret_cast<const uint4 *>(x);
     uint2 *cv = reinterpret_cast<uint2 *>(codes);
+    int test_stall = g_test_stall.exchange(0) ? 1 : 0;
     void *params[] = {(void *)&xv, (void *)&nb, (void *)&share, (void *)&cv, (void *)&scales,
                       (void *)&sl, (void *)&s2, (void *)&mbits, (void *)&m4_count, (void *)&status,
-                      (void *)&arrived, (void *)&slots};
+                      (void *)&arrived, (void *)&slots, (void *)&test_stall};
     return cudaLaunchCooperativeKernel(fn, dim3((unsigned)P), dim3(kGridThreads), params, dyn, s);
 }
 

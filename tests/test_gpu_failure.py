@@ -53,6 +53,26 @@ def test_stalled_single_pass_reports_wait_timeout_and_the_device_recovers():
     _expect_exact(gu, out)
 
 
+def test_stalled_one_grid_group_reports_wait_timeout_and_the_device_recovers():
+    """The lone-group grid (an activation tile of 4096 tokens): its first CTA
+    never reports its amax, every other CTA's bounded wait runs out."""
+    a = workloads.activation_tile(4096, seed=5)
+    x = a.cuda().reshape(1, 4096, -1)
+    lib = mxq.load()
+    torch.cuda.synchronize()
+    lib.mxq_test_stall_next_single_pass(1)
+    t0 = time.perf_counter()
+    out = mxq.quantize_nvfp4(x)
+    torch.cuda.synchronize()
+    elapsed = time.perf_counter() - t0
+    assert int(out["status"].item()) & mxq.DEV_WAIT_TIMEOUT
+    assert elapsed < 5.0, elapsed
+    out = mxq.quantize_nvfp4(x)
+    torch.cuda.synchronize()
+    assert int(out["status"].item()) == 0
+    _expect_exact(a.reshape(1, 4096, -1), out)
+
+
 def test_withdrawn_stall_request_changes_nothing():
     gu, _ = workloads.tiny_moe_layer(seed=4)
     lib = mxq.load()
