@@ -84,8 +84,10 @@ cudaError_t launch_global_scale(const uint16_t *x, int64_t n_groups, int64_t nb,
 // with S2IN, given by the caller (s2_in): then a scale that is negative or
 // not finite sets MXQ_DEV_INVALID_SCALE, and a non-finite element, found
 // through its block amax, sets MXQ_DEV_NONFINITE_INPUT.
+// Four CTAs per SM (64 registers, a few values spilled): 6 % faster on the
+// full-size gate_up stack with given scales than two CTAs at 96 registers.
 template <bool FOUR_SIX, bool S2IN>
-__global__ void __launch_bounds__(kNvThreads)
+__global__ void __launch_bounds__(kNvThreads, 4)
 nvfp4_quant_kernel(const uint4 *__restrict__ x, int64_t n_groups, int64_t nb,
                    const uint32_t *__restrict__ amax_bits, const float *__restrict__ s2_in,
                    uint2 *__restrict__ codes,
