@@ -133,10 +133,11 @@ __device__ __noinline__ void weighted_search_exact(const uint32_t (&w)[8], const
     }
 }
 
-// Three CTAs per SM (80 registers, a few spilled values): the occupancy
-// pays more than the spills cost (8.28 against 9.41 ms per full-size layer
-// at two CTAs and 128 registers).
-__global__ void __launch_bounds__(kNvThreads, 3)
+// Four CTAs per SM (64 registers, some values spilled to an L1 that shared
+// memory does not crowd): the occupancy pays more than the spills cost
+// (7.76 against 8.16 ms per full-size layer at three CTAs and 80 registers,
+// 9.41 ms at two CTAs and 128 registers).
+__global__ void __launch_bounds__(kNvThreads, 4)
 nvfp4_weighted_kernel(const uint4 *__restrict__ x, int64_t n_groups, int64_t nb,
                       const uint32_t *__restrict__ amax_bits, const float *__restrict__ h,
                       int64_t h_stride, uint32_t cb, uint2 *__restrict__ codes,
