@@ -1107,6 +1107,13 @@ def main():
                    "fraction_of_8tbs_nominal": value / 8000.0,
                    "call_ms": dict(zip(["quantize_gate_up", "quantize_down", "verify_gate_up",
                                         "verify_down"], call_ms)),
+                   # algorithmic GB/s of every call of the step and its fraction of the peak
+                   "call_gbs": {k: {"gbs": by / (t * 1e-3) / 1e9, "frac": by / (t * 1e-3) / 1e9 / peak}
+                                for k, by, t in zip(["quantize_gate_up", "quantize_down", "verify_gate_up",
+                                                     "verify_down"],
+                                                    [gu_elems * Q_BYTES, layer.dn.numel() * Q_BYTES,
+                                                     gu_elems * V_BYTES, layer.dn.numel() * V_BYTES],
+                                                    call_ms)},
                    "quality": quality},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
