@@ -280,3 +280,16 @@ def test_values_take_the_ieee_quotient_at_e2m1_ties(orc):
     got = [(int(b) >> (4 * h)) & 0xF for b in c.reshape(-1)[8:16] for h in (0, 1)]
     assert got == list(want)
     assert got[:8] == [7, 0, 2, 2, 4, 4, 6, 6]           # 6, then every tie at its even code
+
+
+def test_groups_and_tensors_without_elements(orc):
+    """A group with no elements has amax 0, so s2 = 0 and no block; a tensor
+    with no elements has both verifier sums 0 and a relative error of 0."""
+    for shape in ((3, 0, 32), (2, 8, 0), (0, 4, 16)):
+        codes, scales, s2, m4 = orc.quantize_nvfp4(np.zeros(shape, np.uint16), mode=1)
+        assert s2.shape == (shape[0],) and np.all(s2 == 0)
+        assert codes.size == 0 and scales.size == 0 and m4.size == 0
+    err, ref = orc.dequant_relerr(np.zeros((3, 0, 32), np.uint16), np.zeros(1, np.uint8),
+                                     np.zeros(1, np.uint8), np.ones(3, np.float32), "nvfp4", 3, 0, 32)
+    assert np.all(err == 0) and np.all(ref == 0)
+    assert np.all(np.asarray(orc.relerr_from_sums(err, ref)) == 0)
