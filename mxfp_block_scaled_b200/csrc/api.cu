@@ -216,6 +216,10 @@ mxq_status mxq_quantize_nvfp4(const uint16_t *x, int64_t n_groups, int64_t rows,
     else    // one group that fits the SMs' shared memory: one grid, one read
         e = launch_nvfp4_grid(x, nb, mode == MXQ_SCALE_FOUR_SIX, codes, scales, sl, s2, mbits, m4_count, status,
                               amax_bits, slots, stream);
+    // a context that may use fewer SMs than the device has (a shared or
+    // partitioned GPU) cannot hold the one-CTA-per-SM grid: two passes instead
+    if (e == cudaErrorCooperativeLaunchTooLarge)
+        e = cudaErrorNotSupported;
     if (e == cudaSuccess)
         return MXQ_OK;
     if (e != cudaErrorNotSupported)
