@@ -69,9 +69,16 @@ def measured_peak():
 
 
 def kernel_source_sha():
+    """Hash of the single-pass quantizer's source: its part of nvfp4.cu (from
+    the argument struct to its launch function) and the headers it uses, so
+    that edits to the other kernels of that file leave the record valid."""
     h = hashlib.sha256()
-    for f in ("nvfp4.cu", "nvfp4_block.cuh", "mxq_device.cuh"):
-        with open(os.path.join(ROOT, "mxfp_block_scaled_b200", "csrc", f), "rb") as fh:
+    csrc = os.path.join(ROOT, "mxfp_block_scaled_b200", "csrc")
+    with open(os.path.join(csrc, "nvfp4.cu"), "rb") as fh:
+        src = fh.read()
+    h.update(src[src.index(b"struct FusedArgs {"):src.index(b"cudaError_t launch_nvfp4_quant(")])
+    for f in ("nvfp4_block.cuh", "mxq_device.cuh", "mxq_internal.h"):
+        with open(os.path.join(csrc, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
