@@ -881,7 +881,7 @@ cudaError_t launch_nvfp4_small(const uint16_t *x, int64_t nb, int four_six, uint
 
 // ---------------------------------------------------------------------------
 // One group too large for a cluster whose blocks still fit the SMs' shared
-// memory (an activation tile of about 800 to 7000 tokens of 2048 values):
+// memory (an activation tile of about 800 to 8000 tokens of 2048 values):
 // a cooperative grid of one CTA per SM (all resident at once).  Each CTA
 // brings its share into shared memory with bulk copies issued together (the
 // whole share in flight), reduces its amax piece by piece as the pieces
